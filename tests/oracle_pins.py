@@ -1,0 +1,310 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+Each check_* function raises AssertionError when the oracle disagrees with a
+closed form, a brute-force sum, a textbook special case or an invariant that
+the pages and the mathematics fix.  The checks look up every oracle function
+through the module object at call time, so tests/test_oracle_mutants.py can
+plant a mistake in the oracle and verify that at least one check fails.
+
+Sources are cited by page title and section:
+[GBLA] SANA-Video 2.0 summary (paper.rainbus.top), prerequisites, "Gated
+       Bilinear Linear Attention" (read-out formula).
+[LA]   same page, prerequisites, "Linear Attention" (state S = sum v (beta k)^T).
+[V1]   SANA-Video notes (papernotes.org), key design 1 (RoPE(ReLU(x)),
+       numerator only, positive denominator).
+[BLK]  same notes, key design 2 (block-causal running sums).
+"""
+import math
+
+import numpy as np
+
+import oracle.gla_oracle as O
+from gated_bidirectional_linear_b200 import workloads
+
+EPS_N = 1e-6  # RMSNorm epsilon of the spec
+
+
+def _close(got, want, tol, what):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    err = np.max(np.abs(got - want) / np.maximum(np.abs(want), 1e-300 + np.abs(want).max()))
+    assert err <= tol, f"{what}: rel err {err:.3e} > {tol:.1e}\n got={got}\nwant={want}"
+
+
+def _rms_scale(x):
+    return 1.0 / math.sqrt(sum(e * e for e in x) / len(x) + EPS_N)
+
+
+def _inputs_f64(wl):
+    return workloads.as_f64(workloads.make_inputs(wl))
+
+
+# ---------------------------------------------------------------- closed forms
+
+def check_single_token_closed_form():
+    """N = 1 at position 0 (no rotation).  S = v (beta k_pls)^T, so
+    pre = v beta c / (c + eps) with c = k_pls . q_pls ([LA], [GBLA]).
+    q = (1,1,1,1): q_pls = q / sqrt(1 + e_n).  k = (2,-2,2,-2): ReLU keeps
+    (2,0,2,0) / sqrt(4 + e_n).  c = 4 / (sqrt(4+e_n) sqrt(1+e_n))."""
+    eps = 1e-3
+    q = np.array([1.0, 1.0, 1.0, 1.0])
+    k = np.array([2.0, -2.0, 2.0, -2.0])
+    v = np.array([1.0, 2.0, 3.0, 4.0])
+    beta = 0.5
+    g = np.array([0.0, math.log(3.0), -math.log(3.0), 0.0])     # sigma = .5 .75 .25 .5
+    c = 4.0 / (math.sqrt(4.0 + EPS_N) * math.sqrt(1.0 + EPS_N))
+    s = beta * c / (c + eps)
+    x = [0.5 * 1.0 * s, 0.75 * 2.0 * s, 0.25 * 3.0 * s, 0.5 * 4.0 * s]
+    out_want = [e * _rms_scale(x) for e in x]
+    shp = (1, 1, 1, 4)
+    r = O.forward(q.reshape(shp), k.reshape(shp), v.reshape(shp), np.full((1, 1, 1), beta),
+                  g.reshape(shp), 1, 1, 1, 10000.0, eps)
+    _close(r["x"].ravel(), x, 1e-12, "N=1 gated read-out")
+    _close(r["out"].ravel(), out_want, 1e-12, "N=1 output")
+    _close(r["den"].ravel(), [c + eps], 1e-12, "N=1 denominator")
+
+
+def _two_token_case():
+    """Two tokens on the time axis (T=2, H=W=1), d = 2: one rotation pair with
+    frequency theta^0 = 1, so token 1 is rotated by exactly 1 rad.
+
+    k0 = (1, 0):  k_pls0 = (a, 0),            a = 1/sqrt(0.5 + e_n)
+    k1 = (-1, 1): k_pls1 = (0, b),            b = 1/sqrt(1 + e_n)
+                  k_til1 = (-b sin1, b cos1)  (rotation after the ReLU)
+    q0 = (0, 2):  q_pls0 = q_til0 = (0, c2),  c2 = 2/sqrt(2 + e_n)
+    q1 = (3, 1):  q_pls1 = (3e, e),           e = 1/sqrt(5 + e_n)
+                  q_til1 = (3e cos1 - e sin1, 3e sin1 + e cos1)
+    Dot products: k_til0.q_til0 = 0, k_til1.q_til0 = b c2 cos1,
+                  k_til0.q_til1 = a e (3 cos1 - sin1), k_til1.q_til1 = b e.
+    Denominators (no rotation): den0 = b c2 + eps, den1 = 3 a e + b e + eps.
+    """
+    eps = 1e-2
+    s1, c1 = math.sin(1.0), math.cos(1.0)
+    a = 1.0 / math.sqrt(0.5 + EPS_N)
+    b = 1.0 / math.sqrt(1.0 + EPS_N)
+    c2 = 2.0 / math.sqrt(2.0 + EPS_N)
+    e = 1.0 / math.sqrt(5.0 + EPS_N)
+    v0, v1 = np.array([1.0, -1.0]), np.array([2.0, 0.5])
+    be0, be1 = 0.5, 0.25
+    pre0 = v1 * be1 * (b * c2 * c1) / (b * c2 + eps)
+    pre1 = (v0 * be0 * (a * e * (3 * c1 - s1)) + v1 * be1 * (b * e)) / (3 * a * e + b * e + eps)
+    sig0 = np.array([0.5, 0.75])                      # g0 = (0, ln 3)
+    sig1 = np.array([0.25, 0.5])                      # g1 = (-ln 3, 0)
+    x0, x1 = sig0 * pre0, sig1 * pre1
+    want = dict(
+        den=[b * c2 + eps, 3 * a * e + b * e + eps],
+        pre=np.stack([pre0, pre1]),
+        out=np.stack([x0 * _rms_scale(x0), x1 * _rms_scale(x1)]),
+    )
+    q = np.array([[0.0, 2.0], [3.0, 1.0]]).reshape(1, 2, 1, 2)
+    k = np.array([[1.0, 0.0], [-1.0, 1.0]]).reshape(1, 2, 1, 2)
+    v = np.stack([v0, v1]).reshape(1, 2, 1, 2)
+    beta = np.array([be0, be1]).reshape(1, 2, 1)
+    g = np.array([[0.0, math.log(3.0)], [-math.log(3.0), 0.0]]).reshape(1, 2, 1, 2)
+    return (q, k, v, beta, g, 2, 1, 1, 10000.0, eps), want
+
+
+def check_two_token_closed_form():
+    args, want = _two_token_case()
+    r = O.forward(*args)
+    _close(r["den"].ravel(), want["den"], 1e-12, "N=2 denominators")
+    _close(r["pre"].reshape(2, 2), want["pre"], 1e-12, "N=2 pre-gate read-out")
+    _close(r["out"].reshape(2, 2), want["out"], 1e-12, "N=2 output")
+
+
+def check_two_token_bruteforce_closed_form():
+    args, want = _two_token_case()
+    r = O.forward_bruteforce(*args)
+    _close(r["pre"].reshape(2, 2), want["pre"], 1e-12, "N=2 brute force")
+    _close(r["out"].reshape(2, 2), want["out"], 1e-12, "N=2 brute-force output")
+
+
+# ------------------------------------------------------------ RoPE (the spec)
+
+def check_rope_split():
+    assert O.rope_pair_split(128) == (22, 21, 21)
+    assert O.rope_pair_split(32) == (6, 5, 5)
+    assert O.rope_pair_split(6) == (1, 1, 1)
+    assert O.rope_pair_split(2) == (1, 0, 0)
+
+
+def check_rope_axis_order():
+    """d = 6: pair 0 turns with t, pair 1 with h, pair 2 with w, each at
+    frequency 1.  Token (t,h,w) = (1,2,3) of a 2x3x4 grid is n = 23; the unit
+    vector (1,0,1,0,1,0) goes to (cos1, sin1, cos2, sin2, cos3, sin3)."""
+    ang = O.rope_angles(6, 2, 3, 4, 10000.0)
+    x = np.zeros((1, 24, 1, 6))
+    x[..., 0::2] = 1.0
+    y = O.rope_rotate(x, ang)[0, 23, 0]
+    want = [math.cos(1), math.sin(1), math.cos(2), math.sin(2), math.cos(3), math.sin(3)]
+    _close(y, want, 1e-15, "RoPE axis order")
+
+
+def check_rope_frequencies():
+    """d = 12, theta = 1e4: two pairs per axis with frequencies 1 and
+    theta^(-1/2) = 0.01.  Token (t,h,w) = (0,0,3) turns only the w pairs
+    (channels 8..11) by 3 and 0.03 rad; (x0, x1) = (0, 1) -> (-sin, cos)."""
+    ang = O.rope_angles(12, 1, 1, 4, 10000.0)
+    x = np.zeros((1, 4, 1, 12))
+    x[..., 1::2] = 1.0
+    y = O.rope_rotate(x, ang)[0, 3, 0]
+    want = [0, 1, 0, 1, 0, 1, 0, 1, -math.sin(3), math.cos(3), -math.sin(0.03), math.cos(0.03)]
+    assert np.max(np.abs(y - np.array(want))) < 1e-15, f"RoPE frequencies: {y}"
+
+
+def check_rope_complex_form():
+    """Rotating pair (x0, x1) equals multiplying x0 + i x1 by exp(i angle)."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((1, 40, 2, 32))
+    ang = O.rope_angles(32, 2, 4, 5, 500.0, t0=3)
+    y = O.rope_rotate(x, ang)
+    zc = (x[..., 0::2] + 1j * x[..., 1::2]) * np.exp(1j * ang)[None, :, None, :]
+    assert np.max(np.abs(y[..., 0::2] - zc.real)) < 1e-13
+    assert np.max(np.abs(y[..., 1::2] - zc.imag)) < 1e-13
+
+
+# ------------------------------------------------- brute force and invariants
+
+def check_factorised_equals_bruteforce():
+    """Tiny workload (1x2 heads, d=32, 2x4x4 grid, seed 0): the S/z form and
+    the O(N^2) pair sum agree to fp64 rounding, before and after gate/norm."""
+    wl = workloads.WORKLOADS["tiny"]
+    x = _inputs_f64(wl)
+    args = (x["q"], x["k"], x["v"], x["beta"], x["g"], wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+    f = O.forward(*args)
+    bf = O.forward_bruteforce(*args)
+    _close(f["pre"], bf["pre"], 1e-12, "factorised vs brute force (pre)")
+    _close(f["out"], bf["out"], 1e-12, "factorised vs brute force (out)")
+
+
+def check_bruteforce_odd_grid():
+    """Brute force vs factorised on a ragged grid and a small head dim."""
+    rng = np.random.default_rng(11)
+    T, H, W, d = 3, 2, 5, 12
+    N = T * H * W
+    q, k, v, g = (rng.standard_normal((2, N, 1, d)) for _ in range(4))
+    beta = rng.uniform(0.05, 0.95, (2, N, 1))
+    args = (q, k, v, beta, g, T, H, W, 50.0, 1e-4, 2)
+    f = O.forward(*args)
+    bf = O.forward_bruteforce(*args)
+    _close(f["pre"], bf["pre"], 1e-12, "odd-grid brute force")
+
+
+def check_denominator_positive():
+    """[V1]: without RoPE in the denominator every pair term k_pls_n . q_pls_j
+    is >= 0, so den >= eps for every token.  Negative control: the same terms
+    taken over rotated features are negative for some pairs, so a rotated
+    denominator would carry no such guarantee."""
+    rng = np.random.default_rng(3)
+    T, H, W, d = 4, 6, 6, 32
+    N = T * H * W
+    q, k, v, g = (rng.standard_normal((1, N, 2, d)) for _ in range(4))
+    beta = rng.uniform(0.0, 1.0, (1, N, 2))
+    eps = 1e-6
+    r = O.forward(q, k, v, beta, g, T, H, W, 10000.0, eps)
+    assert np.all(r["den"] >= eps), "denominator below eps"
+    ang = O.rope_angles(d, T, H, W, 10000.0)
+    q_pls, q_til = O.feature_maps(q, ang)
+    k_pls, k_til = O.feature_maps(k, ang)
+    assert np.all(np.einsum("bnhc,bjhc->bnjh", k_pls, q_pls) >= 0.0)
+    assert np.any(np.einsum("bnhc,bjhc->bnjh", k_til, q_til) < 0.0), \
+        "negative control: every rotated pair term stayed non-negative"
+
+
+def check_time_shift_invariance():
+    """Dot products of rotated features depend on position differences only,
+    and the denominator has no rotation, so a global time offset leaves the
+    bidirectional output unchanged."""
+    wl = workloads.WORKLOADS["tiny"]
+    x = _inputs_f64(wl)
+    args = (x["q"], x["k"], x["v"], x["beta"], x["g"], wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+    a = O.forward(*args, t0=0)
+    b = O.forward(*args, t0=7)
+    _close(b["out"], a["out"], 1e-11, "time-shift invariance")
+
+
+def check_rotation_preserves_norm():
+    wl = workloads.WORKLOADS["tiny"]
+    x = _inputs_f64(wl)
+    ang = O.rope_angles(wl.head_dim, wl.T, wl.H, wl.W, wl.rope_theta)
+    q_pls, q_til = O.feature_maps(x["q"], ang)
+    assert np.allclose(np.linalg.norm(q_pls, axis=-1), np.linalg.norm(q_til, axis=-1),
+                       rtol=1e-13, atol=0)
+
+
+def check_plain_relu_linear_attention():
+    """RoPE off, beta = 1 and g = +30 (sigma = 1 - 9.4e-14): the operator is
+    plain ReLU linear attention on the normalised q/k ([V1]: SANA's ReLU
+    linear attention), written here in textbook matrix form
+        phi(Q) (phi(K)^T V) / (phi(Q) (phi(K)^T 1) + eps),
+    followed by the output RMSNorm."""
+    wl = workloads.WORKLOADS["tiny"]
+    x = _inputs_f64(wl)
+    beta = np.ones_like(x["beta"])
+    g = np.full_like(x["g"], 30.0)
+    r = O.forward(x["q"], x["k"], x["v"], beta, g, wl.T, wl.H, wl.W, 0.0, wl.eps)
+    for h in range(wl.heads):
+        Q, K, V = (x[n][0, :, h, :] for n in ("q", "k", "v"))
+        nq = np.maximum(Q / np.sqrt((Q ** 2).mean(1, keepdims=True) + EPS_N), 0)
+        nk = np.maximum(K / np.sqrt((K ** 2).mean(1, keepdims=True) + EPS_N), 0)
+        num = nq @ (nk.T @ V)
+        den = nq @ (nk.T @ np.ones((nk.shape[0], 1))) + wl.eps
+        la = num / den
+        want = la / np.sqrt((la ** 2).mean(1, keepdims=True) + EPS_N)
+        _close(r["out"][0, :, h, :], want, 1e-11, "plain ReLU linear attention")
+
+
+def check_gate_and_write_scale_invariance():
+    """A uniform write gate c_b and a uniform output gate sigma scale every
+    gated read-out x_j by the same constant c, and the output RMSNorm (gate
+    before the norm) then gives out_b = out_a sqrt((ms + e_n) / (ms + e_n/c^2))
+    with ms = mean(x_a^2) per token.  Every output row has RMS
+    sqrt(ms / (ms + e_n))."""
+    wl = workloads.WORKLOADS["tiny"]
+    x = _inputs_f64(wl)
+    base = (x["q"], x["k"], x["v"])
+    geo = (wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+    a = O.forward(*base, np.full_like(x["beta"], 0.3), np.zeros_like(x["g"]), *geo)
+    b = O.forward(*base, np.full_like(x["beta"], 0.9), np.full_like(x["g"], 30.0), *geo)
+    c = (0.9 / 0.3) * (1.0 / (1.0 + math.exp(-30.0))) / 0.5
+    _close(b["x"], c * a["x"], 1e-12, "uniform gates scale x")
+    ms = np.mean(a["x"] ** 2, axis=-1, keepdims=True)
+    _close(b["out"], a["out"] * np.sqrt((ms + EPS_N) / (ms + EPS_N / c ** 2)), 1e-12,
+           "output norm after uniform gates")
+    rms_out = np.sqrt(np.mean(a["out"] ** 2, axis=-1, keepdims=True))
+    _close(rms_out, np.sqrt(ms / (ms + EPS_N)), 1e-12, "output row RMS")
+
+
+# ---------------------------------------------------------------- block-causal
+
+def _blk_inputs():
+    rng = np.random.default_rng(21)
+    nb, T_blk, H, W, d = 4, 2, 3, 4, 8
+    N = nb * T_blk * H * W
+    q, k, v, g = (rng.standard_normal((1, N, 2, d)) for _ in range(4))
+    beta = rng.uniform(0.0, 1.0, (1, N, 2))
+    return (q, k, v, beta, g), (nb, T_blk, H, W)
+
+
+def check_block_causal_bruteforce():
+    """[BLK]: the carried (S, z) form equals the prefix-masked pair sum where
+    token j sees token n iff block(n) <= block(j)."""
+    (q, k, v, beta, g), (nb, T_blk, H, W) = _blk_inputs()
+    c = O.block_causal_forward(q, k, v, beta, g, nb, T_blk, H, W, 10000.0, 1e-5)
+    bf = O.block_causal_bruteforce(q, k, v, beta, g, nb, T_blk, H, W, 10000.0, 1e-5)
+    _close(c["out"], bf["out"], 1e-11, "block-causal vs prefix-masked brute force")
+
+
+def check_block_causal_final_state():
+    """After the last block the carried state is the full-sequence state and
+    the last block's output is the bidirectional output of those tokens."""
+    (q, k, v, beta, g), (nb, T_blk, H, W) = _blk_inputs()
+    c = O.block_causal_forward(q, k, v, beta, g, nb, T_blk, H, W, 10000.0, 1e-5)
+    f = O.forward(q, k, v, beta, g, nb * T_blk, H, W, 10000.0, 1e-5)
+    _close(c["S"], f["S"], 1e-12, "final block state")
+    _close(c["z"], f["z"], 1e-12, "final key sum")
+    L = T_blk * H * W
+    _close(c["out"][:, -L:], f["out"][:, -L:], 1e-11, "last block = bidirectional")
+
+
+ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

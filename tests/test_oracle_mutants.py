@@ -1,0 +1,117 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and verify that the
+pins catch every one of them: each mutant must fail at least one check."""
+import numpy as np
+import pytest
+
+import oracle.gla_oracle as O
+import oracle_pins
+
+_orig = {name: getattr(O, name) for name in dir(O) if not name.startswith("_")}
+
+
+def _rotate_backwards(x, angles):
+    return _orig["rope_rotate"](x, -angles)
+
+
+def _rope_before_relu(x, angles):
+    x_hat = O.rms_normalize(x)
+    if angles is None:
+        p = O.relu(x_hat)
+        return p, p
+    return O.relu(x_hat), O.relu(_orig["rope_rotate"](x_hat, angles))
+
+
+def _beta_in_keysum(k_til, k_pls, v, beta):
+    S, _ = _orig["state_and_keysum"](k_til, k_pls, v, beta)
+    return S, (beta[..., None] * k_pls).sum(axis=1)
+
+
+def _transposed_state(k_til, k_pls, v, beta):
+    S, z = _orig["state_and_keysum"](k_til, k_pls, v, beta)
+    return np.swapaxes(S, -1, -2), z
+
+
+def _rotated_keysum(k_til, k_pls, v, beta):
+    return _orig["state_and_keysum"](k_til, k_til, v, beta)
+
+
+def _gate_after_norm(S, z, q_pls, q_til, g, eps):
+    r = _orig["read_out"](S, z, q_pls, q_til, g, eps)
+    r["out"] = O.sigmoid(g) * O.rms_normalize(r["pre"])
+    return r
+
+
+def _no_eps_in_den(S, z, q_pls, q_til, g, eps):
+    return _orig["read_out"](S, z, q_pls, q_til, g, 0.0)
+
+
+def _unnormalised_keysum(k_til, k_pls, v, beta):
+    return _orig["state_and_keysum"](k_til, np.abs(k_pls) * 1.5, v, beta)
+
+
+def _rms_sum(x):
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + O.RMS_EPS)
+
+
+def _rms_no_eps(x):
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True))
+
+
+def _freq_doubled(d, T, H, W, rope_theta, t0=0):
+    return _orig["rope_angles"](d, T, H, W, rope_theta ** 2, t0)
+
+
+def _axes_swapped(T, H, W, t0=0):
+    t, h, w = _orig["token_positions"](T, H, W, t0)
+    return t, w, h
+
+
+def _no_time_offset(T, H, W, t0=0):
+    return _orig["token_positions"](T, H, W, 0)
+
+
+def _exclusive_block(S, z, q, k, v, beta, g, T_blk, H, W, t0, rope_theta, eps):
+    d = q.shape[-1]
+    angles = None if rope_theta <= 0 else O.rope_angles(d, T_blk, H, W, rope_theta, t0)
+    q_pls, q_til = O.feature_maps(q, angles)
+    k_pls, k_til = O.feature_maps(k, angles)
+    dS, dz = O.state_and_keysum(k_til, k_pls, v, beta)
+    r = O.read_out(S + 0.0, z + eps, q_pls, q_til, g, eps)   # reads the old state
+    r.update(S=S + dS, z=z + dz)
+    return r
+
+
+def _neg_sigmoid(x):
+    return 1.0 / (1.0 + np.exp(x))
+
+
+MUTANTS = {
+    "rope_backwards": ("rope_rotate", _rotate_backwards),
+    "rope_before_relu": ("feature_maps", _rope_before_relu),
+    "beta_in_keysum": ("state_and_keysum", _beta_in_keysum),
+    "state_transposed": ("state_and_keysum", _transposed_state),
+    "rotated_keysum": ("state_and_keysum", _rotated_keysum),
+    "gate_after_norm": ("read_out", _gate_after_norm),
+    "no_eps_in_den": ("read_out", _no_eps_in_den),
+    "keysum_wrong_features": ("state_and_keysum", _unnormalised_keysum),
+    "rmsnorm_sum": ("rms_normalize", _rms_sum),
+    "rmsnorm_no_eps": ("rms_normalize", _rms_no_eps),
+    "rope_freq_wrong": ("rope_angles", _freq_doubled),
+    "rope_axes_swapped": ("token_positions", _axes_swapped),
+    "rope_no_time_offset": ("token_positions", _no_time_offset),
+    "block_exclusive": ("block_causal_step", _exclusive_block),
+    "sigmoid_sign": ("sigmoid", _neg_sigmoid),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failed = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check()
+        except (AssertionError, FloatingPointError, ValueError):
+            failed.append(check.__name__)
+    assert failed, f"mutant {name} passed every pin"
