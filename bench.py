@@ -1,0 +1,352 @@
+"""Benchmark of gla_forward on one B200 per rank.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 720p] [--impl ours|reference]
+
+One step = one gla_forward call (state reduction, combine, read-out) over one
+batch of the workload's synthetic, seeded inputs already resident in HBM.
+Under torchrun each rank runs its own copy of the workload on its own GPU
+(independent layers, no collective on the data path: weak scaling); the timed
+region is bracketed by a barrier and a device synchronisation on both sides
+and the reported time is the maximum over ranks.  Rank 0 prints one JSON line.
+
+The inputs of one 720p step are 755 MB (q, k, v, g, beta read + out written),
+six times the 126 MB L2, so no step can hit in L2 from the previous one; no
+extra flush is done.
+
+--impl reference times the fp64 CPU oracle (oracle/gla_oracle.py) as it
+stands, on the host cores, on a bounded sample of the same workload per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from gated_bidirectional_linear_b200 import workloads  # noqa: E402
+
+METRIC = "gla_forward tokens/s (20x128 heads, 14720 tok) and HBM GB/s vs B200 peak"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["common.cuh", "ptx.cuh", "tc.cuh", "combine.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="720p", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(wl):
+    return {
+        "workload": (f"{wl.name}: batch {wl.batch}, {wl.heads} heads x {wl.head_dim}, grid "
+                     f"{wl.T}x{wl.H}x{wl.W} ({wl.tokens} tokens), {wl.dtype}, "
+                     f"q/k/v/g ~ N(0,1), beta = sigmoid(N(0,1)), theta {wl.rope_theta:g}, "
+                     f"eps {wl.eps:g}, seed {wl.seed}"),
+        "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+        "grid": [wl.T, wl.H, wl.W], "tokens_per_step": wl.batch * wl.tokens,
+        "l2": (f"no flush: {wl.alg_bytes_per_call() / 1e6:.0f} MB moved per step vs "
+               "126 MB L2"),
+    }
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def source_sha():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "gated_bidirectional_linear_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, workload):
+    """ncu DRAM bytes per launch from profiles/traffic.json, if it was taken on
+    the current kernel sources; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            doc = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = doc.get(kernel, {}).get(workload)
+    if not ent or ent.get("source_sha") != source_sha():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockMonitor:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                maxes.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sms)) if sms else None,
+                "sm_max_mhz": max(maxes) if maxes else None,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def cpu_oracle_rate(wl, seconds):
+    """The oracle, as it stands, on whole heads of the workload until
+    `seconds` have passed: returns (tokens/s of the full layer, heads, s)."""
+    import oracle.gla_oracle as O
+    from threadpoolctl import threadpool_info
+    t_used, th = 0.0, 0
+    heads = 0
+    for idx in range(wl.batch * wl.heads):
+        x = workloads.as_f64(workloads.draw(1, wl.tokens, 1, wl.head_dim, wl.dtype, 1000 + idx))
+        t0 = time.perf_counter()
+        O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], wl.T, wl.H, wl.W,
+                  wl.rope_theta, wl.eps)
+        t_used += time.perf_counter() - t0
+        th += wl.tokens
+        heads += 1
+        if t_used >= seconds:
+            break
+    blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+    cores = blas[0] if blas else 1
+    return th / t_used / wl.heads, heads, t_used, cores
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    import oracle.gla_oracle as O
+    from threadpoolctl import threadpool_info
+    # One step = the oracle on one head over the first two latent frames.
+    T_s = min(2, wl.T)
+    n_s = T_s * wl.H * wl.W
+    x = workloads.as_f64(workloads.draw(1, n_s, 1, wl.head_dim, wl.dtype, 77))
+    for _ in range(args.warmup):
+        O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T_s, wl.H, wl.W, wl.rope_theta, wl.eps)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T_s, wl.H, wl.W, wl.rope_theta, wl.eps)
+    dt = time.perf_counter() - t0
+    value = n_s * args.steps / dt / wl.heads
+    blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+    cores = blas[0] if blas else 1
+    sample = (f"per step: oracle.forward on 1 of {wl.batch * wl.heads} heads, first {T_s} "
+              f"frames ({n_s} tokens); tokens/s of the full layer = token-heads/s / {wl.heads}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    wl = workloads.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+
+    from gated_bidirectional_linear_b200 import gla
+    gla.lib()  # fail loudly if the library is missing
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    inp = workloads.make_inputs(wl, seed=wl.seed + rank)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    B, N, Hh, hd = d["q"].shape
+    code = gla.GLA_DTYPE_BF16 if d["q"].dtype == torch.bfloat16 else gla.GLA_DTYPE_F32
+    out = torch.empty_like(d["q"])
+    ws = gla.alloc_workspace(gla.gla_forward_workspace_size(B, Hh, hd, wl.T, wl.H, wl.W, code), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events):
+        gla.gla_forward_timed(d["q"], d["k"], d["v"], d["beta"], d["g"], wl.T, wl.H, wl.W,
+                              events, wl.rope_theta, wl.eps, out=out, workspace=ws,
+                              stream=stream)
+
+    none4 = [None] * 4
+    for _ in range(max(args.warmup, 3)):
+        step(none4)
+    torch.cuda.synchronize(dev)
+    assert gla.gla_get_device_status(stream) == gla.GLA_OK
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockMonitor(local) as mon:
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist:
+            dist.barrier()
+    status = gla.gla_get_device_status(stream)
+    if status != gla.GLA_OK:
+        raise RuntimeError(f"device status after the timed region: {gla.status_string(status)}")
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if dist:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    k_state = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    k_comb = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    k_apply = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+
+    # ---- end to end: host buffers through gla_forward_host, copies timed.
+    pinned = {k: v.pin_memory() for k, v in inp.items()}
+    out_h = torch.empty_like(pinned["q"]).pin_memory()
+    arena = gla.alloc_workspace(gla.gla_forward_host_arena_size(B, Hh, hd, wl.T, wl.H, wl.W, code), dev)
+    e2e_steps = max(3, min(args.steps, 200))
+    for _ in range(3):
+        gla.gla_forward_host(pinned["q"], pinned["k"], pinned["v"], pinned["beta"], pinned["g"],
+                             wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, out=out_h, arena=arena,
+                             stream=stream)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        gla.gla_forward_host(pinned["q"], pinned["k"], pinned["v"], pinned["beta"], pinned["g"],
+                             wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, out=out_h, arena=arena,
+                             stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    th = B * N * Hh
+    esz = 2 if code == gla.GLA_DTYPE_BF16 else 4
+    tokens_per_step = B * N
+    ms_per_step = elapsed_ms / args.steps
+    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    peak, peak_kind = measured_peaks()
+    apply_bytes = th * hd * esz * 3                # q, g read + out written
+    state_bytes = th * hd * esz * 2 + th * esz     # k, v, beta read
+    apply_gbs = apply_bytes / (k_apply * 1e-3) / 1e9
+    state_gbs = state_bytes / (k_state * 1e-3) / 1e9
+    step_gbs = wl.alg_bytes_per_call() / (ms_per_step * 1e-3) / 1e9
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            rate, heads, secs, cores = cpu_oracle_rate(wl, args.cpu_sample_seconds)
+            cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                   "sample": (f"oracle.forward on {heads} whole heads ({wl.tokens} tokens each) "
+                              f"of the {wl.name} workload, {secs:.1f} s; tokens/s of the full "
+                              f"layer = token-heads/s / {wl.heads}; cores = BLAS threads")}
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(workload_config(wl), parallelism=f"replicas x{world}"),
+            "hbm_gbs_per_gpu": step_gbs,
+            "roofline": {"bound": "hbm", "kernel": "tc_apply_kernel", "achieved": apply_gbs,
+                         "peak": peak, "unit": "GB/s", "frac": apply_gbs / peak,
+                         "peak_kind": peak_kind,
+                         "traffic": traffic_for("tc_apply_kernel", wl.name),
+                         "alg_bytes_per_launch": apply_bytes, "ms_per_launch": k_apply},
+            "kernels_ms": {"tc_state_kernel": k_state, "combine_kernel": k_comb,
+                           "tc_apply_kernel": k_apply},
+            "kernels_gbs": {"tc_state_kernel": state_gbs, "tc_apply_kernel": apply_gbs},
+            "step_frac_of_peak": step_gbs / peak,
+            "e2e": {"value": e2e_value, "unit": "tokens/s",
+                    "h2d_bytes_per_step": th * hd * esz * 4 + th * esz,
+                    "d2h_bytes_per_step": th * hd * esz, "steps": e2e_steps},
+            "gpu_launches": 3 * args.steps,
+            "clocks": mon.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,186 @@
+// Shared device/host definitions of libgla: problem geometry, the split-N
+// partition of the state reduction, and the per-CTA 3D-RoPE cos/sin table.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gla {
+
+constexpr float kRmsEps = 1e-6f;     // RMSNorm epsilon of q, k and the output
+constexpr int kMaxStateCtas = 512;   // upper bound of the state-kernel grid
+
+// Library-wide device error word (bit 0: a bounded wait timed out).
+__device__ unsigned int g_device_error;
+
+enum : unsigned { kErrTimeout = 1u };
+
+// ----------------------------------------------------------------- geometry
+
+struct Geom {
+  int B, Hh, d;          // batch, heads, head dim
+  int T, H, W, N;        // latent grid of this call, N = T*H*W
+  int t0;                // time position of local frame 0
+  int pt, ph, pw;        // rotation pairs per axis (t, h, w)
+  int rope_on;           // 0: identity rotation
+  float theta;           // RoPE base
+  float eps;             // denominator epsilon
+};
+
+__host__ __device__ inline void rope_split(int d, int* pt, int* ph, int* pw) {
+  int p = d / 2;
+  int hw = p / 3;
+  *pt = p - 2 * hw;
+  *ph = hw;
+  *pw = hw;
+}
+
+// --------------------------------------------------------------- partition
+//
+// The state reduction walks "items" = (head bh, tile i) in the order
+// item = bh * tiles_per_head + i.  CTA c of G owns the items
+// [floor(c*I/G), floor((c+1)*I/G)).  The partial of CTA c for head bh is
+// stored in slot c + bh: along the item order (c, bh) never decreases in either
+// component and changes in at least one at every segment boundary, so slots
+// are unique and at most G + BH are used.
+
+struct Partition {
+  int BH;              // batch * heads
+  int tile;            // tokens per item
+  int tiles_per_head;  // ceil(N / tile)
+  long long items;     // BH * tiles_per_head
+  int grid;            // G
+};
+
+__host__ __device__ inline long long part_begin(const Partition& p, int c) {
+  return (long long)c * p.items / p.grid;
+}
+
+// CTA owning item w: the largest c with floor(c*I/G) <= w.
+__host__ __device__ inline int part_cta_of(const Partition& p, long long w) {
+  return (int)(((w + 1) * (long long)p.grid - 1) / p.items);
+}
+
+inline Partition make_partition(int BH, int N, int tile, int max_grid) {
+  Partition p;
+  p.BH = BH;
+  p.tile = tile;
+  p.tiles_per_head = (N + tile - 1) / tile;
+  p.items = (long long)BH * p.tiles_per_head;
+  long long g = p.items < max_grid ? p.items : max_grid;
+  if (g > kMaxStateCtas) g = kMaxStateCtas;
+  if (g < 1) g = 1;
+  p.grid = (int)g;
+  return p;
+}
+
+// --------------------------------------------------------------- RoPE table
+//
+// Each CTA keeps cos/sin of the rotations it needs in shared memory, as float2
+// (cos, sin) entries:
+//   time axis:   pt pairs x Lt frames   (frames t_lo .. t_lo+Lt-1, wrapping
+//                                        modulo T when the CTA's tokens cross
+//                                        from the end of one head's sequence
+//                                        to the start of the next)
+//   height axis: ph pairs x H
+//   width axis:  pw pairs x W
+// Angles are formed and evaluated in double precision, then rounded to fp32.
+
+struct RopeWindow {
+  int t_lo;   // first local frame held
+  int Lt;     // frames held (<= T)
+};
+
+__host__ __device__ inline int rope_table_entries(const Geom& g, int Lt) {
+  return g.pt * Lt + g.ph * g.H + g.pw * g.W;
+}
+
+// Frames touched by the items [w0, w1] (inclusive) of a partition.
+__host__ __device__ inline RopeWindow rope_window(const Geom& g, const Partition& p,
+                                                  long long w0, long long w1) {
+  const int HW = g.H * g.W;
+  const int bh0 = (int)(w0 / p.tiles_per_head), bh1 = (int)(w1 / p.tiles_per_head);
+  const int n0 = (int)(w0 % p.tiles_per_head) * p.tile;
+  int n1 = (int)(w1 % p.tiles_per_head) * p.tile + p.tile - 1;
+  if (n1 > g.N - 1) n1 = g.N - 1;
+  const int f0 = n0 / HW, f1 = n1 / HW;
+  RopeWindow r;
+  if (bh0 == bh1 && f1 >= f0) {
+    r.t_lo = f0;
+    r.Lt = f1 - f0 + 1;
+  } else if (bh1 == bh0 + 1 && f1 < f0) {
+    r.t_lo = f0;                      // f0 .. T-1, then 0 .. f1
+    r.Lt = (g.T - f0) + (f1 + 1);
+  } else {
+    r.t_lo = 0;
+    r.Lt = g.T;
+  }
+  if (r.Lt > g.T) { r.t_lo = 0; r.Lt = g.T; }
+  return r;
+}
+
+__device__ inline void rope_build(float2* tab, const Geom& g, RopeWindow win, int tid,
+                                  int nthr) {
+  if (!g.rope_on) return;
+  const int nt = g.pt * win.Lt, nh = g.ph * g.H, nw = g.pw * g.W;
+  const double log_theta = log((double)g.theta);
+  for (int e = tid; e < nt + nh + nw; e += nthr) {
+    int i, p;
+    double pos;
+    if (e < nt) {
+      i = e / win.Lt;
+      p = g.pt;
+      int f = win.t_lo + e % win.Lt;
+      if (f >= g.T) f -= g.T;
+      pos = (double)(g.t0 + f);
+    } else if (e < nt + nh) {
+      i = (e - nt) / g.H;
+      p = g.ph;
+      pos = (double)((e - nt) % g.H);
+    } else {
+      i = (e - nt - nh) / g.W;
+      p = g.pw;
+      pos = (double)((e - nt - nh) % g.W);
+    }
+    const double ang = pos * exp(-((double)i / (double)p) * log_theta);
+    double s, c;
+    sincos(ang, &s, &c);
+    tab[e] = make_float2((float)c, (float)s);
+  }
+}
+
+// Index of the (cos, sin) entry of rotation pair `pr` (0 .. d/2-1) for a token
+// at local frame f, row hh, column ww.
+__device__ inline int rope_index(const Geom& g, RopeWindow win, int pr, int f, int hh,
+                                 int ww) {
+  if (pr < g.pt) {
+    int tl = f - win.t_lo;
+    if (tl < 0) tl += g.T;
+    return pr * win.Lt + tl;
+  }
+  if (pr < g.pt + g.ph) return g.pt * win.Lt + (pr - g.pt) * g.H + hh;
+  return g.pt * win.Lt + g.ph * g.H + (pr - g.pt - g.ph) * g.W + ww;
+}
+
+// ------------------------------------------------------------------ dtypes
+
+template <typename T> __device__ inline float to_f32(T x);
+template <> __device__ inline float to_f32<float>(float x) { return x; }
+template <> __device__ inline float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T> __device__ inline T from_f32(float x);
+template <> __device__ inline float from_f32<float>(float x) { return x; }
+template <> __device__ inline __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ inline float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+}  // namespace gla

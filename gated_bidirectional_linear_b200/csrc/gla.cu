@@ -1,0 +1,440 @@
+// libgla: host side of the C ABI declared in include/gla.h.
+//
+// One translation unit: the kernels live in the included .cuh files.
+// Host code validates arguments, plans the split-N partition, carves the
+// caller's workspace and launches the kernels on the caller's stream.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "gla.h"
+
+#include "common.cuh"
+#include "combine.cuh"
+#include "simt.cuh"
+#include "tc.cuh"
+
+using namespace gla;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxZParts = kStTW;   // z partials per state slot (tensor path)
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct WsLayout {
+  size_t part_S, part_z, S, z, S_img, S_rs, total;
+  int slots;
+};
+
+// Workspace carve-up; independent of the GPU (uses the maximum grid).
+WsLayout ws_layout(int BH, int d, bool own_state) {
+  WsLayout L;
+  L.slots = kMaxStateCtas + BH;
+  size_t off = 0;
+  L.part_S = off; off = align_up(off + (size_t)L.slots * d * d * 4, kAlign);
+  L.part_z = off; off = align_up(off + (size_t)L.slots * kMaxZParts * d * 4, kAlign);
+  if (own_state) {
+    L.S = off; off = align_up(off + (size_t)BH * d * d * 4, kAlign);
+    L.z = off; off = align_up(off + (size_t)BH * d * 4, kAlign);
+  } else {
+    L.S = L.z = 0;
+  }
+  L.S_img = off;
+  if (d == 128) off = align_up(off + (size_t)BH * d * d * 2, kAlign);
+  L.S_rs = off;
+  if (d == 128) off = align_up(off + (size_t)BH * d * 4, kAlign);
+  L.total = off;
+  return L;
+}
+
+bool dims_ok(int batch, int heads, int head_dim, int T, int H, int W) {
+  if (batch <= 0 || heads <= 0 || T <= 0 || H <= 0 || W <= 0) return false;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return false;
+  const long long N = (long long)T * H * W;
+  const long long elems = (long long)batch * N * heads * head_dim;
+  if (N > (1LL << 30) || elems > (1LL << 40)) return false;
+  return true;
+}
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return -1;
+  if (dev >= 0 && dev < 64) cache[dev] = sms;
+  return sms;
+}
+
+Geom make_geom(int batch, int heads, int head_dim, int T, int H, int W, int t0,
+               float rope_theta, float eps) {
+  Geom g;
+  g.B = batch; g.Hh = heads; g.d = head_dim;
+  g.T = T; g.H = H; g.W = W; g.N = T * H * W;
+  g.t0 = t0;
+  rope_split(head_dim, &g.pt, &g.ph, &g.pw);
+  g.rope_on = rope_theta > 0.f ? 1 : 0;
+  g.theta = rope_theta;
+  g.eps = eps;
+  return g;
+}
+
+// Largest per-CTA RoPE table (entries) over the CTAs of a partition.
+int max_table_entries(const Geom& g, const Partition& p) {
+  if (!g.rope_on) return 1;
+  int mx = 1;
+  for (int c = 0; c < p.grid; ++c) {
+    const long long w0 = part_begin(p, c), w1 = part_begin(p, c + 1) - 1;
+    const RopeWindow win = rope_window(g, p, w0, w1);
+    const int e = rope_table_entries(g, win.Lt);
+    if (e > mx) mx = e;
+  }
+  return mx;
+}
+
+int tile_table_entries(const Geom& g, int tile) {
+  if (!g.rope_on) return 1;
+  Partition tp;
+  tp.BH = 1; tp.tile = tile; tp.tiles_per_head = (g.N + tile - 1) / tile;
+  tp.items = tp.tiles_per_head; tp.grid = (int)tp.items;
+  return max_table_entries(g, tp);
+}
+
+struct Call {
+  Geom g;
+  int dtype;
+  int path;          // resolved: GLA_PATH_SIMT or GLA_PATH_TENSOR
+  const void *q, *k, *v, *beta, *gate;
+  void* out;
+  float* S;          // combined state (workspace or caller's carried state)
+  float* z;
+  bool carry;        // S/z hold a carried state to add to
+  unsigned char* ws;
+  WsLayout L;
+  cudaStream_t stream;
+  float *S_dbg, *z_dbg, *den_dbg, *x_dbg;
+  void* const* events;   // optional [4] cudaEvent_t records around the kernels
+};
+
+inline cudaError_t mark(const Call& c, int i) {
+  if (!c.events || !c.events[i]) return cudaSuccess;
+  return cudaEventRecord(static_cast<cudaEvent_t>(c.events[i]), c.stream);
+}
+
+int resolve_path(int requested, int dtype, int d) {
+  const bool tensor_ok = dtype == GLA_DTYPE_BF16 && d == 128;
+  if (requested == GLA_PATH_AUTO) return tensor_ok ? GLA_PATH_TENSOR : GLA_PATH_SIMT;
+  if (requested == GLA_PATH_SIMT) return GLA_PATH_SIMT;
+  if (requested == GLA_PATH_TENSOR) return tensor_ok ? GLA_PATH_TENSOR : -1;
+  return -1;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int D, typename Tin>
+gla_status run_simt(const Call& c) {
+  const Geom& g = c.g;
+  const int sms = device_sm_count();
+  if (sms <= 0) return GLA_ERR_CUDA;
+  const Partition part = make_partition(g.B * g.Hh, g.N, kSimtTile, 2 * sms);
+
+  SimtStateParams sp;
+  sp.g = g; sp.part = part;
+  sp.k = c.k; sp.v = c.v; sp.beta = c.beta;
+  sp.part_S = reinterpret_cast<float*>(c.ws + c.L.part_S);
+  sp.part_z = reinterpret_cast<float*>(c.ws + c.L.part_z);
+  sp.tab_entries = max_table_entries(g, part);
+  const size_t smem_state = (size_t)(2 * kSimtTile * D + 8 * D) * 4 + (size_t)sp.tab_entries * 8;
+  if (smem_state > 200 * 1024) return GLA_ERR_UNSUPPORTED;
+  if (set_smem(simt_state_kernel<D, Tin>, smem_state) != cudaSuccess) return GLA_ERR_CUDA;
+  if (mark(c, 0) != cudaSuccess) return GLA_ERR_CUDA;
+  simt_state_kernel<D, Tin><<<part.grid, kSimtThreads, smem_state, c.stream>>>(sp);
+  if (cudaGetLastError() != cudaSuccess || mark(c, 1) != cudaSuccess) return GLA_ERR_CUDA;
+
+  CombineParams cp;
+  cp.part = part; cp.d = D; cp.zparts = 1;
+  cp.part_S = sp.part_S; cp.part_z = sp.part_z;
+  cp.S_in = c.carry ? c.S : nullptr;
+  cp.z_in = c.carry ? c.z : nullptr;
+  cp.S_out = c.S; cp.z_out = c.z;
+  cp.S_img = nullptr; cp.S_rs = nullptr;
+  dim3 cgrid((D * D + kCombineElems - 1) / kCombineElems, g.B * g.Hh);
+  combine_kernel<<<cgrid, kCombineThreads, 0, c.stream>>>(cp);
+  if (cudaGetLastError() != cudaSuccess || mark(c, 2) != cudaSuccess) return GLA_ERR_CUDA;
+
+  SimtApplyParams ap;
+  ap.g = g; ap.q = c.q; ap.gate = c.gate; ap.S = c.S; ap.z = c.z; ap.out = c.out;
+  ap.den_out = c.den_dbg; ap.x_out = c.x_dbg;
+  ap.tab_entries = tile_table_entries(g, kSimtApplyTile);
+  const size_t smem_apply = (size_t)(D * D + D + 8 * D) * 4 + (size_t)ap.tab_entries * 8;
+  if (smem_apply > 200 * 1024) return GLA_ERR_UNSUPPORTED;
+  if (set_smem(simt_apply_kernel<D, Tin>, smem_apply) != cudaSuccess) return GLA_ERR_CUDA;
+  dim3 agrid((g.N + kSimtApplyTile - 1) / kSimtApplyTile, g.B * g.Hh);
+  simt_apply_kernel<D, Tin><<<agrid, kSimtThreads, smem_apply, c.stream>>>(ap);
+  if (cudaGetLastError() != cudaSuccess || mark(c, 3) != cudaSuccess) return GLA_ERR_CUDA;
+  return GLA_OK;
+}
+
+template <typename Tin>
+gla_status run_simt_dtype(const Call& c) {
+  switch (c.g.d) {
+    case 32: return run_simt<32, Tin>(c);
+    case 64: return run_simt<64, Tin>(c);
+    case 128: return run_simt<128, Tin>(c);
+  }
+  return GLA_ERR_UNSUPPORTED;
+}
+
+gla_status run_call(Call& c) {
+  gla_status st;
+  if (c.path == GLA_PATH_TENSOR) {
+    st = run_tensor(c.g, c.q, c.k, c.v, c.beta, c.gate, c.out, c.S, c.z, c.carry,
+                    reinterpret_cast<float*>(c.ws + c.L.part_S),
+                    reinterpret_cast<float*>(c.ws + c.L.part_z),
+                    reinterpret_cast<__half*>(c.ws + c.L.S_img),
+                    reinterpret_cast<float*>(c.ws + c.L.S_rs), c.den_dbg, c.x_dbg,
+                    device_sm_count(), c.stream, c.events);
+  } else {
+    st = c.dtype == GLA_DTYPE_F32 ? run_simt_dtype<float>(c)
+                                  : run_simt_dtype<__nv_bfloat16>(c);
+  }
+  if (st != GLA_OK) return st;
+  const size_t dd = (size_t)c.g.B * c.g.Hh * c.g.d * c.g.d;
+  const size_t dz = (size_t)c.g.B * c.g.Hh * c.g.d;
+  if (c.S_dbg && cudaMemcpyAsync(c.S_dbg, c.S, dd * 4, cudaMemcpyDeviceToDevice, c.stream) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  if (c.z_dbg && cudaMemcpyAsync(c.z_dbg, c.z, dz * 4, cudaMemcpyDeviceToDevice, c.stream) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  return GLA_OK;
+}
+
+gla_status forward_common(const void* q, const void* k, const void* v, const void* beta,
+                          const void* g, int batch, int heads, int head_dim, int T, int H,
+                          int W, float rope_theta, float eps, int dtype, void* out,
+                          void* workspace, size_t workspace_bytes, void* stream, int path,
+                          float* S_out, float* z_out, float* den_out, float* x_out,
+                          void* const* events = nullptr) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W)) return GLA_ERR_INVALID_ARG;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+  if (!(eps > 0.f) || !isfinite(eps) || !isfinite(rope_theta)) return GLA_ERR_INVALID_ARG;
+  const void* ptrs[6] = {q, k, v, beta, g, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
+  const int resolved = resolve_path(path, dtype, head_dim);
+  if (resolved < 0) return GLA_ERR_UNSUPPORTED;
+  const WsLayout L = ws_layout(batch * heads, head_dim, true);
+  if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < L.total)
+    return GLA_ERR_WORKSPACE;
+  Call c;
+  c.g = make_geom(batch, heads, head_dim, T, H, W, 0, rope_theta, eps);
+  c.dtype = dtype; c.path = resolved;
+  c.q = q; c.k = k; c.v = v; c.beta = beta; c.gate = g; c.out = out;
+  c.ws = static_cast<unsigned char*>(workspace);
+  c.L = L;
+  c.S = reinterpret_cast<float*>(c.ws + L.S);
+  c.z = reinterpret_cast<float*>(c.ws + L.z);
+  c.carry = false;
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.S_dbg = S_out; c.z_dbg = z_out; c.den_dbg = den_out; c.x_dbg = x_out;
+  c.events = events;
+  return run_call(c);
+}
+
+}  // namespace
+
+extern "C" {
+
+int gla_version(void) { return 100; }
+
+const char* gla_status_string(int status) {
+  switch (status) {
+    case GLA_OK: return "GLA_OK";
+    case GLA_ERR_INVALID_ARG: return "GLA_ERR_INVALID_ARG: invalid argument";
+    case GLA_ERR_UNSUPPORTED: return "GLA_ERR_UNSUPPORTED: unsupported configuration";
+    case GLA_ERR_WORKSPACE: return "GLA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case GLA_ERR_CUDA: return "GLA_ERR_CUDA: CUDA runtime error";
+    case GLA_ERR_TIMEOUT: return "GLA_ERR_TIMEOUT: a device-side wait timed out";
+  }
+  return "unknown gla_status";
+}
+
+size_t gla_forward_workspace_size(int batch, int heads, int head_dim, int T, int H, int W,
+                                  int dtype) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W)) return 0;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return 0;
+  return ws_layout(batch * heads, head_dim, true).total;
+}
+
+size_t gla_block_causal_workspace_size(int batch, int heads, int head_dim, int T_blk, int H,
+                                       int W, int dtype) {
+  if (!dims_ok(batch, heads, head_dim, T_blk, H, W)) return 0;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return 0;
+  return ws_layout(batch * heads, head_dim, false).total;
+}
+
+gla_status gla_forward(const void* q, const void* k, const void* v, const void* beta,
+                       const void* g, int batch, int heads, int head_dim, int T, int H, int W,
+                       float rope_theta, float eps, int dtype, void* out, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return forward_common(q, k, v, beta, g, batch, heads, head_dim, T, H, W, rope_theta, eps,
+                        dtype, out, workspace, workspace_bytes, stream, GLA_PATH_AUTO,
+                        nullptr, nullptr, nullptr, nullptr);
+}
+
+gla_status gla_forward_ex(const void* q, const void* k, const void* v, const void* beta,
+                          const void* g, int batch, int heads, int head_dim, int T, int H,
+                          int W, float rope_theta, float eps, int dtype, void* out,
+                          void* workspace, size_t workspace_bytes, void* stream, int path) {
+  return forward_common(q, k, v, beta, g, batch, heads, head_dim, T, H, W, rope_theta, eps,
+                        dtype, out, workspace, workspace_bytes, stream, path, nullptr,
+                        nullptr, nullptr, nullptr);
+}
+
+gla_status gla_forward_debug(const void* q, const void* k, const void* v, const void* beta,
+                             const void* g, int batch, int heads, int head_dim, int T, int H,
+                             int W, float rope_theta, float eps, int dtype, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream, int path,
+                             float* S_out, float* z_out, float* den_out, float* x_out) {
+  return forward_common(q, k, v, beta, g, batch, heads, head_dim, T, H, W, rope_theta, eps,
+                        dtype, out, workspace, workspace_bytes, stream, path, S_out, z_out,
+                        den_out, x_out);
+}
+
+gla_status gla_forward_timed(const void* q, const void* k, const void* v, const void* beta,
+                             const void* g, int batch, int heads, int head_dim, int T, int H,
+                             int W, float rope_theta, float eps, int dtype, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream, int path,
+                             void* const* events) {
+  return forward_common(q, k, v, beta, g, batch, heads, head_dim, T, H, W, rope_theta, eps,
+                        dtype, out, workspace, workspace_bytes, stream, path, nullptr,
+                        nullptr, nullptr, nullptr, events);
+}
+
+gla_status gla_block_causal_step_ex(float* state, float* z, const void* q, const void* k,
+                                    const void* v, const void* beta, const void* g,
+                                    int batch, int heads, int head_dim, int T_blk, int H,
+                                    int W, int t0, float rope_theta, float eps, int dtype,
+                                    void* out, void* workspace, size_t workspace_bytes,
+                                    void* stream, int path) {
+  if (!dims_ok(batch, heads, head_dim, T_blk, H, W) || t0 < 0) return GLA_ERR_INVALID_ARG;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+  if (!(eps > 0.f) || !isfinite(eps) || !isfinite(rope_theta)) return GLA_ERR_INVALID_ARG;
+  const void* ptrs[8] = {state, z, q, k, v, beta, g, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
+  const int resolved = resolve_path(path, dtype, head_dim);
+  if (resolved < 0) return GLA_ERR_UNSUPPORTED;
+  const WsLayout L = ws_layout(batch * heads, head_dim, false);
+  if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < L.total)
+    return GLA_ERR_WORKSPACE;
+  Call c;
+  c.g = make_geom(batch, heads, head_dim, T_blk, H, W, t0, rope_theta, eps);
+  c.dtype = dtype; c.path = resolved;
+  c.q = q; c.k = k; c.v = v; c.beta = beta; c.gate = g; c.out = out;
+  c.ws = static_cast<unsigned char*>(workspace);
+  c.L = L;
+  c.S = state; c.z = z; c.carry = true;
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.S_dbg = c.z_dbg = c.den_dbg = c.x_dbg = nullptr;
+  c.events = nullptr;
+  return run_call(c);
+}
+
+gla_status gla_block_causal_step(float* state, float* z, const void* q, const void* k,
+                                 const void* v, const void* beta, const void* g, int batch,
+                                 int heads, int head_dim, int T_blk, int H, int W, int t0,
+                                 float rope_theta, float eps, int dtype, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return gla_block_causal_step_ex(state, z, q, k, v, beta, g, batch, heads, head_dim, T_blk,
+                                  H, W, t0, rope_theta, eps, dtype, out, workspace,
+                                  workspace_bytes, stream, GLA_PATH_AUTO);
+}
+
+size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, int T, int H, int W,
+                                   int dtype) {
+  const size_t ws = gla_forward_workspace_size(batch, heads, head_dim, T, H, W, dtype);
+  if (!ws) return 0;
+  const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
+  const size_t th = (size_t)batch * T * H * W * heads;
+  return 5 * align_up(th * head_dim * esz, kAlign) + align_up(th * esz, kAlign) + ws;
+}
+
+gla_status gla_forward_host(const void* q_h, const void* k_h, const void* v_h,
+                            const void* beta_h, const void* g_h, int batch, int heads,
+                            int head_dim, int T, int H, int W, float rope_theta, float eps,
+                            int dtype, void* out_h, void* arena, size_t arena_bytes,
+                            void* stream) {
+  const size_t need = gla_forward_host_arena_size(batch, heads, head_dim, T, H, W, dtype);
+  if (!need) return GLA_ERR_INVALID_ARG;
+  const void* hp[6] = {q_h, k_h, v_h, beta_h, g_h, out_h};
+  for (const void* p : hp)
+    if (!p) return GLA_ERR_INVALID_ARG;
+  if (!arena || ((uintptr_t)arena % kAlign) != 0 || arena_bytes < need) return GLA_ERR_WORKSPACE;
+  const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
+  const size_t th = (size_t)batch * T * H * W * heads;
+  const size_t big = th * head_dim * esz, small = th * esz;
+  unsigned char* a = static_cast<unsigned char*>(arena);
+  unsigned char* dq = a;
+  unsigned char* dk = dq + align_up(big, kAlign);
+  unsigned char* dv = dk + align_up(big, kAlign);
+  unsigned char* dg = dv + align_up(big, kAlign);
+  unsigned char* dout = dg + align_up(big, kAlign);
+  unsigned char* dbeta = dout + align_up(big, kAlign);
+  unsigned char* dws = dbeta + align_up(small, kAlign);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(dq, q_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dg, g_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dbeta, beta_h, small, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  const gla_status st = gla_forward(dq, dk, dv, dbeta, dg, batch, heads, head_dim, T, H, W,
+                                    rope_theta, eps, dtype, dout, dws,
+                                    arena_bytes - (size_t)(dws - a), stream);
+  if (st != GLA_OK) return st;
+  if (cudaMemcpyAsync(out_h, dout, big, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  return GLA_OK;
+}
+
+gla_status gla_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  unsigned int w = 0;
+  if (cudaMemcpyFromSymbol(&w, g_device_error, sizeof(w)) != cudaSuccess) return GLA_ERR_CUDA;
+  if (w) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+      return GLA_ERR_CUDA;
+    return GLA_ERR_TIMEOUT;
+  }
+  return GLA_OK;
+}
+
+gla_status gla_plan(int batch, int heads, int head_dim, int T, int H, int W, int dtype,
+                    int path, int num_sms, int* grid, int* tile_tokens, int* path_used) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W) || num_sms <= 0) return GLA_ERR_INVALID_ARG;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+  if (!grid || !tile_tokens || !path_used) return GLA_ERR_INVALID_ARG;
+  const int resolved = resolve_path(path, dtype, head_dim);
+  if (resolved < 0) return GLA_ERR_UNSUPPORTED;
+  const int N = T * H * W;
+  Partition p = resolved == GLA_PATH_TENSOR
+                    ? make_partition(batch * heads, N, kTcTile, num_sms)
+                    : make_partition(batch * heads, N, kSimtTile, 2 * num_sms);
+  *grid = p.grid;
+  *tile_tokens = p.tile;
+  *path_used = resolved;
+  return GLA_OK;
+}
+
+}  // extern "C"

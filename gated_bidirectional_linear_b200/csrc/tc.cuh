@@ -1,0 +1,856 @@
+// Tensor-core path (bf16 inputs, head dim 128) for sm_100a.
+//
+//   tc_state_kernel  persistent split-N state reduction.  TMA streams 128-token
+//                    tiles of k and v (128-byte swizzle) into a 3-stage ring;
+//                    transform warps apply RMSNorm, ReLU, 3D RoPE and beta to
+//                    the k tile in place (bf16) while summing z in registers;
+//                    one thread issues tcgen05.mma  S += V^T (beta K_til)  with
+//                    both operands MN-major, accumulating in TMEM; epilogue warps
+//                    drain each finished head segment to its partial slot.
+//   combine_kernel   (combine.cuh) fixed-order sum of the partials, plus the
+//                    swizzled bf16 image of S.
+//   tc_apply_kernel  persistent read-out.  TMA streams q and g tiles; transform
+//                    warps turn q into q_til (fp16, in place) and the
+//                    denominator z.q_pls + eps; one thread issues
+//                    tcgen05.mma  U = Q_til S^T  into a double-buffered TMEM
+//                    accumulator; epilogue warps (one token row per thread)
+//                    apply sigmoid(g) / den, the output RMSNorm, round to bf16
+//                    into the g tile and TMA-store it.
+//
+// All waits are bounded (mbar_wait): on expiry the kernel records a timeout in
+// the device error word, stops issuing work, drains its copies and frees TMEM.
+#pragma once
+
+#include "combine.cuh"
+#include "ptx.cuh"
+
+namespace gla {
+
+constexpr int kTcTile = 128;                 // tokens per tile
+constexpr uint32_t kBox = 16384;             // one TMA box: 128 rows x 128 bytes
+constexpr uint32_t kTileBytes = 2 * kBox;    // 128 tokens x 128 channels bf16
+constexpr int kPosBits = 11;                 // packed (t, h, w) offsets, < 2048 each
+
+// --------------------------------------------------------------- state kernel
+
+constexpr int kStStages = 3;
+constexpr int kStTW = 8;                     // transform warps
+constexpr int kStTW0 = 6;                    // first transform warp
+constexpr int kStEW0 = 2;                    // epilogue warps 2..5
+constexpr int kStThreads = (kStTW0 + kStTW) * 32;
+constexpr int kStRowsPerPass = kStTW * 4;
+
+struct TcStateSmem {
+  static constexpr uint32_t K = 0;
+  static constexpr uint32_t V = kStStages * kTileBytes;
+  static constexpr uint32_t BAR = 2 * kStStages * kTileBytes;         // barriers
+  static constexpr uint32_t NBAR = 3 * kStStages + 5;
+  static constexpr uint32_t MISC = BAR + NBAR * 8;                     // tmem base, abort
+  static constexpr uint32_t TAB = (MISC + 16 + 15) & ~15u;              // RoPE table
+};
+
+struct TcStateParams {
+  Geom g;
+  Partition part;
+  const __nv_bfloat16* beta;
+  float* part_S;
+  float* part_z;
+  int tab_entries;
+};
+
+__device__ __forceinline__ bool seg_first(const Partition& p, long long w, long long wb) {
+  return w == wb || (w % p.tiles_per_head) == 0;
+}
+__device__ __forceinline__ bool seg_last(const Partition& p, long long w, long long we) {
+  return w == we - 1 || ((w + 1) % p.tiles_per_head) == 0;
+}
+
+// Per-lane rotation-pair lookup: lane j of a row group handles channels
+// 16j .. 16j+15, i.e. pairs 8j .. 8j+7.
+struct PairInfo {
+  int base[8];
+  int shift[8];
+};
+
+__device__ __forceinline__ void pair_info(const Geom& g, RopeWindow win, int j, PairInfo& pi) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int p = 8 * j + i;
+    if (p < g.pt) {
+      pi.base[i] = p * win.Lt;
+      pi.shift[i] = 0;
+    } else if (p < g.pt + g.ph) {
+      pi.base[i] = g.pt * win.Lt + (p - g.pt) * g.H;
+      pi.shift[i] = kPosBits;
+    } else {
+      pi.base[i] = g.pt * win.Lt + g.ph * g.H + (p - g.pt - g.ph) * g.W;
+      pi.shift[i] = 2 * kPosBits;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t packed_pos(const Geom& g, RopeWindow win, int n) {
+  const int HW = g.H * g.W;
+  const int f = n / HW;
+  const int rem = n - f * HW;
+  const int hh = rem / g.W;
+  const int ww = rem - hh * g.W;
+  int tl = f - win.t_lo;
+  if (tl < 0) tl += g.T;
+  return (uint32_t)tl | ((uint32_t)hh << kPosBits) | ((uint32_t)ww << (2 * kPosBits));
+}
+
+// Shared-memory addresses of the two 16-byte chunks a lane owns in row r of a
+// 128x128 bf16 tile stored as two 128-byte-swizzled boxes.
+__device__ __forceinline__ void lane_chunks(uint32_t tile, int r, int j, uint32_t& a0,
+                                            uint32_t& a1) {
+  const uint32_t row = tile + (uint32_t)(j >> 2) * kBox + (uint32_t)r * 128u;
+  const uint32_t c0 = (uint32_t)((2 * j) & 7);
+  a0 = row + (((c0) ^ (uint32_t)(r & 7)) << 4);
+  a1 = row + (((c0 + 1) ^ (uint32_t)(r & 7)) << 4);
+}
+
+__device__ __forceinline__ void unpack16(uint4 a, uint4 b, float (&x)[16]) {
+  x[0] = bf_lo(a.x); x[1] = bf_hi(a.x); x[2] = bf_lo(a.y); x[3] = bf_hi(a.y);
+  x[4] = bf_lo(a.z); x[5] = bf_hi(a.z); x[6] = bf_lo(a.w); x[7] = bf_hi(a.w);
+  x[8] = bf_lo(b.x); x[9] = bf_hi(b.x); x[10] = bf_lo(b.y); x[11] = bf_hi(b.y);
+  x[12] = bf_lo(b.z); x[13] = bf_hi(b.z); x[14] = bf_lo(b.w); x[15] = bf_hi(b.w);
+}
+
+// RMSNorm + ReLU of one row shared by the 8 lanes of a row group.
+__device__ __forceinline__ void norm_relu16(float (&x)[16]) {
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) ss = fmaf(x[i], x[i], ss);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+  const float rstd = rsqrtf(ss * (1.f / 128.f) + kRmsEps);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x[i] = fmaxf(x[i] * rstd, 0.f);
+}
+
+// y = scale * RoPE(x) for the lane's 8 pairs, packed to bf16 (or fp16).
+template <bool kHalf>
+__device__ __forceinline__ void rope_pack16(const Geom& g, const float2* tab, const PairInfo& pi,
+                                            uint32_t opk, const float (&x)[16], float scale,
+                                            uint4& o0, uint4& o1) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float y0 = x[2 * i], y1 = x[2 * i + 1];
+    if (g.rope_on) {
+      const float2 cs = tab[pi.base[i] + (int)((opk >> pi.shift[i]) & ((1u << kPosBits) - 1))];
+      const float r0 = fmaf(-y1, cs.y, y0 * cs.x);
+      const float r1 = fmaf(y1, cs.x, y0 * cs.y);
+      y0 = r0;
+      y1 = r1;
+    }
+    w[i] = kHalf ? pack_f16(y0 * scale, y1 * scale) : pack_bf16(y0 * scale, y1 * scale);
+  }
+  o0 = make_uint4(w[0], w[1], w[2], w[3]);
+  o1 = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+__global__ void __launch_bounds__(kStThreads, 1)
+    tc_state_kernel(const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, TcStateParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + TcStateSmem::BAR);
+  uint64_t* full = bars;
+  uint64_t* kready = bars + kStStages;
+  uint64_t* empty = bars + 2 * kStStages;
+  uint64_t* accfull = bars + 3 * kStStages;
+  uint64_t* accempty = accfull + 2;
+  uint64_t* drain = accempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + TcStateSmem::MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + TcStateSmem::MISC + 4);
+  float2* tab = reinterpret_cast<float2*>(sm + TcStateSmem::TAB);
+
+  const Geom& g = p.g;
+  const Partition& part = p.part;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const long long wb = part_begin(part, c), we = part_begin(part, c + 1);
+  const RopeWindow win = rope_window(g, part, wb, we - 1);
+  const int tph = part.tiles_per_head;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&kready[s], kStTW);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accfull[a], 1);
+      mbar_init(&accempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 256);
+    tmem_relinquish();
+  }
+  if (warp >= kStTW0) rope_build(tab, g, win, threadIdx.x - kStTW0 * 32, kStTW * 32);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      long long it = 0;
+      int issued = 0;
+      for (long long w = wb; w < we; ++w, ++it) {
+        const int s = (int)(it % kStStages);
+        const uint32_t ph = (uint32_t)((it / kStStages) & 1);
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
+        const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
+        const int n0 = (int)(w % tph) * kTcTile;
+        mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
+        unsigned char* kt = sm + TcStateSmem::K + s * kTileBytes;
+        unsigned char* vt = sm + TcStateSmem::V + s * kTileBytes;
+        tma_load_3d(kt, &tmK, &full[s], h * 128, n0, b, pol);
+        tma_load_3d(kt + kBox, &tmK, &full[s], h * 128 + 64, n0, b, pol);
+        tma_load_3d(vt, &tmV, &full[s], h * 128, n0, b, pol);
+        tma_load_3d(vt + kBox, &tmV, &full[s], h * 128 + 64, n0, b, pol);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // Let every load in flight land before shared memory is released.
+        long long first = it - (issued < kStStages ? issued : kStStages);
+        for (long long i2 = first; i2 < it; ++i2) {
+          int dummy = 0;
+          mbar_wait(&full[i2 % kStStages], (uint32_t)((i2 / kStStages) & 1),
+                    reinterpret_cast<volatile int*>(&dummy));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, 128, true, true);
+      long long it = 0;
+      int seg = 0;
+      for (long long w = wb; w < we; ++w, ++it) {
+        const int s = (int)(it % kStStages);
+        const uint32_t ph = (uint32_t)((it / kStStages) & 1);
+        const bool first = seg_first(part, w, wb), last = seg_last(part, w, we);
+        const int ab = seg & 1;
+        if (first && !mbar_wait(&accempty[ab], (uint32_t)(((seg >> 1) & 1) ^ 1), abort_flag))
+          break;
+        if (!mbar_wait(&kready[s], ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t kt = sbase + TcStateSmem::K + s * kTileBytes;
+        const uint32_t vt = sbase + TcStateSmem::V + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = sdesc_sw128(vt + kk * 2048, kBox, 1024);
+          const uint64_t bd = sdesc_sw128(kt + kk * 2048, kBox, 1024);
+          umma_f16kind(tmem + ab * 128, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
+        }
+        umma_commit(&empty[s]);
+        if (last) {
+          umma_commit(&accfull[ab]);
+          ++seg;
+        }
+      }
+      // Every MMA issued above has completed before TMEM is released.
+      umma_commit(drain);
+      int dummy = 0;
+      mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy));
+    }
+  } else if (warp < kStTW0) {
+    // ------------------------------------------------ epilogue: S partials
+    const int q4 = warp & 3;
+    const int a = q4 * 32 + lane;
+    int seg = 0;
+    for (long long w = wb; w < we; ++w) {
+      if (!seg_last(part, w, we)) continue;
+      const int bh = (int)(w / tph);
+      const int ab = seg & 1;
+      if (!mbar_wait(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag)) break;
+      tc_fence_after();
+      float* dst = p.part_S + ((size_t)c + bh) * 128 * 128 + (size_t)a * 128;
+#pragma unroll 1
+      for (int cb = 0; cb < 4; ++cb) {
+        float r[32];
+        tmem_ld32(tmem + (uint32_t)(ab * 128 + cb * 32) + ((uint32_t)(q4 * 32) << 16), r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + cb * 32 + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[ab]);
+      ++seg;
+    }
+  } else {
+    // ------------------------------------------- transform warps: k -> beta k_til
+    const int tw = warp - kStTW0;
+    const int rg = lane >> 3, j = lane & 7;
+    PairInfo pi;
+    pair_info(g, win, j, pi);
+    const uint64_t pol_beta = policy_evict_last();
+    float zacc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) zacc[i] = 0.f;
+    long long it = 0;
+    bool ok = true;
+    for (long long w = wb; w < we && ok; ++w, ++it) {
+      const int s = (int)(it % kStStages);
+      const uint32_t ph = (uint32_t)((it / kStStages) & 1);
+      const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
+      const int n0 = (int)(w % tph) * kTcTile;
+      constexpr int kPasses = (kTcTile + kStRowsPerPass - 1) / kStRowsPerPass;
+      float be[kPasses];
+#pragma unroll
+      for (int ps = 0; ps < kPasses; ++ps) {
+        const int n = n0 + ps * kStRowsPerPass + tw * 4 + rg;
+        be[ps] = 0.f;
+        if (n < g.N) {
+          const uint16_t raw = ld_u16_policy(p.beta + ((size_t)b * g.N + n) * g.Hh + h, pol_beta);
+          be[ps] = __uint_as_float((uint32_t)raw << 16);
+        }
+      }
+      if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
+      const uint32_t kt = sbase + TcStateSmem::K + s * kTileBytes;
+#pragma unroll
+      for (int ps = 0; ps < kPasses; ++ps) {
+        const int r = ps * kStRowsPerPass + tw * 4 + rg;
+        const int n = n0 + r;
+        uint32_t a0, a1;
+        lane_chunks(kt, r, j, a0, a1);
+        float x[16];
+        unpack16(lds128(a0), lds128(a1), x);
+        norm_relu16(x);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) zacc[i] += x[i];
+        const uint32_t opk = packed_pos(g, win, n < g.N ? n : n0);
+        uint4 o0, o1;
+        rope_pack16<false>(g, tab, pi, opk, x, be[ps], o0, o1);
+        sts128(a0, o0);
+        sts128(a1, o1);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&kready[s]);
+
+      if (seg_last(part, w, we)) {
+        // z of this head segment: sum the warp's four row groups, then store
+        // one partial per warp (the combine adds them in warp order).
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          zacc[i] += __shfl_xor_sync(0xffffffffu, zacc[i], 8);
+          zacc[i] += __shfl_xor_sync(0xffffffffu, zacc[i], 16);
+        }
+        if (rg == 0) {
+          float* zd = p.part_z + (((size_t)c + bh) * kStTW + tw) * 128 + 16 * j;
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(zd + i) = make_float4(zacc[i], zacc[i + 1], zacc[i + 2], zacc[i + 3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) zacc[i] = 0.f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// --------------------------------------------------------------- apply kernel
+
+constexpr int kApQ = 2;                      // q ring
+constexpr int kApG = 3;                      // g / out ring
+constexpr int kApAcc = 2;                    // TMEM accumulators
+constexpr int kApDen = kApQ + kApAcc;        // den ring
+constexpr int kApTW = 8;
+constexpr int kApTW0 = 3;                    // transform warps 3..10
+constexpr int kApEW0 = kApTW0 + kApTW;       // epilogue warps 11..18
+constexpr int kApEW = 4 * kApAcc;
+constexpr int kApThreads = (kApEW0 + kApEW) * 32;
+constexpr int kApRowsPerPass = kApTW * 4;
+
+struct TcApplySmem {
+  static constexpr uint32_t Q = 0;
+  static constexpr uint32_t G = kApQ * kTileBytes;
+  static constexpr uint32_t SIMG = G + kApG * kTileBytes;
+  static constexpr uint32_t Z = SIMG + kTileBytes;
+  static constexpr uint32_t RS = Z + 512;
+  static constexpr uint32_t DEN = RS + 512;                 // [kApDen][128] den per tile
+  static constexpr uint32_t RSR = DEN + kApDen * 512;       // [kApDen][128] row scales per tile
+  static constexpr uint32_t BAR = RSR + kApDen * 512;
+  static constexpr uint32_t NBAR = 3 * kApQ + 2 * kApG + 2 * kApAcc + 3;
+  static constexpr uint32_t MISC = BAR + NBAR * 8;
+  static constexpr uint32_t TAB = (MISC + 16 + 15) & ~15u;
+};
+
+struct TcApplyParams {
+  Geom g;
+  Partition part;
+  const __half* S_img;         // [BH][128*128] swizzled fp16 image of S (row-scaled)
+  const float* S_rs;           // [BH][128] inverse row scales of the image
+  const float* z;              // [BH][128]
+  float* den_out;              // optional
+  float* x_out;                // optional
+  int tab_entries;
+};
+
+template <bool kDebug>
+__global__ void __launch_bounds__(kApThreads, 1)
+    tc_apply_kernel(const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmG,
+                    const __grid_constant__ CUtensorMap tmO, TcApplyParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + TcApplySmem::BAR);
+  uint64_t* qfull = bars;
+  uint64_t* qready = qfull + kApQ;
+  uint64_t* qempty = qready + kApQ;
+  uint64_t* gfull = qempty + kApQ;
+  uint64_t* gempty = gfull + kApG;
+  uint64_t* accfull = gempty + kApG;
+  uint64_t* accempty = accfull + kApAcc;
+  uint64_t* sfull = accempty + kApAcc;
+  uint64_t* sfree = sfull + 1;
+  uint64_t* drain = sfree + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + TcApplySmem::MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + TcApplySmem::MISC + 4);
+  float* zs = reinterpret_cast<float*>(sm + TcApplySmem::Z);
+  const float* rs = reinterpret_cast<const float*>(sm + TcApplySmem::RS);
+  float* den_ring = reinterpret_cast<float*>(sm + TcApplySmem::DEN);
+  float* rs_ring = reinterpret_cast<float*>(sm + TcApplySmem::RSR);
+  float2* tab = reinterpret_cast<float2*>(sm + TcApplySmem::TAB);
+
+  const Geom& g = p.g;
+  const Partition& part = p.part;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const long long wb = part_begin(part, c), we = part_begin(part, c + 1);
+  const RopeWindow win = rope_window(g, part, wb, we - 1);
+  const int tph = part.tiles_per_head;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kApQ; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qready[s], kApTW);
+      mbar_init(&qempty[s], 1);
+    }
+    for (int s = 0; s < kApG; ++s) {
+      mbar_init(&gfull[s], 1);
+      mbar_init(&gempty[s], 1);
+    }
+    for (int a = 0; a < kApAcc; ++a) {
+      mbar_init(&accfull[a], 1);
+      mbar_init(&accempty[a], 4);
+    }
+    mbar_init(sfull, 1);
+    mbar_init(sfree, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 256);
+    tmem_relinquish();
+  }
+  if (warp >= kApTW0 && warp < kApEW0)
+    rope_build(tab, g, win, threadIdx.x - kApTW0 * 32, kApTW * 32);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == 0) {
+    // ------------------------------------------------- producer: S image + q
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      long long it = 0;
+      int seg = 0, issued = 0;
+      for (long long w = wb; w < we; ++w, ++it) {
+        const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
+        if (seg_first(part, w, wb)) {
+          if (!mbar_wait(sfree, (uint32_t)((seg & 1) ^ 1), abort_flag)) break;
+          mbar_arrive_expect_tx(sfull, kTileBytes + 1024);
+          bulk_load(sm + TcApplySmem::SIMG, p.S_img + (size_t)bh * 128 * 128, kTileBytes, sfull);
+          bulk_load(sm + TcApplySmem::Z, p.z + (size_t)bh * 128, 512, sfull);
+          bulk_load(sm + TcApplySmem::RS, p.S_rs + (size_t)bh * 128, 512, sfull);
+          ++seg;
+        }
+        const int s = (int)(it % kApQ);
+        const uint32_t ph = (uint32_t)((it / kApQ) & 1);
+        if (!mbar_wait(&qempty[s], ph ^ 1u, abort_flag)) break;
+        const int n0 = (int)(w % tph) * kTcTile;
+        mbar_arrive_expect_tx(&qfull[s], kTileBytes);
+        unsigned char* qt = sm + TcApplySmem::Q + s * kTileBytes;
+        tma_load_3d(qt, &tmQ, &qfull[s], h * 128, n0, b, pol);
+        tma_load_3d(qt + kBox, &tmQ, &qfull[s], h * 128 + 64, n0, b, pol);
+        ++issued;
+      }
+      if (*abort_flag) {
+        long long first = it - (issued < kApQ ? issued : kApQ);
+        for (long long i2 = first; i2 < it; ++i2) {
+          int dummy = 0;
+          mbar_wait(&qfull[i2 % kApQ], (uint32_t)((i2 / kApQ) & 1),
+                    reinterpret_cast<volatile int*>(&dummy));
+        }
+        int dummy = 0;
+        if (seg > 0) mbar_wait(sfull, (uint32_t)((seg - 1) & 1), reinterpret_cast<volatile int*>(&dummy));
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------ producer: g
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      long long it = 0;
+      int issued = 0;
+      for (long long w = wb; w < we; ++w, ++it) {
+        const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
+        const int s = (int)(it % kApG);
+        const uint32_t ph = (uint32_t)((it / kApG) & 1);
+        if (!mbar_wait(&gempty[s], ph ^ 1u, abort_flag)) break;
+        const int n0 = (int)(w % tph) * kTcTile;
+        mbar_arrive_expect_tx(&gfull[s], kTileBytes);
+        unsigned char* gt = sm + TcApplySmem::G + s * kTileBytes;
+        tma_load_3d(gt, &tmG, &gfull[s], h * 128, n0, b, pol);
+        tma_load_3d(gt + kBox, &tmG, &gfull[s], h * 128 + 64, n0, b, pol);
+        ++issued;
+      }
+      if (*abort_flag) {
+        long long first = it - (issued < kApG ? issued : kApG);
+        for (long long i2 = first; i2 < it; ++i2) {
+          int dummy = 0;
+          mbar_wait(&gfull[i2 % kApG], (uint32_t)((i2 / kApG) & 1),
+                    reinterpret_cast<volatile int*>(&dummy));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(128, 128, false, false);
+      long long it = 0;
+      int seg = 0;
+      const uint32_t simg = sbase + TcApplySmem::SIMG;
+      for (long long w = wb; w < we; ++w, ++it) {
+        const bool first = seg_first(part, w, wb), last = seg_last(part, w, we);
+        if (first && !mbar_wait(sfull, (uint32_t)(seg & 1), abort_flag)) break;
+        const int ab = (int)(it % kApAcc);
+        const uint32_t aph = (uint32_t)((it / kApAcc) & 1);
+        if (!mbar_wait(&accempty[ab], aph ^ 1u, abort_flag)) break;
+        const int s = (int)(it % kApQ);
+        const uint32_t ph = (uint32_t)((it / kApQ) & 1);
+        if (!mbar_wait(&qready[s], ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t qt = sbase + TcApplySmem::Q + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32;
+          const uint64_t ad = sdesc_sw128(qt + koff, 16, 1024);
+          const uint64_t bd = sdesc_sw128(simg + koff, 16, 1024);
+          umma_f16kind(tmem + ab * 128, ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&qempty[s]);
+        umma_commit(&accfull[ab]);
+        if (last) {
+          umma_commit(sfree);
+          ++seg;
+        }
+      }
+      umma_commit(drain);
+      int dummy = 0;
+      mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy));
+    }
+  } else if (warp < kApEW0) {
+    // ------------------------------------ transform warps: q -> q_til, den
+    const int tw = warp - kApTW0;
+    const int rg = lane >> 3, j = lane & 7;
+    PairInfo pi;
+    pair_info(g, win, j, pi);
+    float zr[16];
+    long long it = 0;
+    int seg = 0;
+    for (long long w = wb; w < we; ++w, ++it) {
+      const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
+      if (seg_first(part, w, wb)) {
+        if (!mbar_wait(sfull, (uint32_t)(seg & 1), abort_flag)) break;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) zr[i] = zs[16 * j + i];
+        ++seg;
+      }
+      const int s = (int)(it % kApQ);
+      const uint32_t ph = (uint32_t)((it / kApQ) & 1);
+      if (!mbar_wait(&qfull[s], ph, abort_flag)) break;
+      const int n0 = (int)(w % tph) * kTcTile;
+      const uint32_t qt = sbase + TcApplySmem::Q + s * kTileBytes;
+      float* den = den_ring + (it % kApDen) * 128;
+#pragma unroll 1
+      for (int ps = 0; ps < kTcTile / kApRowsPerPass; ++ps) {
+        const int r = ps * kApRowsPerPass + tw * 4 + rg;
+        const int n = n0 + r;
+        uint32_t a0, a1;
+        lane_chunks(qt, r, j, a0, a1);
+        float x[16];
+        unpack16(lds128(a0), lds128(a1), x);
+        norm_relu16(x);
+        float dp = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dp = fmaf(zr[i], x[i], dp);
+        dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+        dp += __shfl_xor_sync(0xffffffffu, dp, 2);
+        dp += __shfl_xor_sync(0xffffffffu, dp, 4);
+        const float dn = dp + g.eps;
+        const uint32_t opk = packed_pos(g, win, n < g.N ? n : n0);
+        uint4 o0, o1;
+        rope_pack16<true>(g, tab, pi, opk, x, 1.f, o0, o1);
+        sts128(a0, o0);
+        sts128(a1, o1);
+        if (j == 0) {
+          den[r] = dn;
+          if (kDebug && p.den_out && n < g.N) p.den_out[((size_t)b * g.N + n) * g.Hh + h] = dn;
+        }
+      }
+      // The epilogue of this tile reads the row scales of S from this ring
+      // slot, which (like den) stays untouched until that epilogue is done;
+      // the shared copy at RS may meanwhile be replaced by the next head's.
+      if (lane < 16) rs_ring[(it % kApDen) * 128 + tw * 16 + lane] = rs[tw * 16 + lane];
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qready[s]);
+    }
+  } else {
+    // ---------------------- epilogue warps: gate, denominator, RMSNorm, store
+    const int ew = warp - kApEW0;
+    const int grp = ew >> 2;            // accumulator this group drains
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const bool storer = (ew & 3) == 0 && lane == 0;
+    const uint64_t pol = policy_evict_first();
+    long long it = 0;
+    for (long long w = wb; w < we; ++w, ++it) {
+      if ((int)(it % kApAcc) != grp) continue;
+      const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
+      const int n0 = (int)(w % tph) * kTcTile;
+      const uint32_t aph = (uint32_t)((it / kApAcc) & 1);
+      if (!mbar_wait(&accfull[grp], aph, abort_flag)) break;
+      tc_fence_after();
+      const int gsl = (int)(it % kApG);
+      const uint32_t gph = (uint32_t)((it / kApG) & 1);
+      if (!mbar_wait(&gfull[gsl], gph, abort_flag)) break;
+      const float inv_den = 1.f / den_ring[(it % kApDen) * 128 + row];
+      const float* rsc = rs_ring + (it % kApDen) * 128;
+      const uint32_t taddr = tmem + (uint32_t)(grp * 128) + ((uint32_t)(q4 * 32) << 16);
+      const uint32_t gt = sbase + TcApplySmem::G + gsl * kTileBytes;
+      const uint32_t grow = gt + (uint32_t)row * 128u;
+      const uint32_t sw = (uint32_t)(row & 7);
+      float ss = 0.f;
+#pragma unroll 1
+      for (int cb = 0; cb < 4; ++cb) {
+        float u[32];
+        tmem_ld32(taddr + cb * 32, u);
+        const uint32_t rbase = grow + (uint32_t)(cb >> 1) * kBox;
+        uint4 gv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) gv[q] = lds128(rbase + ((((uint32_t)((cb & 1) * 4 + q)) ^ sw) << 4));
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t wv[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float g0 = bf_lo(wv[e]), g1 = bf_hi(wv[e]);
+            const float s0 = __fdividef(1.f, 1.f + __expf(-g0));
+            const float s1 = __fdividef(1.f, 1.f + __expf(-g1));
+            const int col = cb * 32 + q * 8 + 2 * e;
+            float& x0 = u[q * 8 + 2 * e];
+            float& x1 = u[q * 8 + 2 * e + 1];
+            x0 = (s0 * inv_den) * (x0 * rsc[col]);
+            x1 = (s1 * inv_den) * (x1 * rsc[col + 1]);
+            ss = fmaf(x0, x0, ss);
+            ss = fmaf(x1, x1, ss);
+          }
+        }
+        if (kDebug && p.x_out && n0 + row < g.N) {
+          float* xo = p.x_out + (((size_t)b * g.N + n0 + row) * g.Hh + h) * 128 + cb * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(xo + i) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
+        }
+        tmem_st32(taddr + cb * 32, u);
+      }
+      tmem_wait_st();
+      const float rstd = rsqrtf(ss * (1.f / 128.f) + kRmsEps);
+#pragma unroll 1
+      for (int cb = 0; cb < 4; ++cb) {
+        float x[32];
+        tmem_ld32(taddr + cb * 32, x);
+        tmem_wait_ld();
+        const uint32_t rbase = grow + (uint32_t)(cb >> 1) * kBox;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 o;
+          o.x = pack_bf16(x[q * 8 + 0] * rstd, x[q * 8 + 1] * rstd);
+          o.y = pack_bf16(x[q * 8 + 2] * rstd, x[q * 8 + 3] * rstd);
+          o.z = pack_bf16(x[q * 8 + 4] * rstd, x[q * 8 + 5] * rstd);
+          o.w = pack_bf16(x[q * 8 + 6] * rstd, x[q * 8 + 7] * rstd);
+          sts128(rbase + ((((uint32_t)((cb & 1) * 4 + q)) ^ sw) << 4), o);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[grp]);
+      fence_proxy_async_smem();
+      named_barrier(2 + grp, 128);
+      if (storer) {
+        tma_store_3d(&tmO, sm + TcApplySmem::G + gsl * kTileBytes, h * 128, n0, b, pol);
+        tma_store_3d(&tmO, sm + TcApplySmem::G + gsl * kTileBytes + kBox, h * 128 + 64, n0, b, pol);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(&gempty[gsl]);
+      }
+    }
+    if (storer) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ------------------------------------------------------------------- host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [B][N][Hh][128] bf16 activations as a 3D map (channel, token, batch) with
+// boxes of 64 channels x 128 tokens, 128-byte swizzle, zero fill past N.
+inline bool make_act_map(CUtensorMap* m, const void* ptr, const Geom& g) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)g.Hh * 128, (cuuint64_t)g.N, (cuuint64_t)g.B};
+  cuuint64_t strides[2] = {(cuuint64_t)g.Hh * 128 * 2, (cuuint64_t)g.N * g.Hh * 128 * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline size_t tc_state_smem(int tab_entries) {
+  return 1024 + TcStateSmem::TAB + (size_t)tab_entries * 8;
+}
+inline size_t tc_apply_smem(int tab_entries) {
+  return 1024 + TcApplySmem::TAB + (size_t)tab_entries * 8;
+}
+constexpr size_t kMaxSmem = 232448;
+
+// Per-CTA RoPE table size of the tensor partition (max over CTAs).
+inline int tc_table_entries(const Geom& g, const Partition& part) {
+  if (!g.rope_on) return 1;
+  int mx = 1;
+  for (int c = 0; c < part.grid; ++c) {
+    const RopeWindow win = rope_window(g, part, part_begin(part, c), part_begin(part, c + 1) - 1);
+    const int e = rope_table_entries(g, win.Lt);
+    if (e > mx) mx = e;
+  }
+  return mx;
+}
+
+inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const void* v,
+                             const void* beta, const void* gate, void* out, float* S,
+                             float* z, bool carry, float* part_S, float* part_z,
+                             __half* S_img, float* S_rs, float* den_dbg, float* x_dbg,
+                             int sms, cudaStream_t stream, void* const* events) {
+  auto mark = [&](int i) {
+    if (!events || !events[i]) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream);
+  };
+  if (sms <= 0) return GLA_ERR_CUDA;
+  if (g.H >= (1 << kPosBits) || g.W >= (1 << kPosBits) || g.T >= (1 << kPosBits))
+    return GLA_ERR_UNSUPPORTED;
+  const Partition part = make_partition(g.B * g.Hh, g.N, kTcTile, sms);
+  const int tab = tc_table_entries(g, part);
+  const size_t smem_st = tc_state_smem(tab), smem_ap = tc_apply_smem(tab);
+  if (smem_st > kMaxSmem || smem_ap > kMaxSmem) return GLA_ERR_UNSUPPORTED;
+
+  CUtensorMap mK, mV, mQ, mG, mO;
+  if (!make_act_map(&mK, k, g) || !make_act_map(&mV, v, g) || !make_act_map(&mQ, q, g) ||
+      !make_act_map(&mG, gate, g) || !make_act_map(&mO, out, g))
+    return GLA_ERR_CUDA;
+
+  TcStateParams sp;
+  sp.g = g; sp.part = part;
+  sp.beta = static_cast<const __nv_bfloat16*>(beta);
+  sp.part_S = part_S; sp.part_z = part_z; sp.tab_entries = tab;
+  if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_st) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  if (mark(0) != cudaSuccess) return GLA_ERR_CUDA;
+  tc_state_kernel<<<part.grid, kStThreads, smem_st, stream>>>(mK, mV, sp);
+  if (cudaGetLastError() != cudaSuccess || mark(1) != cudaSuccess) return GLA_ERR_CUDA;
+
+  CombineParams cp;
+  cp.part = part; cp.d = 128; cp.zparts = kStTW;
+  cp.part_S = part_S; cp.part_z = part_z;
+  cp.S_in = carry ? S : nullptr;
+  cp.z_in = carry ? z : nullptr;
+  cp.S_out = S; cp.z_out = z; cp.S_img = S_img; cp.S_rs = S_rs;
+  dim3 cgrid(128 * 128 / kCombineElems, g.B * g.Hh);
+  combine_kernel<<<cgrid, kCombineThreads, 0, stream>>>(cp);
+  if (cudaGetLastError() != cudaSuccess || mark(2) != cudaSuccess) return GLA_ERR_CUDA;
+
+  TcApplyParams ap;
+  ap.g = g; ap.part = part; ap.S_img = S_img; ap.S_rs = S_rs; ap.z = z;
+  ap.den_out = den_dbg; ap.x_out = x_dbg; ap.tab_entries = tab;
+  const bool dbg = den_dbg != nullptr || x_dbg != nullptr;
+  if (dbg) {
+    if (cudaFuncSetAttribute(tc_apply_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_ap) != cudaSuccess)
+      return GLA_ERR_CUDA;
+    tc_apply_kernel<true><<<part.grid, kApThreads, smem_ap, stream>>>(mQ, mG, mO, ap);
+  } else {
+    if (cudaFuncSetAttribute(tc_apply_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_ap) != cudaSuccess)
+      return GLA_ERR_CUDA;
+    tc_apply_kernel<false><<<part.grid, kApThreads, smem_ap, stream>>>(mQ, mG, mO, ap);
+  }
+  if (cudaGetLastError() != cudaSuccess || mark(3) != cudaSuccess) return GLA_ERR_CUDA;
+  return GLA_OK;
+}
+
+}  // namespace gla

@@ -1,0 +1,228 @@
+"""ctypes binding of libgla.so (include/gla.h).
+
+Argument marshalling only: every step of the operator runs in the library's
+CUDA kernels.  Tensors are torch tensors (device memory for the device entry
+points, host memory for gla_forward_host); the binding passes their data
+pointers, sizes and the current CUDA stream.  A missing or unloadable library
+raises immediately: there is no fallback.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgla.so")
+
+GLA_OK, GLA_ERR_INVALID_ARG, GLA_ERR_UNSUPPORTED, GLA_ERR_WORKSPACE, GLA_ERR_CUDA, \
+    GLA_ERR_TIMEOUT = range(6)
+GLA_DTYPE_F32, GLA_DTYPE_BF16 = 0, 1
+GLA_PATH_AUTO, GLA_PATH_SIMT, GLA_PATH_TENSOR = 0, 1, 2
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_fp = ctypes.POINTER(ctypes.c_float)
+
+_SIGS = {
+    "gla_version": (_i, []),
+    "gla_status_string": (ctypes.c_char_p, [_i]),
+    "gla_forward_workspace_size": (_sz, [_i] * 7),
+    "gla_block_causal_workspace_size": (_sz, [_i] * 7),
+    "gla_forward_host_arena_size": (_sz, [_i] * 7),
+    "gla_forward": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
+    "gla_forward_ex": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp, _i]),
+    "gla_forward_debug": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp, _i]
+                          + [_vp] * 4),
+    "gla_forward_timed": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp, _i,
+                                                        ctypes.POINTER(_vp)]),
+    "gla_block_causal_step": (_i, [_vp] * 7 + [_i] * 7 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
+    "gla_block_causal_step_ex": (_i, [_vp] * 7 + [_i] * 7
+                                 + [_f, _f, _i, _vp, _vp, _sz, _vp, _i]),
+    "gla_forward_host": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
+    "gla_get_device_status": (_i, [_vp]),
+    "gla_plan": (_i, [_i] * 9 + [ctypes.POINTER(_i)] * 3),
+}
+
+_lib = None
+
+
+class GlaError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+def lib():
+    """The loaded libgla.so (raises OSError if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"libgla.so not built ({LIB_PATH}); run "
+                          "python -m gated_bidirectional_linear_b200.build")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def status_string(status):
+    return lib().gla_status_string(int(status)).decode()
+
+
+def _check(status, what):
+    if status != GLA_OK:
+        raise GlaError(status, what)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return GLA_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return GLA_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dims(q, T, H, W):
+    B, N, Hh, d = q.shape
+    if N != T * H * W:
+        raise ValueError(f"q has {N} tokens, grid {T}x{H}x{W} has {T * H * W}")
+    return B, Hh, d
+
+
+def gla_forward_workspace_size(batch, heads, head_dim, T, H, W, dtype):
+    return lib().gla_forward_workspace_size(batch, heads, head_dim, T, H, W, dtype)
+
+
+def gla_block_causal_workspace_size(batch, heads, head_dim, T_blk, H, W, dtype):
+    return lib().gla_block_causal_workspace_size(batch, heads, head_dim, T_blk, H, W, dtype)
+
+
+def gla_forward_host_arena_size(batch, heads, head_dim, T, H, W, dtype):
+    return lib().gla_forward_host_arena_size(batch, heads, head_dim, T, H, W, dtype)
+
+
+def alloc_workspace(nbytes, device="cuda"):
+    """A 256-byte aligned device buffer of nbytes (torch allocations are)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def gla_forward(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, out=None,
+                workspace=None, stream=None, path=GLA_PATH_AUTO):
+    """o = RMSNorm(sigmoid(g) * S q_til / (z.q_pls + eps)) over all T*H*W tokens.
+
+    q, k, v, g: [B, N, Hh, d]; beta: [B, N, Hh]; all on the GPU, same dtype."""
+    B, Hh, d = _dims(q, T, H, W)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(gla_forward_workspace_size(B, Hh, d, T, H, W, code), q.device)
+    st = lib().gla_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T, H,
+                              W, rope_theta, eps, code, _ptr(out), _ptr(workspace),
+                              workspace.numel(), _stream(stream), path)
+    _check(st, "gla_forward")
+    return out
+
+
+def gla_forward_timed(q, k, v, beta, g, T, H, W, events, rope_theta=10000.0, eps=1e-6,
+                      out=None, workspace=None, stream=None, path=GLA_PATH_AUTO):
+    """gla_forward recording four torch.cuda.Event objects around its kernels
+    (before the state reduction, after it, after the combine, after the
+    read-out)."""
+    B, Hh, d = _dims(q, T, H, W)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(gla_forward_workspace_size(B, Hh, d, T, H, W, code), q.device)
+    ev = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) if e is not None else None
+                                 for e in events])
+    st = lib().gla_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
+                                 H, W, rope_theta, eps, code, _ptr(out), _ptr(workspace),
+                                 workspace.numel(), _stream(stream), path, ev)
+    _check(st, "gla_forward_timed")
+    return out
+
+
+def gla_forward_debug(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6,
+                      path=GLA_PATH_AUTO, stream=None):
+    """gla_forward plus the hidden intermediates S, z, den and x (pre-norm)."""
+    B, Hh, d = _dims(q, T, H, W)
+    N = q.shape[1]
+    code = _dtype_code(q)
+    dev = q.device
+    out = torch.empty_like(q)
+    S = torch.empty(B, Hh, d, d, dtype=torch.float32, device=dev)
+    z = torch.empty(B, Hh, d, dtype=torch.float32, device=dev)
+    den = torch.empty(B, N, Hh, dtype=torch.float32, device=dev)
+    x = torch.empty(B, N, Hh, d, dtype=torch.float32, device=dev)
+    ws = alloc_workspace(gla_forward_workspace_size(B, Hh, d, T, H, W, code), dev)
+    st = lib().gla_forward_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
+                                 H, W, rope_theta, eps, code, _ptr(out), _ptr(ws), ws.numel(),
+                                 _stream(stream), path, _ptr(S), _ptr(z), _ptr(den), _ptr(x))
+    _check(st, "gla_forward_debug")
+    return dict(out=out, S=S, z=z, den=den, x=x)
+
+
+def gla_block_causal_step(state, z, q, k, v, beta, g, T_blk, H, W, t0, rope_theta=10000.0,
+                          eps=1e-6, out=None, workspace=None, stream=None,
+                          path=GLA_PATH_AUTO):
+    """One block: state += block state, z += block key sum (in place), then the
+    block is read out against the updated state.  state [B,Hh,d,d], z [B,Hh,d]
+    fp32 on the GPU."""
+    B, Hh, d = _dims(q, T_blk, H, W)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(
+            gla_block_causal_workspace_size(B, Hh, d, T_blk, H, W, code), q.device)
+    st = lib().gla_block_causal_step_ex(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(beta), _ptr(g), B, Hh, d, T_blk, H, W, t0,
+                                        rope_theta, eps, code, _ptr(out), _ptr(workspace),
+                                        workspace.numel(), _stream(stream), path)
+    _check(st, "gla_block_causal_step")
+    return out
+
+
+def gla_forward_host(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, out=None,
+                     arena=None, stream=None):
+    """gla_forward on host tensors (pin them for asynchronous copies): one H2D
+    copy per input into the device `arena`, the operator, one D2H copy of out.
+    Asynchronous on `stream`; synchronise before reading `out`."""
+    B, Hh, d = _dims(q, T, H, W)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if arena is None:
+        arena = alloc_workspace(gla_forward_host_arena_size(B, Hh, d, T, H, W, code))
+    st = lib().gla_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
+                                H, W, rope_theta, eps, code, _ptr(out), _ptr(arena),
+                                arena.numel(), _stream(stream))
+    _check(st, "gla_forward_host")
+    return out
+
+
+def gla_get_device_status(stream=None):
+    """Synchronise the stream and return (and clear) the device error status."""
+    return lib().gla_get_device_status(_stream(stream))
+
+
+def gla_plan(batch, heads, head_dim, T, H, W, dtype, path, num_sms):
+    grid, tile, used = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    st = lib().gla_plan(batch, heads, head_dim, T, H, W, dtype, path, num_sms,
+                        ctypes.byref(grid), ctypes.byref(tile), ctypes.byref(used))
+    _check(st, "gla_plan")
+    return grid.value, tile.value, used.value

@@ -1,0 +1,206 @@
+/*
+ * gla.h - C ABI of libgla.so: gated bidirectional ReLU linear attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operator (per batch element b and head h, head dim d, N = T*H*W latent
+ * tokens in raster order n = (t*H + h)*W + w):
+ *
+ *   q_hat = RMSNorm(q), k_hat = RMSNorm(k)       over d, no weight, eps 1e-6
+ *   q_pls = ReLU(q_hat), k_pls = ReLU(k_hat)
+ *   q_til = RoPE3D(q_pls), k_til = RoPE3D(k_pls)  (rotation after the ReLU)
+ *   S     = sum_n v_n (beta_n k_til_n)^T            d x d, S[a][c]
+ *   z     = sum_n k_pls_n                           d
+ *   den_j = z . q_pls_j + eps                       (no rotation: stays > 0)
+ *   o_j   = RMSNorm( sigmoid(g_j) * (S q_til_j) / den_j )
+ *
+ * Sources: the SANA-Video 2.0 summary (paper.rainbus.top), prerequisites
+ * "Gated Bilinear Linear Attention" (the read-out o_j, normalised q/k, phi =
+ * ReLU, write gate beta, sigmoid output gate g, bidirectional sum) and
+ * "Linear Attention" (S = sum_n v_n (beta_n k_n)^T); the SANA-Video notes
+ * (papernotes.org), key design 1 (RoPE(ReLU(x)), RoPE in the numerator only so
+ * the denominator stays positive) and key design 2 (block-causal linear
+ * attention carries the running sums of S and of the key features).  The
+ * output projection W_o of the read-out formula is not part of this library.
+ *
+ * 3D RoPE (the pages fix no split; this is the library's normative spec):
+ *   P = d/2 rotation pairs.  Time gets P - 2*floor(P/3) pairs, height and
+ *   width floor(P/3) each (22/21/21 for d = 128, 6/5/5 for d = 32), as
+ *   contiguous channel chunks in the order t, h, w.  Inside an axis chunk of
+ *   p pairs, pair i is channels (2i, 2i+1), frequency theta^(-i/p), angle
+ *   pos * frequency, and (x0, x1) -> (x0 cos - x1 sin, x0 sin + x1 cos).
+ *   Positions are integers from 0; the time position is t0 + local frame in
+ *   gla_block_causal_step (0 in gla_forward).  rope_theta <= 0 disables RoPE.
+ *
+ * Layouts (all caller-owned DEVICE memory unless stated, contiguous, 16-byte
+ * aligned):  q, k, v, g, out: [batch][N][heads][head_dim] in `dtype`;
+ * beta: [batch][N][heads] in `dtype` (taken as given: apply its sigmoid
+ * before the call); g holds gate logits (the operator applies the sigmoid).
+ * State S: [batch][heads][d][d] fp32 with S[a][c] = sum_n v_n[a] beta_n
+ * k_til_n[c]; z: [batch][heads][d] fp32.
+ *
+ * Supported: dtype F32 or BF16; head_dim 32, 64 or 128.  BF16 with
+ * head_dim 128 runs on the tcgen05 tensor-core path (TMA-fed state reduction
+ * and read-out); every other case, or path GLA_PATH_SIMT, runs on CUDA cores
+ * with fp32 arithmetic.  Accumulation is always fp32.  On the tensor path the
+ * MMA operands beta*k_til, q_til and S are rounded to bf16; outputs are
+ * rounded to nearest even.
+ *
+ * Errors: every entry point validates its arguments first and returns an
+ * error code with nothing launched.  A CUDA launch failure returns
+ * GLA_ERR_CUDA.  Calls are asynchronous on `stream` (a cudaStream_t passed as
+ * void*; NULL = legacy default stream).  Device-side wait timeouts (the
+ * tensor path's bounded mbarrier waits) are recorded in a library-owned
+ * device word and reported by gla_get_device_status().
+ *
+ * Determinism: the state is reduced in a fixed split order, so the same
+ * inputs on the same GPU model give bitwise-identical results.
+ *
+ * Memory: the library allocates no device memory.  Scratch space is the
+ * caller's `workspace` of at least *_workspace_size() bytes, 256-byte
+ * aligned; its contents need no initialisation and are overwritten.
+ */
+#ifndef GLA_H
+#define GLA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GLA_API __attribute__((visibility("default")))
+#else
+#define GLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gla_status {
+  GLA_OK = 0,
+  GLA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, eps <= 0 */
+  GLA_ERR_UNSUPPORTED = 2,  /* head_dim/dtype/path combination not built */
+  GLA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+  GLA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  GLA_ERR_TIMEOUT = 5       /* a device-side bounded wait expired */
+} gla_status;
+
+typedef enum gla_dtype { GLA_DTYPE_F32 = 0, GLA_DTYPE_BF16 = 1 } gla_dtype;
+
+typedef enum gla_path {
+  GLA_PATH_AUTO = 0,   /* tensor path when supported, else SIMT */
+  GLA_PATH_SIMT = 1,   /* CUDA-core fp32 kernels */
+  GLA_PATH_TENSOR = 2  /* tcgen05 + TMA kernels (bf16, head_dim 128 only) */
+} gla_path;
+
+/* RMSNorm epsilon used for q, k and the output (a fixed library constant). */
+#define GLA_RMS_EPS 1e-6f
+
+/* Library version, major*10000 + minor*100 + patch. */
+GLA_API int gla_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+GLA_API const char* gla_status_string(int status);
+
+/* Bytes of workspace gla_forward / gla_forward_ex / gla_forward_debug need
+ * for this problem (independent of the GPU).  0 for invalid sizes. */
+GLA_API size_t gla_forward_workspace_size(int batch, int heads, int head_dim, int T, int H,
+                                  int W, int dtype);
+
+/* The bidirectional operator over all N = T*H*W tokens (the read-out formula
+ * of the "Gated Bilinear Linear Attention" prerequisite).  Writes out; reads
+ * q, k, v, beta, g.  eps > 0 is the denominator epsilon. */
+GLA_API gla_status gla_forward(const void* q, const void* k, const void* v, const void* beta,
+                       const void* g, int batch, int heads, int head_dim, int T, int H,
+                       int W, float rope_theta, float eps, int dtype, void* out,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* gla_forward with an explicit path (gla_path). */
+GLA_API gla_status gla_forward_ex(const void* q, const void* k, const void* v, const void* beta,
+                          const void* g, int batch, int heads, int head_dim, int T, int H,
+                          int W, float rope_theta, float eps, int dtype, void* out,
+                          void* workspace, size_t workspace_bytes, void* stream, int path);
+
+/* gla_forward that also exports the hidden intermediates (tests):
+ * S_out [batch][heads][d][d] fp32, z_out [batch][heads][d] fp32,
+ * den_out [batch][N][heads] fp32 (den_j), x_out [batch][N][heads][d] fp32
+ * (sigmoid(g_j) * S q_til_j / den_j, before the output RMSNorm).  Any of the
+ * four may be NULL.  Slower than gla_forward. */
+GLA_API gla_status gla_forward_debug(const void* q, const void* k, const void* v, const void* beta,
+                             const void* g, int batch, int heads, int head_dim, int T,
+                             int H, int W, float rope_theta, float eps, int dtype,
+                             void* out, void* workspace, size_t workspace_bytes,
+                             void* stream, int path, float* S_out, float* z_out,
+                             float* den_out, float* x_out);
+
+/* gla_forward that also records caller-created CUDA events (cudaEvent_t
+ * passed as void*) on `stream` around its kernels: events[0] before the state
+ * reduction, events[1] after it, events[2] after the combine, events[3] after
+ * the read-out.  For per-kernel timing in benchmarks; `events` may be NULL and
+ * any of its four entries may be NULL. */
+GLA_API gla_status gla_forward_timed(const void* q, const void* k, const void* v,
+                                     const void* beta, const void* g, int batch, int heads,
+                                     int head_dim, int T, int H, int W, float rope_theta,
+                                     float eps, int dtype, void* out, void* workspace,
+                                     size_t workspace_bytes, void* stream, int path,
+                                     void* const* events);
+
+/* Workspace bytes of gla_block_causal_step for one block of T_blk*H*W tokens. */
+GLA_API size_t gla_block_causal_workspace_size(int batch, int heads, int head_dim, int T_blk,
+                                       int H, int W, int dtype);
+
+/* One step of the block-causal variant (key design 2 of the SANA-Video notes:
+ * a new block only adds its own state to the carried running sums).
+ * state [batch][heads][d][d] fp32 and z [batch][heads][d] fp32 are caller-owned
+ * device memory, read and updated in place: state += sum over the block of
+ * v_n (beta_n k_til_n)^T, z += sum over the block of k_pls_n (added in a fixed
+ * order).  The block's tokens are then read out against the UPDATED state (a
+ * block sees itself).  RoPE time positions are t0 + local frame.  Zero state
+ * and z before the first step. */
+GLA_API gla_status gla_block_causal_step(float* state, float* z, const void* q, const void* k,
+                                 const void* v, const void* beta, const void* g,
+                                 int batch, int heads, int head_dim, int T_blk, int H,
+                                 int W, int t0, float rope_theta, float eps, int dtype,
+                                 void* out, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/* gla_block_causal_step with an explicit path (gla_path). */
+GLA_API gla_status gla_block_causal_step_ex(float* state, float* z, const void* q, const void* k,
+                                    const void* v, const void* beta, const void* g,
+                                    int batch, int heads, int head_dim, int T_blk, int H,
+                                    int W, int t0, float rope_theta, float eps, int dtype,
+                                    void* out, void* workspace, size_t workspace_bytes,
+                                    void* stream, int path);
+
+/* Bytes of the device arena gla_forward_host needs: room for the five inputs,
+ * the output and the workspace. */
+GLA_API size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, int T, int H, int W,
+                                   int dtype);
+
+/* gla_forward on HOST buffers (q_h .. out_h; pinned memory gives asynchronous
+ * copies).  Enqueues on `stream`: one host-to-device copy per input into the
+ * caller's device `arena`, the operator, and one device-to-host copy of the
+ * output.  Returns after enqueueing; synchronise `stream` before reading
+ * out_h.  The arena is caller-owned device memory of at least
+ * gla_forward_host_arena_size() bytes, 256-byte aligned. */
+GLA_API gla_status gla_forward_host(const void* q_h, const void* k_h, const void* v_h,
+                            const void* beta_h, const void* g_h, int batch, int heads,
+                            int head_dim, int T, int H, int W, float rope_theta, float eps,
+                            int dtype, void* out_h, void* arena, size_t arena_bytes,
+                            void* stream);
+
+/* Synchronises `stream`, then reports and clears the library's device error
+ * word: GLA_ERR_TIMEOUT if a kernel gave up a bounded wait since the last
+ * call, GLA_ERR_CUDA if the synchronisation itself failed, else GLA_OK. */
+GLA_API gla_status gla_get_device_status(void* stream);
+
+/* Host-only planning query (no GPU needed): the grid of the state-reduction
+ * kernel and the tokens per tile for this problem on a GPU with `num_sms`
+ * SMs and the given path.  Returns GLA_OK and fills *grid, *tile_tokens,
+ * *path_used; used by tests to check the split-N partition. */
+GLA_API gla_status gla_plan(int batch, int heads, int head_dim, int T, int H, int W, int dtype,
+                    int path, int num_sms, int* grid, int* tile_tokens, int* path_used);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLA_H */

@@ -1,0 +1,53 @@
+"""Shared helpers of the GPU parity tests: seeded inputs on the device, the
+oracle on selected heads, and the tolerance metrics."""
+import numpy as np
+import torch
+
+import oracle.gla_oracle as O
+from gated_bidirectional_linear_b200 import workloads
+
+# Tolerances (the benchmark spec: 1e-5 for fp32 inputs; 2e-2 relative to the
+# output RMS for bf16 inputs).  Hidden intermediates of the bf16 path: S within
+# 1e-2 of rms(S) (bf16 rounding of the beta*k_til operand), z and den within
+# 1e-3 relative (fp32 sums of exact bf16 inputs).
+F32_TOL = 1e-5
+BF16_TOL = 2e-2
+S_TOL_BF16 = 1e-2
+ZDEN_TOL = 1e-3
+
+
+def to_device(inputs, device="cuda"):
+    return {k: v.to(device) for k, v in inputs.items()}
+
+
+def head_slice(inputs, b, h):
+    """One (batch, head) of the inputs as float64 arrays of shape [1,N,1,d]."""
+    out = {}
+    for k, v in inputs.items():
+        if k == "beta":
+            out[k] = v[b:b + 1, :, h:h + 1].to(torch.float64).numpy()
+        else:
+            out[k] = v[b:b + 1, :, h:h + 1, :].to(torch.float64).numpy()
+    return out
+
+
+def oracle_forward(x, T, H, W, theta, eps, t0=0):
+    return O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T, H, W, theta, eps, t0)
+
+
+def rel_rms(got, ref):
+    return O.max_err_over_rms(got, ref)
+
+
+def rel_floor(got, ref):
+    return O.max_rel_err_rms_floor(got, ref)
+
+
+def rel_elem(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.max(np.abs(got - ref) / np.abs(ref)))
+
+
+def np64(t):
+    return t.detach().to("cpu", torch.float64).numpy()

@@ -1,0 +1,229 @@
+"""CUDA path against the fp64 oracle, element by element, through the C ABI.
+
+Small workloads are compared on every output and on the hidden intermediates
+(S, z, den and the gated pre-norm read-out x, exported by gla_forward_debug).
+The full-size workloads run in the launch configuration the benchmark times
+(gla_forward, tensor path) and are compared on every token of sampled heads,
+which the oracle recomputes from scratch."""
+import numpy as np
+import pytest
+import torch
+
+from gated_bidirectional_linear_b200 import gla, workloads
+from gpu_common import (BF16_TOL, F32_TOL, S_TOL_BF16, ZDEN_TOL, head_slice, np64,
+                        oracle_forward, rel_elem, rel_floor, rel_rms, to_device)
+import oracle.gla_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TENSOR, SIMT = gla.GLA_PATH_TENSOR, gla.GLA_PATH_SIMT
+
+
+def _oracle_all(inputs, T, H, W, theta, eps, t0=0):
+    x = workloads.as_f64(inputs)
+    return O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T, H, W, theta, eps, t0)
+
+
+def _debug(inp, T, H, W, theta, eps, path):
+    d = to_device(inp)
+    r = gla.gla_forward_debug(d["q"], d["k"], d["v"], d["beta"], d["g"], T, H, W, theta, eps,
+                              path=path)
+    torch.cuda.synchronize()
+    assert gla.gla_get_device_status() == gla.GLA_OK
+    return {k: np64(v) for k, v in r.items()}
+
+
+# ----------------------------------------------------------------- tiny fp32
+
+def test_tiny_fp32_all_outputs_and_intermediates():
+    wl = workloads.WORKLOADS["tiny"]
+    inp = workloads.make_inputs(wl)
+    ref = _oracle_all(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+    got = _debug(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, gla.GLA_PATH_AUTO)
+    assert rel_floor(got["out"], ref["out"]) <= F32_TOL
+    assert rel_floor(got["S"], ref["S"]) <= F32_TOL
+    assert rel_elem(got["z"], ref["z"]) <= F32_TOL
+    assert rel_elem(got["den"], ref["den"]) <= F32_TOL
+    assert rel_floor(got["x"], ref["x"]) <= F32_TOL
+
+
+# --------------------------------------------------------------- 480p bf16
+
+@pytest.fixture(scope="module")
+def w480():
+    wl = workloads.WORKLOADS["480p"]
+    inp = workloads.make_inputs(wl)
+    ref = _oracle_all(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+    return wl, inp, ref
+
+
+@pytest.mark.parametrize("path", [TENSOR, SIMT], ids=["tensor", "simt"])
+def test_480p_all_outputs(w480, path):
+    wl, inp, ref = w480
+    got = _debug(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, path)
+    err = rel_rms(got["out"], ref["out"])
+    print(f"480p {path}: out err/rms {err:.3e}")
+    assert err <= BF16_TOL
+    assert rel_rms(got["x"], ref["x"]) <= BF16_TOL
+    assert np.max(np.abs(got["S"] - ref["S"])) / np.sqrt(np.mean(ref["S"] ** 2)) <= S_TOL_BF16
+    assert rel_elem(got["z"], ref["z"]) <= ZDEN_TOL
+    assert rel_elem(got["den"], ref["den"]) <= ZDEN_TOL
+
+
+def test_480p_paths_agree(w480):
+    wl, inp, _ = w480
+    a = _debug(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, TENSOR)
+    b = _debug(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, SIMT)
+    assert rel_rms(a["x"], b["x"]) <= BF16_TOL
+
+
+# ------------------------------------------------- full sizes, sampled heads
+
+def _sampled_parity(name, heads):
+    wl = workloads.WORKLOADS[name]
+    inp = workloads.make_inputs(wl)
+    d = to_device(inp)
+    out = gla.gla_forward(d["q"], d["k"], d["v"], d["beta"], d["g"], wl.T, wl.H, wl.W,
+                          wl.rope_theta, wl.eps)
+    torch.cuda.synchronize()
+    assert gla.gla_get_device_status() == gla.GLA_OK
+    out = out.cpu()
+    worst = 0.0
+    for b, h in heads:
+        ref = oracle_forward(head_slice(inp, b, h), wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+        got = out[b:b + 1, :, h:h + 1, :].to(torch.float64).numpy()
+        worst = max(worst, rel_rms(got, ref["out"]))
+    print(f"{name}: sampled heads {heads}: out err/rms {worst:.3e}")
+    assert worst <= BF16_TOL
+
+
+def test_720p_sampled_heads():
+    _sampled_parity("720p", [(0, 0), (0, 19), (1, 7), (1, 13)])
+
+
+def test_14b_sampled_heads():
+    _sampled_parity("14b", [(0, 0), (0, 17), (0, 31)])
+
+
+# ------------------------------------------------------------- block-causal
+
+def _run_blocks(wl, inp, path):
+    L = wl.tokens
+    d = to_device(inp)
+    B, N, Hh, hd = d["q"].shape
+    state = torch.zeros(B, Hh, hd, hd, dtype=torch.float32, device="cuda")
+    z = torch.zeros(B, Hh, hd, dtype=torch.float32, device="cuda")
+    out = torch.empty_like(d["q"])
+    ws = gla.alloc_workspace(gla.gla_block_causal_workspace_size(
+        B, Hh, hd, wl.T, wl.H, wl.W, gla.GLA_DTYPE_BF16 if d["q"].dtype == torch.bfloat16 else 0))
+    for i in range(wl.n_blocks):
+        sl = slice(i * L, (i + 1) * L)
+        blk = {k: v[:, sl].contiguous() for k, v in d.items()}
+        o = gla.gla_block_causal_step(state, z, blk["q"], blk["k"], blk["v"], blk["beta"],
+                                      blk["g"], wl.T, wl.H, wl.W, i * wl.T, wl.rope_theta,
+                                      wl.eps, workspace=ws, path=path)
+        out[:, sl] = o
+    torch.cuda.synchronize()
+    assert gla.gla_get_device_status() == gla.GLA_OK
+    return out.cpu(), state.cpu(), z.cpu()
+
+
+def test_block_causal_sampled_heads():
+    wl = workloads.WORKLOADS["blk"]
+    inp = workloads.make_inputs(wl)
+    out, state, z = _run_blocks(wl, inp, gla.GLA_PATH_AUTO)
+    for b, h in [(0, 0), (0, 11), (0, 19)]:
+        x = head_slice(inp, b, h)
+        ref = O.block_causal_forward(x["q"], x["k"], x["v"], x["beta"], x["g"], wl.n_blocks,
+                                     wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+        got = out[b:b + 1, :, h:h + 1, :].to(torch.float64).numpy()
+        assert rel_rms(got, ref["out"]) <= BF16_TOL
+        S = state[b, h].double().numpy()
+        assert np.max(np.abs(S - ref["S"][0, 0])) / np.sqrt(np.mean(ref["S"] ** 2)) <= S_TOL_BF16
+        assert rel_elem(z[b, h].double().numpy(), ref["z"][0, 0]) <= ZDEN_TOL
+
+
+def test_block_causal_fp32_tiny_grid():
+    """fp32 block-causal on a small grid (4 blocks x 2x3x4) vs the oracle."""
+    wl = workloads.Workload("blk-tiny", 1, 2, 32, 2, 3, 4, "f32", seed=9, n_blocks=4)
+    inp = workloads.make_inputs(wl)
+    out, state, z = _run_blocks(wl, inp, gla.GLA_PATH_AUTO)
+    x = workloads.as_f64(inp)
+    ref = O.block_causal_forward(x["q"], x["k"], x["v"], x["beta"], x["g"], wl.n_blocks,
+                                 wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+    assert rel_floor(out.double().numpy(), ref["out"]) <= F32_TOL
+    assert rel_floor(state.double().numpy(), ref["S"]) <= F32_TOL
+
+
+# ----------------------------------------------------------------- edge cases
+
+EDGE = [
+    # (B, Hh, d, T, H, W, dtype, theta)
+    (2, 3, 128, 1, 1, 1, "bf16", 1e4),        # one token per head
+    (1, 5, 128, 1, 10, 10, "bf16", 1e4),      # N = 100 < one tile
+    (2, 3, 128, 1, 1, 257, "bf16", 1e4),      # ragged tail of one token
+    (1, 2, 128, 10, 32, 40, "bf16", 1e4),     # CTAs straddle the head boundary
+    (1, 3, 128, 7, 9, 11, "bf16", 0.0),       # RoPE off
+    (1, 4, 64, 3, 5, 7, "bf16", 1e4),         # d = 64 (CUDA-core path)
+    (1, 4, 32, 3, 5, 7, "bf16", 500.0),       # d = 32 bf16
+    (2, 3, 64, 3, 5, 7, "f32", 1e4),          # d = 64 fp32
+    (1, 2, 128, 2, 3, 33, "f32", 1e4),        # d = 128 fp32
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[str(c) for c in EDGE])
+def test_edge_shapes(case):
+    B, Hh, d, T, H, W, dt, theta = case
+    inp = workloads.draw(B, T * H * W, Hh, d, dt, seed=123)
+    ref = _oracle_all(inp, T, H, W, theta, 1e-6)
+    paths = [gla.GLA_PATH_AUTO] + ([SIMT] if (dt == "bf16" and d == 128) else [])
+    for path in paths:
+        got = _debug(inp, T, H, W, theta, 1e-6, path)
+        if dt == "f32":
+            assert rel_floor(got["out"], ref["out"]) <= F32_TOL
+            assert rel_floor(got["S"], ref["S"]) <= F32_TOL
+        else:
+            assert rel_rms(got["out"], ref["out"]) <= BF16_TOL
+            assert rel_rms(got["x"], ref["x"]) <= BF16_TOL
+            assert np.max(np.abs(got["S"] - ref["S"])) / np.sqrt(np.mean(ref["S"] ** 2)) <= S_TOL_BF16
+        assert rel_elem(got["z"], ref["z"]) <= ZDEN_TOL
+        assert np.all(got["den"] >= 1e-6 * (1 - 1e-6))
+
+
+# ---------------------------------------------------- determinism and host API
+
+def test_bitwise_deterministic():
+    wl = workloads.WORKLOADS["480p"]
+    d = to_device(workloads.make_inputs(wl))
+    a = gla.gla_forward(d["q"], d["k"], d["v"], d["beta"], d["g"], wl.T, wl.H, wl.W)
+    b = gla.gla_forward(d["q"], d["k"], d["v"], d["beta"], d["g"], wl.T, wl.H, wl.W)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_host_entry_matches_device_entry():
+    wl = workloads.WORKLOADS["480p"]
+    inp = workloads.make_inputs(wl)
+    pinned = {k: v.pin_memory() for k, v in inp.items()}
+    out_h = torch.empty_like(pinned["q"]).pin_memory()
+    gla.gla_forward_host(pinned["q"], pinned["k"], pinned["v"], pinned["beta"], pinned["g"],
+                         wl.T, wl.H, wl.W, out=out_h)
+    torch.cuda.synchronize()
+    d = to_device(inp)
+    dev = gla.gla_forward(d["q"], d["k"], d["v"], d["beta"], d["g"], wl.T, wl.H, wl.W)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, dev.cpu())
+
+
+def test_time_offset_invariance_single_block():
+    """One block from zero state with t0 = 0 and t0 = 7 (fp32): rotated dot
+    products depend on position differences only."""
+    inp = workloads.draw(1, 2 * 3 * 4, 2, 32, "f32", seed=5)
+    d = to_device(inp)
+    outs = []
+    for t0 in (0, 7):
+        st = torch.zeros(1, 2, 32, 32, device="cuda")
+        z = torch.zeros(1, 2, 32, device="cuda")
+        outs.append(gla.gla_block_causal_step(st, z, d["q"], d["k"], d["v"], d["beta"], d["g"],
+                                              2, 3, 4, t0).cpu().double().numpy())
+    assert rel_floor(outs[1], outs[0]) <= F32_TOL
