@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="only run warmup + steps of gla_forward (for ncu captures)")
     return ap.parse_args()
 
 
@@ -238,12 +240,26 @@ def main():
                               stream=stream)
 
     none4 = [None] * 4
+    if args.profile:
+        for _ in range(args.warmup + args.steps):
+            step(none4)
+        torch.cuda.synchronize(dev)
+        status = gla.gla_get_device_status(stream)
+        print(json.dumps({"profile_run": wl.name, "steps": args.warmup + args.steps,
+                          "status": gla.status_string(status)}))
+        if status != gla.GLA_OK:
+            sys.exit(1)
+        return
     for _ in range(max(args.warmup, 3)):
         step(none4)
     torch.cuda.synchronize(dev)
     assert gla.gla_get_device_status(stream) == gla.GLA_OK
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e4 in evs:          # torch creates its events lazily, at the first record
+        for e in e4:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockMonitor(local) as mon:

@@ -5,21 +5,28 @@
 //   S = (((S_in + P_{c_lo}) + P_{c_lo+1}) + ... ) + P_{c_hi}
 // in that fixed order (S_in = 0 for the bidirectional call, the carried state
 // for a block-causal step), so the result does not depend on scheduling.
-// Besides S (fp32) the kernel can write the fp16 image of S that the tensor
-// read-out kernel copies into shared memory as its B operand: two K-blocks of
-// [d rows][64 columns], rows of 128 bytes, 16-byte chunks XOR-swizzled by
-// (row & 7) - the canonical K-major 128-byte-swizzle layout of tcgen05.
-// Row a of the image holds S[a][:] * 2^e_a with e_a chosen so the row's
-// largest magnitude lands in [2^13, 2^14) (far inside the fp16 range, full
-// fp16 precision for the entries that matter); S_rs[a] = 2^-e_a undoes it in
-// the read-out epilogue.
+//
+// One cluster of kCombineCluster CTAs handles one head; each CTA sums a slice
+// of S.  For the tensor read-out the kernel also writes the fp16 image of S
+// that the read-out copies into shared memory as its B operand: two K-blocks
+// of [128 rows][64 columns], rows of 128 bytes, 16-byte chunks XOR-swizzled by
+// (row & 7) -- the canonical K-major 128-byte-swizzle layout of tcgen05.  The
+// image is S * 2^e with one power of two per head, chosen from the head's
+// largest |S| (exchanged across the cluster through distributed shared
+// memory) so that it lands in [2^13, 2^14): every entry that matters is a
+// normal fp16 number with full fp16 precision.  S_scale[bh][0] = 2^e.
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 
 #include "common.cuh"
 
 namespace gla {
+
+constexpr int kCombineCluster = 8;
+constexpr int kMaxZPartsCombined = 4 * kCombineCluster;   // z partials per slot it can add
+constexpr int kCombineThreads = 256;
 
 struct CombineParams {
   Partition part;
@@ -31,12 +38,9 @@ struct CombineParams {
   const float* z_in;     // optional carried key sum (may alias z_out)
   float* S_out;          // [BH][d][d]
   float* z_out;          // [BH][d]
-  __half* S_img;         // optional [BH][d*d] swizzled fp16 image (d = 128)
-  float* S_rs;           // [BH][d] inverse row scales of the image
+  __half* S_img;         // optional [BH][128*128] swizzled fp16 image (d = 128)
+  float* S_scale;        // [BH][4]: [0] = scale of the image
 };
-
-constexpr int kCombineThreads = 256;
-constexpr int kCombineElems = 1024;  // state elements per CTA
 
 // Byte offset of S[a][c] (a = row = output feature, c = reduction index) in
 // the swizzled image of a 128 x 128 16-bit matrix.
@@ -47,53 +51,120 @@ __host__ __device__ inline uint32_t simg_offset(int a, int c) {
   return (uint32_t)(kb * 16384 + a * 128 + (((chunk ^ (a & 7)) << 4) | (byte_in_row & 15)));
 }
 
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineParams p) {
+__device__ __forceinline__ void add4(float4& s, const float4 t) {
+  s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
+}
+
+__global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombineThreads)
+    combine_kernel(CombineParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ float red[kCombineThreads / 32];
+  __shared__ float cta_max;
+
   const int bh = blockIdx.y;
+  const int rank = (int)cluster.block_rank();
   const int d = p.d;
   const long long tph = p.part.tiles_per_head;
   const int c_lo = part_cta_of(p.part, (long long)bh * tph);
   const int c_hi = part_cta_of(p.part, (long long)(bh + 1) * tph - 1);
   const size_t dd = (size_t)d * d;
-  const int e0 = blockIdx.x * kCombineElems;
+  const int chunk = (int)(dd / kCombineCluster);        // 2048 for d = 128
+  const int e_base = rank * chunk;
 
-  for (int e = e0 + threadIdx.x * 4; e < e0 + kCombineElems && e < (int)dd; e += kCombineThreads * 4) {
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (p.S_in) s = *reinterpret_cast<const float4*>(p.S_in + bh * dd + e);
-    for (int c = c_lo; c <= c_hi; ++c) {
-      const float4 t = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + bh) * dd + e);
-      s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
-    }
-    *reinterpret_cast<float4*>(p.S_out + bh * dd + e) = s;
-    if (p.S_img) {
-      // One warp holds one full row (d = 128: 32 threads x 4 elements).
-      float m = fmaxf(fmaxf(fabsf(s.x), fabsf(s.y)), fmaxf(fabsf(s.z), fabsf(s.w)));
+  // Each thread owns up to two float4 groups: e = e_base + 4*tid + 1024*k.
+  float4 acc[2];
+  float m = 0.f;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      // m = f * 2^E, f in [0.5, 1): scale by 2^(14 - E).
-      int E = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 126;
-      if (m == 0.f || E < -100) E = -100;
-      if (E > 140) E = 140;
-      const float sc = __uint_as_float((uint32_t)(127 + 14 - E) << 23);
-      const int a = e / d, cc = e % d;
-      if ((threadIdx.x & 31) == 0) p.S_rs[(size_t)bh * d + a] = __uint_as_float((uint32_t)(127 - 14 + E) << 23);
-      unsigned char* img = reinterpret_cast<unsigned char*>(p.S_img + bh * dd);
-      __half2 lo = __floats2half2_rn(s.x * sc, s.y * sc);
-      __half2 hi = __floats2half2_rn(s.z * sc, s.w * sc);
-      // c .. c+3 stay inside one 16-byte chunk (c is a multiple of 4).
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t*>(&lo);
-      pk.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(img + simg_offset(a, cc)) = pk;
+  for (int k = 0; k < 2; ++k) {
+    const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
+    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e >= e_base + chunk) continue;
+    if (p.S_in) acc[k] = *reinterpret_cast<const float4*>(p.S_in + bh * dd + e);
+    int c = c_lo;
+    // Issue four independent loads at a time; add them in slot order.
+    for (; c + 3 <= c_hi; c += 4) {
+      const float4 t0 = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + bh) * dd + e);
+      const float4 t1 = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + 1 + bh) * dd + e);
+      const float4 t2 = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + 2 + bh) * dd + e);
+      const float4 t3 = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + 3 + bh) * dd + e);
+      add4(acc[k], t0); add4(acc[k], t1); add4(acc[k], t2); add4(acc[k], t3);
     }
+    for (; c <= c_hi; ++c)
+      add4(acc[k], *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + bh) * dd + e));
+    *reinterpret_cast<float4*>(p.S_out + bh * dd + e) = acc[k];
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(acc[k].x), fabsf(acc[k].y)),
+                       fmaxf(fabsf(acc[k].z), fabsf(acc[k].w))));
   }
-  if (blockIdx.x == 0) {
+
+  // z: rank r sums the z partials r, r + 8, ... of every contributing slot
+  // (slot-major, in order); rank 0 then adds the ranks' sums in rank order.
+  __shared__ float zsum[128];
+  for (int e = threadIdx.x; e < d; e += kCombineThreads) {
+    float s = 0.f;
+    for (int c = c_lo; c <= c_hi; ++c) {
+      const float* zc = p.part_z + ((size_t)c + bh) * p.zparts * d + e;
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int zp = rank + kCombineCluster * k;
+        if (zp < p.zparts) t[k] = zc[(size_t)zp * d];
+      }
+      s += t[0]; s += t[1]; s += t[2]; s += t[3];
+    }
+    zsum[e] = s;
+  }
+  cluster.sync();
+  if (rank == 0) {
     for (int e = threadIdx.x; e < d; e += kCombineThreads) {
       float s = p.z_in ? p.z_in[(size_t)bh * d + e] : 0.f;
-      for (int c = c_lo; c <= c_hi; ++c)
-        for (int zp = 0; zp < p.zparts; ++zp)
-          s += p.part_z[(((size_t)c + bh) * p.zparts + zp) * d + e];
+      for (int r = 0; r < kCombineCluster; ++r) s += *cluster.map_shared_rank(&zsum[e], r);
       p.z_out[(size_t)bh * d + e] = s;
     }
+  }
+  cluster.sync();   // zsum of every rank stays valid until rank 0 has read it
+
+  if (p.S_img == nullptr) return;     // uniform over the whole grid
+
+  // Head maximum: warp, CTA, then the cluster through distributed smem.
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float mm = red[0];
+    for (int w = 1; w < kCombineThreads / 32; ++w) mm = fmaxf(mm, red[w]);
+    cta_max = mm;
+  }
+  cluster.sync();
+  float hm = 0.f;
+  for (int r = 0; r < kCombineCluster; ++r)
+    hm = fmaxf(hm, *cluster.map_shared_rank(&cta_max, r));
+  cluster.sync();   // no CTA leaves while others still read its cta_max
+
+  // hm = f * 2^E with f in [0.5, 1): scale by 2^(14 - E).
+  int E = (int)((__float_as_uint(hm) >> 23) & 0xFFu) - 126;
+  if (hm == 0.f || E < -100) E = -100;
+  if (E > 140) E = 140;
+  const float sc = __uint_as_float((uint32_t)(127 + 14 - E) << 23);
+  if (rank == 0 && threadIdx.x == 0) {
+    p.S_scale[(size_t)bh * 4 + 0] = sc;
+    p.S_scale[(size_t)bh * 4 + 1] = 0.f;
+    p.S_scale[(size_t)bh * 4 + 2] = 0.f;
+    p.S_scale[(size_t)bh * 4 + 3] = 0.f;
+  }
+  unsigned char* img = reinterpret_cast<unsigned char*>(p.S_img + bh * dd);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
+    if (e >= e_base + chunk) continue;
+    const int a = e / d, cc = e % d;
+    __half2 lo = __floats2half2_rn(acc[k].x * sc, acc[k].y * sc);
+    __half2 hi = __floats2half2_rn(acc[k].z * sc, acc[k].w * sc);
+    uint2 pk;   // cc .. cc+3 stay inside one 16-byte chunk (cc is a multiple of 4)
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(img + simg_offset(a, cc)) = pk;
   }
 }
 

@@ -18,6 +18,27 @@ enum : unsigned { kErrTimeout = 1u };
 
 // ----------------------------------------------------------------- geometry
 
+// Division by a runtime-invariant divisor d >= 1 for 0 <= n < 2^30:
+// q = (umulhi(n, m) + n) >> l with l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994, section 4).
+struct FastDiv {
+  uint32_t m, l, d;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.l = 0;
+  while ((1ull << f.l) < d) ++f.l;
+  f.m = (uint32_t)((((1ull << 32) * ((1ull << f.l) - d)) / d) + 1);
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.m) + n) >> f.l;
+}
+
 struct Geom {
   int B, Hh, d;          // batch, heads, head dim
   int T, H, W, N;        // latent grid of this call, N = T*H*W
@@ -26,6 +47,7 @@ struct Geom {
   int rope_on;           // 0: identity rotation
   float theta;           // RoPE base
   float eps;             // denominator epsilon
+  FastDiv div_HW, div_W; // n -> frame, n % HW -> row
 };
 
 __host__ __device__ inline void rope_split(int d, int* pt, int* ph, int* pw) {
@@ -78,13 +100,14 @@ inline Partition make_partition(int BH, int N, int tile, int max_grid) {
 // --------------------------------------------------------------- RoPE table
 //
 // Each CTA keeps cos/sin of the rotations it needs in shared memory, as float2
-// (cos, sin) entries:
-//   time axis:   pt pairs x Lt frames   (frames t_lo .. t_lo+Lt-1, wrapping
+// (cos, sin) entries, position-major inside each axis so that the pairs of one
+// position are adjacent:
+//   time axis:   [Lt frames][pt pairs]  (frames t_lo .. t_lo+Lt-1, wrapping
 //                                        modulo T when the CTA's tokens cross
 //                                        from the end of one head's sequence
 //                                        to the start of the next)
-//   height axis: ph pairs x H
-//   width axis:  pw pairs x W
+//   height axis: [H][ph]
+//   width axis:  [W][pw]
 // Angles are formed and evaluated in double precision, then rounded to fp32.
 
 struct RopeWindow {
@@ -129,19 +152,19 @@ __device__ inline void rope_build(float2* tab, const Geom& g, RopeWindow win, in
     int i, p;
     double pos;
     if (e < nt) {
-      i = e / win.Lt;
+      i = e % g.pt;
       p = g.pt;
-      int f = win.t_lo + e % win.Lt;
+      int f = win.t_lo + e / g.pt;
       if (f >= g.T) f -= g.T;
       pos = (double)(g.t0 + f);
     } else if (e < nt + nh) {
-      i = (e - nt) / g.H;
+      i = (e - nt) % g.ph;
       p = g.ph;
-      pos = (double)((e - nt) % g.H);
+      pos = (double)((e - nt) / g.ph);
     } else {
-      i = (e - nt - nh) / g.W;
+      i = (e - nt - nh) % g.pw;
       p = g.pw;
-      pos = (double)((e - nt - nh) % g.W);
+      pos = (double)((e - nt - nh) / g.pw);
     }
     const double ang = pos * exp(-((double)i / (double)p) * log_theta);
     double s, c;
@@ -157,10 +180,10 @@ __device__ inline int rope_index(const Geom& g, RopeWindow win, int pr, int f, i
   if (pr < g.pt) {
     int tl = f - win.t_lo;
     if (tl < 0) tl += g.T;
-    return pr * win.Lt + tl;
+    return tl * g.pt + pr;
   }
-  if (pr < g.pt + g.ph) return g.pt * win.Lt + (pr - g.pt) * g.H + hh;
-  return g.pt * win.Lt + g.ph * g.H + (pr - g.pt - g.ph) * g.W + ww;
+  if (pr < g.pt + g.ph) return g.pt * win.Lt + hh * g.ph + (pr - g.pt);
+  return g.pt * win.Lt + g.ph * g.H + ww * g.pw + (pr - g.pt - g.ph);
 }
 
 // ------------------------------------------------------------------ dtypes

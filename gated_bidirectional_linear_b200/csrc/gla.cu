@@ -26,7 +26,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 struct WsLayout {
-  size_t part_S, part_z, S, z, S_img, S_rs, total;
+  size_t part_S, part_z, S, z, S_img, S_scale, total;
   int slots;
 };
 
@@ -45,8 +45,8 @@ WsLayout ws_layout(int BH, int d, bool own_state) {
   }
   L.S_img = off;
   if (d == 128) off = align_up(off + (size_t)BH * d * d * 2, kAlign);
-  L.S_rs = off;
-  if (d == 128) off = align_up(off + (size_t)BH * d * 4, kAlign);
+  L.S_scale = off;
+  if (d == 128) off = align_up(off + (size_t)BH * 4 * 4, kAlign);
   L.total = off;
   return L;
 }
@@ -82,6 +82,8 @@ Geom make_geom(int batch, int heads, int head_dim, int T, int H, int W, int t0,
   g.rope_on = rope_theta > 0.f ? 1 : 0;
   g.theta = rope_theta;
   g.eps = eps;
+  g.div_HW = make_fastdiv((uint32_t)(H * W));
+  g.div_W = make_fastdiv((uint32_t)W);
   return g;
 }
 
@@ -127,8 +129,18 @@ inline cudaError_t mark(const Call& c, int i) {
   return cudaEventRecord(static_cast<cudaEvent_t>(c.events[i]), c.stream);
 }
 
-int resolve_path(int requested, int dtype, int d) {
-  const bool tensor_ok = dtype == GLA_DTYPE_BF16 && d == 128;
+// The tensor path keeps the RoPE table of each CTA in shared memory next to
+// its tile rings; grids whose table does not fit use the CUDA-core path.
+bool tensor_fits(const Geom& g, int sms) {
+  if (g.H >= (1 << kPosBits) || g.W >= (1 << kPosBits) || g.T >= (1 << kPosBits)) return false;
+  const Partition part = make_partition(g.B * g.Hh, g.N, kTcTile, sms);
+  const int tab = tc_table_entries(g, part);
+  return tc_state_smem(tab) <= kMaxSmem && tc_apply_smem(tab) <= kMaxSmem;
+}
+
+int resolve_path(int requested, int dtype, int d, const Geom* g = nullptr, int sms = 0) {
+  bool tensor_ok = dtype == GLA_DTYPE_BF16 && d == 128;
+  if (tensor_ok && requested == GLA_PATH_AUTO && g && sms > 0) tensor_ok = tensor_fits(*g, sms);
   if (requested == GLA_PATH_AUTO) return tensor_ok ? GLA_PATH_TENSOR : GLA_PATH_SIMT;
   if (requested == GLA_PATH_SIMT) return GLA_PATH_SIMT;
   if (requested == GLA_PATH_TENSOR) return tensor_ok ? GLA_PATH_TENSOR : -1;
@@ -166,8 +178,8 @@ gla_status run_simt(const Call& c) {
   cp.S_in = c.carry ? c.S : nullptr;
   cp.z_in = c.carry ? c.z : nullptr;
   cp.S_out = c.S; cp.z_out = c.z;
-  cp.S_img = nullptr; cp.S_rs = nullptr;
-  dim3 cgrid((D * D + kCombineElems - 1) / kCombineElems, g.B * g.Hh);
+  cp.S_img = nullptr; cp.S_scale = nullptr;
+  dim3 cgrid(kCombineCluster, g.B * g.Hh);
   combine_kernel<<<cgrid, kCombineThreads, 0, c.stream>>>(cp);
   if (cudaGetLastError() != cudaSuccess || mark(c, 2) != cudaSuccess) return GLA_ERR_CUDA;
 
@@ -201,7 +213,7 @@ gla_status run_call(Call& c) {
                     reinterpret_cast<float*>(c.ws + c.L.part_S),
                     reinterpret_cast<float*>(c.ws + c.L.part_z),
                     reinterpret_cast<__half*>(c.ws + c.L.S_img),
-                    reinterpret_cast<float*>(c.ws + c.L.S_rs), c.den_dbg, c.x_dbg,
+                    reinterpret_cast<float*>(c.ws + c.L.S_scale), c.den_dbg, c.x_dbg,
                     device_sm_count(), c.stream, c.events);
   } else {
     st = c.dtype == GLA_DTYPE_F32 ? run_simt_dtype<float>(c)
@@ -229,14 +241,15 @@ gla_status forward_common(const void* q, const void* k, const void* v, const voi
   const void* ptrs[6] = {q, k, v, beta, g, out};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
-  const int resolved = resolve_path(path, dtype, head_dim);
-  if (resolved < 0) return GLA_ERR_UNSUPPORTED;
+  if (resolve_path(path, dtype, head_dim) < 0) return GLA_ERR_UNSUPPORTED;
   const WsLayout L = ws_layout(batch * heads, head_dim, true);
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < L.total)
     return GLA_ERR_WORKSPACE;
   Call c;
   c.g = make_geom(batch, heads, head_dim, T, H, W, 0, rope_theta, eps);
-  c.dtype = dtype; c.path = resolved;
+  const int sms = device_sm_count();
+  if (sms <= 0) return GLA_ERR_CUDA;
+  c.dtype = dtype; c.path = resolve_path(path, dtype, head_dim, &c.g, sms);
   c.q = q; c.k = k; c.v = v; c.beta = beta; c.gate = g; c.out = out;
   c.ws = static_cast<unsigned char*>(workspace);
   c.L = L;
@@ -331,14 +344,15 @@ gla_status gla_block_causal_step_ex(float* state, float* z, const void* q, const
   const void* ptrs[8] = {state, z, q, k, v, beta, g, out};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
-  const int resolved = resolve_path(path, dtype, head_dim);
-  if (resolved < 0) return GLA_ERR_UNSUPPORTED;
+  if (resolve_path(path, dtype, head_dim) < 0) return GLA_ERR_UNSUPPORTED;
   const WsLayout L = ws_layout(batch * heads, head_dim, false);
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < L.total)
     return GLA_ERR_WORKSPACE;
   Call c;
   c.g = make_geom(batch, heads, head_dim, T_blk, H, W, t0, rope_theta, eps);
-  c.dtype = dtype; c.path = resolved;
+  const int sms = device_sm_count();
+  if (sms <= 0) return GLA_ERR_CUDA;
+  c.dtype = dtype; c.path = resolve_path(path, dtype, head_dim, &c.g, sms);
   c.q = q; c.k = k; c.v = v; c.beta = beta; c.gate = g; c.out = out;
   c.ws = static_cast<unsigned char*>(workspace);
   c.L = L;
@@ -425,7 +439,8 @@ gla_status gla_plan(int batch, int heads, int head_dim, int T, int H, int W, int
   if (!dims_ok(batch, heads, head_dim, T, H, W) || num_sms <= 0) return GLA_ERR_INVALID_ARG;
   if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
   if (!grid || !tile_tokens || !path_used) return GLA_ERR_INVALID_ARG;
-  const int resolved = resolve_path(path, dtype, head_dim);
+  const Geom g = make_geom(batch, heads, head_dim, T, H, W, 0, 10000.f, 1e-6f);
+  const int resolved = resolve_path(path, dtype, head_dim, &g, num_sms);
   if (resolved < 0) return GLA_ERR_UNSUPPORTED;
   const int N = T * H * W;
   Partition p = resolved == GLA_PATH_TENSOR

@@ -34,16 +34,19 @@ constexpr int kPosBits = 11;                 // packed (t, h, w) offsets, < 2048
 // --------------------------------------------------------------- state kernel
 
 constexpr int kStStages = 3;
-constexpr int kStTW = 8;                     // transform warps
-constexpr int kStTW0 = 6;                    // first transform warp
-constexpr int kStEW0 = 2;                    // epilogue warps 2..5
+constexpr int kStTW = 12;                    // transform warps; the first four
+                                             // also drain finished S partials
+constexpr int kStTW0 = 2;                    // first transform warp
 constexpr int kStThreads = (kStTW0 + kStTW) * 32;
+static_assert(kStTW <= kMaxZPartsCombined, "combine adds at most this many z partials");
+static_assert((kStTW * 4) % 8 == 0, "rows per pass keep the 8-row swizzle phase");
 constexpr int kStRowsPerPass = kStTW * 4;
 
 struct TcStateSmem {
   static constexpr uint32_t K = 0;
   static constexpr uint32_t V = kStStages * kTileBytes;
-  static constexpr uint32_t BAR = 2 * kStStages * kTileBytes;         // barriers
+  static constexpr uint32_t ROWPOS = 2 * kStStages * kTileBytes;      // [stage][128] uint2
+  static constexpr uint32_t BAR = ROWPOS + kStStages * 1024;          // barriers
   static constexpr uint32_t NBAR = 3 * kStStages + 5;
   static constexpr uint32_t MISC = BAR + NBAR * 8;                     // tmem base, abort
   static constexpr uint32_t TAB = (MISC + 16 + 15) & ~15u;              // RoPE table
@@ -65,43 +68,76 @@ __device__ __forceinline__ bool seg_last(const Partition& p, long long w, long l
   return w == we - 1 || ((w + 1) % p.tiles_per_head) == 0;
 }
 
-// Per-lane rotation-pair lookup: lane j of a row group handles channels
-// 16j .. 16j+15, i.e. pairs 8j .. 8j+7.
-struct PairInfo {
-  int base[8];
-  int shift[8];
-};
-
-__device__ __forceinline__ void pair_info(const Geom& g, RopeWindow win, int j, PairInfo& pi) {
+// Per-tile row metadata.  For every row r of a tile (token n0 + r) the
+// producer warp stores the byte offsets, inside the RoPE table, of the token's
+// time, height and width rows: (offT | offH << 16, offW).  The table is at
+// most 22.5 KB, so 16 bits hold each offset.
+__device__ __forceinline__ void tile_rowpos(const Geom& g, RopeWindow win, int n0, int lane,
+                                            uint2* rowpos) {
+  const uint32_t HW = g.div_HW.d, W = g.div_W.d;
+  const uint32_t baseH = (uint32_t)(g.pt * win.Lt), baseW = baseH + (uint32_t)(g.ph * g.H);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int p = 8 * j + i;
-    if (p < g.pt) {
-      pi.base[i] = p * win.Lt;
-      pi.shift[i] = 0;
-    } else if (p < g.pt + g.ph) {
-      pi.base[i] = g.pt * win.Lt + (p - g.pt) * g.H;
-      pi.shift[i] = kPosBits;
-    } else {
-      pi.base[i] = g.pt * win.Lt + g.ph * g.H + (p - g.pt - g.ph) * g.W;
-      pi.shift[i] = 2 * kPosBits;
-    }
+  for (int k = 0; k < 4; ++k) {
+    const int r = lane + 32 * k;
+    int n = n0 + r;
+    if (n >= g.N) n = n0;
+    const uint32_t f = fdiv((uint32_t)n, g.div_HW);
+    const uint32_t rem = (uint32_t)n - f * HW;
+    const uint32_t hh = fdiv(rem, g.div_W);
+    const uint32_t ww = rem - hh * W;
+    int tl = (int)f - win.t_lo;
+    if (tl < 0) tl += g.T;
+    const uint32_t offT = 8u * (uint32_t)(tl * g.pt);
+    const uint32_t offH = 8u * (baseH + hh * (uint32_t)g.ph);
+    const uint32_t offW = 8u * (baseW + ww * (uint32_t)g.pw);
+    rowpos[r] = make_uint2(offT | (offH << 16), offW);
   }
 }
 
-__device__ __forceinline__ uint32_t packed_pos(const Geom& g, RopeWindow win, int n) {
-  const int HW = g.H * g.W;
-  const int f = n / HW;
-  const int rem = n - f * HW;
-  const int hh = rem / g.W;
-  const int ww = rem - hh * g.W;
-  int tl = f - win.t_lo;
-  if (tl < 0) tl += g.T;
-  return (uint32_t)tl | ((uint32_t)hh << kPosBits) | ((uint32_t)ww << (2 * kPosBits));
+// Per-lane view of the RoPE table.  Lane j of a row group handles channels
+// 16j .. 16j+15, i.e. rotation pairs 8j .. 8j+7; for d = 128 every axis has at
+// least 21 pairs, so those 8 pairs lie on at most two axes A and B.  With the
+// position-major table, pair i of the lane sits at byte
+//   offA(row) + inA + 8 i   (pairs on axis A)
+//   offB(row) + inB + 8 i   (pairs on axis B, useB[i] = 1)
+// where offX(row) is the row's metadata for axis X.
+struct LaneRope {
+  int inA, inB;          // byte offset of pair p0 = 8j inside its axis row
+  int wA, shA, wB, shB;  // where offA / offB sit in the row metadata
+  int useB[8];
+};
+
+__device__ __forceinline__ int axis_of(const Geom& g, int p) {
+  return p < g.pt ? 0 : (p < g.pt + g.ph ? 1 : 2);
+}
+
+__device__ __forceinline__ void lane_rope(const Geom& g, int j, LaneRope& lr) {
+  const int p0 = 8 * j;
+  const int start[3] = {0, g.pt, g.pt + g.ph};
+  const int aA = axis_of(g, p0), aB = axis_of(g, p0 + 7);
+  lr.inA = 8 * (p0 - start[aA]);
+  lr.inB = 8 * (p0 - start[aB]);
+  lr.wA = aA == 2 ? 1 : 0;
+  lr.shA = aA == 1 ? 16 : 0;
+  lr.wB = aB == 2 ? 1 : 0;
+  lr.shB = aB == 1 ? 16 : 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) lr.useB[i] = axis_of(g, p0 + i) != aA ? 1 : 0;
+}
+
+// Table pointer of the lane's pair 0 for a row, and the entry distance from
+// its axis-A run to its axis-B run.
+__device__ __forceinline__ void lane_rope_row(const LaneRope& lr, const float2* tab, uint2 m,
+                                              const float2*& pA, int& dE) {
+  const uint32_t offA = ((lr.wA ? m.y : m.x) >> lr.shA) & 0xFFFFu;
+  const uint32_t offB = ((lr.wB ? m.y : m.x) >> lr.shB) & 0xFFFFu;
+  const int bA = (int)offA + lr.inA, bB = (int)offB + lr.inB;
+  pA = reinterpret_cast<const float2*>(reinterpret_cast<const char*>(tab) + bA);
+  dE = (bB - bA) >> 3;
 }
 
 // Shared-memory addresses of the two 16-byte chunks a lane owns in row r of a
-// 128x128 bf16 tile stored as two 128-byte-swizzled boxes.
+// 128x128 16-bit tile stored as two 128-byte-swizzled boxes.
 __device__ __forceinline__ void lane_chunks(uint32_t tile, int r, int j, uint32_t& a0,
                                             uint32_t& a1) {
   const uint32_t row = tile + (uint32_t)(j >> 2) * kBox + (uint32_t)r * 128u;
@@ -110,43 +146,52 @@ __device__ __forceinline__ void lane_chunks(uint32_t tile, int r, int j, uint32_
   a1 = row + (((c0 + 1) ^ (uint32_t)(r & 7)) << 4);
 }
 
-__device__ __forceinline__ void unpack16(uint4 a, uint4 b, float (&x)[16]) {
-  x[0] = bf_lo(a.x); x[1] = bf_hi(a.x); x[2] = bf_lo(a.y); x[3] = bf_hi(a.y);
-  x[4] = bf_lo(a.z); x[5] = bf_hi(a.z); x[6] = bf_lo(a.w); x[7] = bf_hi(a.w);
-  x[8] = bf_lo(b.x); x[9] = bf_hi(b.x); x[10] = bf_lo(b.y); x[11] = bf_hi(b.y);
-  x[12] = bf_lo(b.z); x[13] = bf_hi(b.z); x[14] = bf_lo(b.w); x[15] = bf_hi(b.w);
+// The lane's 16 elements of a row as 8 fp32 pairs (channels 2i, 2i+1).
+__device__ __forceinline__ void unpack8(uint4 a, uint4 b, f2_t (&x)[8]) {
+  x[0] = f2_bf(a.x); x[1] = f2_bf(a.y); x[2] = f2_bf(a.z); x[3] = f2_bf(a.w);
+  x[4] = f2_bf(b.x); x[5] = f2_bf(b.y); x[6] = f2_bf(b.z); x[7] = f2_bf(b.w);
 }
 
-// RMSNorm + ReLU of one row shared by the 8 lanes of a row group.
-__device__ __forceinline__ void norm_relu16(float (&x)[16]) {
-  float ss = 0.f;
+// 1/RMS of a row whose 128 elements are spread over the 8 lanes of a group.
+__device__ __forceinline__ float row_rstd(const f2_t (&x)[8]) {
+  f2_t ss = 0ull;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) ss = fmaf(x[i], x[i], ss);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-  const float rstd = rsqrtf(ss * (1.f / 128.f) + kRmsEps);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) x[i] = fmaxf(x[i] * rstd, 0.f);
+  for (int i = 0; i < 8; ++i) ss = f2_fma(x[i], x[i], ss);
+  float s = f2_lo(ss) + f2_hi(ss);
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 4);
+  return rsqrtf(s * (1.f / 128.f) + kRmsEps);
 }
 
-// y = scale * RoPE(x) for the lane's 8 pairs, packed to bf16 (or fp16).
+__device__ __forceinline__ f2_t f2_relu(f2_t x) {
+  return f2(fmaxf(f2_lo(x), 0.f), fmaxf(f2_hi(x), 0.f));
+}
+
+// Rotate the lane's 8 ReLU'd pairs r (still unnormalised), scaled by `scl`:
+// y = scl * RoPE(r), packed to bf16 (kHalf = false) or fp16.
 template <bool kHalf>
-__device__ __forceinline__ void rope_pack16(const Geom& g, const float2* tab, const PairInfo& pi,
-                                            uint32_t opk, const float (&x)[16], float scale,
-                                            uint4& o0, uint4& o1) {
+__device__ __forceinline__ void rope_scale_pack(const Geom& g, const LaneRope& lr,
+                                                const float2* pA, int dE,
+                                                const f2_t (&r)[8], float scl, uint4& o0,
+                                                uint4& o1) {
   uint32_t w[8];
+  const f2_t scl2 = f2(scl, scl);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    float y0 = x[2 * i], y1 = x[2 * i + 1];
+    const float r0 = f2_lo(r[i]), r1 = f2_hi(r[i]);
+    float y0, y1;
     if (g.rope_on) {
-      const float2 cs = tab[pi.base[i] + (int)((opk >> pi.shift[i]) & ((1u << kPosBits) - 1))];
-      const float r0 = fmaf(-y1, cs.y, y0 * cs.x);
-      const float r1 = fmaf(y1, cs.x, y0 * cs.y);
-      y0 = r0;
-      y1 = r1;
+      const float2 e = pA[lr.useB[i] * dE + i];
+      const f2_t cs = f2_mul(f2(e.x, e.y), scl2);
+      const float c = f2_lo(cs), sn = f2_hi(cs);
+      y0 = fmaf(-r1, sn, r0 * c);
+      y1 = fmaf(r1, c, r0 * sn);
+    } else {
+      y0 = r0 * scl;
+      y1 = r1 * scl;
     }
-    w[i] = kHalf ? pack_f16(y0 * scale, y1 * scale) : pack_bf16(y0 * scale, y1 * scale);
+    w[i] = kHalf ? pack_f16(y0, y1) : pack_bf16(y0, y1);
   }
   o0 = make_uint4(w[0], w[1], w[2], w[3]);
   o1 = make_uint4(w[4], w[5], w[6], w[7]);
@@ -204,7 +249,8 @@ __global__ void __launch_bounds__(kStThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // All lanes compute the tile's row metadata; lane 0 issues the copies.
+    {
       const uint64_t pol = policy_evict_first();
       long long it = 0;
       int issued = 0;
@@ -214,8 +260,11 @@ __global__ void __launch_bounds__(kStThreads, 1)
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
         const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
         const int n0 = (int)(w % tph) * kTcTile;
-        mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
-        unsigned char* kt = sm + TcStateSmem::K + s * kTileBytes;
+        if (g.rope_on)
+          tile_rowpos(g, win, n0, lane, reinterpret_cast<uint2*>(sm + TcStateSmem::ROWPOS + s * 1024));
+        __syncwarp();
+        if (lane != 0) { ++issued; continue; }
+        mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);        unsigned char* kt = sm + TcStateSmem::K + s * kTileBytes;
         unsigned char* vt = sm + TcStateSmem::V + s * kTileBytes;
         tma_load_3d(kt, &tmK, &full[s], h * 128, n0, b, pol);
         tma_load_3d(kt + kBox, &tmK, &full[s], h * 128 + 64, n0, b, pol);
@@ -223,7 +272,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
         tma_load_3d(vt + kBox, &tmV, &full[s], h * 128 + 64, n0, b, pol);
         ++issued;
       }
-      if (*abort_flag) {
+      if (*abort_flag && lane == 0) {
         // Let every load in flight land before shared memory is released.
         long long first = it - (issued < kStStages ? issued : kStStages);
         for (long long i2 = first; i2 < it; ++i2) {
@@ -267,43 +316,22 @@ __global__ void __launch_bounds__(kStThreads, 1)
       int dummy = 0;
       mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy));
     }
-  } else if (warp < kStTW0) {
-    // ------------------------------------------------ epilogue: S partials
-    const int q4 = warp & 3;
-    const int a = q4 * 32 + lane;
-    int seg = 0;
-    for (long long w = wb; w < we; ++w) {
-      if (!seg_last(part, w, we)) continue;
-      const int bh = (int)(w / tph);
-      const int ab = seg & 1;
-      if (!mbar_wait(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag)) break;
-      tc_fence_after();
-      float* dst = p.part_S + ((size_t)c + bh) * 128 * 128 + (size_t)a * 128;
-#pragma unroll 1
-      for (int cb = 0; cb < 4; ++cb) {
-        float r[32];
-        tmem_ld32(tmem + (uint32_t)(ab * 128 + cb * 32) + ((uint32_t)(q4 * 32) << 16), r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(dst + cb * 32 + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[ab]);
-      ++seg;
-    }
   } else {
     // ------------------------------------------- transform warps: k -> beta k_til
     const int tw = warp - kStTW0;
     const int rg = lane >> 3, j = lane & 7;
-    PairInfo pi;
-    pair_info(g, win, j, pi);
+    LaneRope lr;
+    lane_rope(g, j, lr);
     const uint64_t pol_beta = policy_evict_last();
-    float zacc[16];
+    // This lane's two 16-byte chunks in row (tw*4 + rg) of a tile; rows of later
+    // passes add whole multiples of 8 rows, which keeps the swizzle phase.
+    uint32_t ch0, ch1;
+    lane_chunks(0, tw * 4 + rg, j, ch0, ch1);
+    f2_t zacc[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) zacc[i] = 0.f;
+    for (int i = 0; i < 8; ++i) zacc[i] = 0ull;
     long long it = 0;
+    int seg = 0;
     bool ok = true;
     for (long long w = wb; w < we && ok; ++w, ++it) {
       const int s = (int)(it % kStStages);
@@ -311,32 +339,40 @@ __global__ void __launch_bounds__(kStThreads, 1)
       const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
       const int n0 = (int)(w % tph) * kTcTile;
       constexpr int kPasses = (kTcTile + kStRowsPerPass - 1) / kStRowsPerPass;
-      float be[kPasses];
+      static_assert(kPasses <= 4, "beta prefetch holds four rows");
+      float be[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ps = 0; ps < kPasses; ++ps) {
         const int n = n0 + ps * kStRowsPerPass + tw * 4 + rg;
-        be[ps] = 0.f;
-        if (n < g.N) {
+        if (n < g.N && ps * kStRowsPerPass + tw * 4 < kTcTile) {
           const uint16_t raw = ld_u16_policy(p.beta + ((size_t)b * g.N + n) * g.Hh + h, pol_beta);
           be[ps] = __uint_as_float((uint32_t)raw << 16);
         }
       }
       if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
       const uint32_t kt = sbase + TcStateSmem::K + s * kTileBytes;
-#pragma unroll
+#pragma unroll 1
       for (int ps = 0; ps < kPasses; ++ps) {
         const int r = ps * kStRowsPerPass + tw * 4 + rg;
-        const int n = n0 + r;
-        uint32_t a0, a1;
-        lane_chunks(kt, r, j, a0, a1);
-        float x[16];
-        unpack16(lds128(a0), lds128(a1), x);
-        norm_relu16(x);
+        if (ps * kStRowsPerPass + tw * 4 >= kTcTile) break;
+        const float bcur = ps == 0 ? be[0] : (ps == 1 ? be[1] : (ps == 2 ? be[2] : be[3]));
+        const uint32_t a0 = kt + ch0 + ps * kStRowsPerPass * 128;
+        const uint32_t a1 = kt + ch1 + ps * kStRowsPerPass * 128;
+        const float2* pA = tab;
+        int dE = 0;
+        if (g.rope_on)
+          lane_rope_row(lr, tab, reinterpret_cast<const uint2*>(sm + TcStateSmem::ROWPOS + s * 1024)[r], pA, dE);
+        f2_t x[8];
+        unpack8(lds128(a0), lds128(a1), x);
+        const float rstd = row_rstd(x);
+        const f2_t rstd2 = f2(rstd, rstd);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) zacc[i] += x[i];
-        const uint32_t opk = packed_pos(g, win, n < g.N ? n : n0);
+        for (int i = 0; i < 8; ++i) {
+          x[i] = f2_relu(x[i]);                     // ReLU before the (positive) scale
+          zacc[i] = f2_fma(x[i], rstd2, zacc[i]);   // z += k_pls
+        }
         uint4 o0, o1;
-        rope_pack16<false>(g, tab, pi, opk, x, be[ps], o0, o1);
+        rope_scale_pack<false>(g, lr, pA, dE, x, rstd * bcur, o0, o1);
         sts128(a0, o0);
         sts128(a1, o1);
       }
@@ -347,19 +383,50 @@ __global__ void __launch_bounds__(kStThreads, 1)
       if (seg_last(part, w, we)) {
         // z of this head segment: sum the warp's four row groups, then store
         // one partial per warp (the combine adds them in warp order).
+        float zf[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          zf[2 * i] = f2_lo(zacc[i]);
+          zf[2 * i + 1] = f2_hi(zacc[i]);
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          zacc[i] += __shfl_xor_sync(0xffffffffu, zacc[i], 8);
-          zacc[i] += __shfl_xor_sync(0xffffffffu, zacc[i], 16);
+          zf[i] += __shfl_xor_sync(0xffffffffu, zf[i], 8);
+          zf[i] += __shfl_xor_sync(0xffffffffu, zf[i], 16);
         }
         if (rg == 0) {
           float* zd = p.part_z + (((size_t)c + bh) * kStTW + tw) * 128 + 16 * j;
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(zd + i) = make_float4(zacc[i], zacc[i + 1], zacc[i + 2], zacc[i + 3]);
+            *reinterpret_cast<float4*>(zd + i) = make_float4(zf[i], zf[i + 1], zf[i + 2], zf[i + 3]);
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) zacc[i] = 0.f;
+        for (int i = 0; i < 8; ++i) zacc[i] = 0ull;
+
+        // Warps tw = 0..3 (one per TMEM lane quarter) drain the finished
+        // accumulator: row a of the partial S is TMEM lane a.
+        if (tw < 4) {
+          const int q4 = warp & 3;
+          const int a = q4 * 32 + lane;
+          const int ab = seg & 1;
+          if (!mbar_wait(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          float* dst = p.part_S + ((size_t)c + bh) * 128 * 128 + (size_t)a * 128;
+#pragma unroll 1
+          for (int cb = 0; cb < 4; ++cb) {
+            float rr[32];
+            tmem_ld32(tmem + (uint32_t)(ab * 128 + cb * 32) + ((uint32_t)(q4 * 32) << 16), rr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + cb * 32 + i) =
+                  make_float4(rr[i], rr[i + 1], rr[i + 2], rr[i + 3]);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&accempty[ab]);
+        }
+        ++seg;
       }
     }
   }
@@ -389,11 +456,11 @@ struct TcApplySmem {
   static constexpr uint32_t Q = 0;
   static constexpr uint32_t G = kApQ * kTileBytes;
   static constexpr uint32_t SIMG = G + kApG * kTileBytes;
-  static constexpr uint32_t Z = SIMG + kTileBytes;
-  static constexpr uint32_t RS = Z + 512;
-  static constexpr uint32_t DEN = RS + 512;                 // [kApDen][128] den per tile
-  static constexpr uint32_t RSR = DEN + kApDen * 512;       // [kApDen][128] row scales per tile
-  static constexpr uint32_t BAR = RSR + kApDen * 512;
+  static constexpr uint32_t Z = SIMG + kTileBytes;         // z [128] f32
+  static constexpr uint32_t SCL = Z + 512;                  // image scale [4] f32
+  static constexpr uint32_t DEN = SCL + 16;                 // [kApDen][128] den*scale per tile
+  static constexpr uint32_t ROWPOS = DEN + kApDen * 512;    // [q slot][128] uint2
+  static constexpr uint32_t BAR = ROWPOS + kApQ * 1024;
   static constexpr uint32_t NBAR = 3 * kApQ + 2 * kApG + 2 * kApAcc + 3;
   static constexpr uint32_t MISC = BAR + NBAR * 8;
   static constexpr uint32_t TAB = (MISC + 16 + 15) & ~15u;
@@ -402,8 +469,8 @@ struct TcApplySmem {
 struct TcApplyParams {
   Geom g;
   Partition part;
-  const __half* S_img;         // [BH][128*128] swizzled fp16 image of S (row-scaled)
-  const float* S_rs;           // [BH][128] inverse row scales of the image
+  const __half* S_img;         // [BH][128*128] swizzled fp16 image of S * scale
+  const float* S_scale;        // [BH][4]: [0] = scale of the image
   const float* z;              // [BH][128]
   float* den_out;              // optional
   float* x_out;                // optional
@@ -432,9 +499,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + TcApplySmem::MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + TcApplySmem::MISC + 4);
   float* zs = reinterpret_cast<float*>(sm + TcApplySmem::Z);
-  const float* rs = reinterpret_cast<const float*>(sm + TcApplySmem::RS);
+  const float* scl_s = reinterpret_cast<const float*>(sm + TcApplySmem::SCL);
   float* den_ring = reinterpret_cast<float*>(sm + TcApplySmem::DEN);
-  float* rs_ring = reinterpret_cast<float*>(sm + TcApplySmem::RSR);
   float2* tab = reinterpret_cast<float2*>(sm + TcApplySmem::TAB);
 
   const Geom& g = p.g;
@@ -479,31 +545,39 @@ __global__ void __launch_bounds__(kApThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------- producer: S image + q
-    if (lane == 0) {
+    // All lanes compute the tile's row metadata; lane 0 issues the copies.
+    {
       const uint64_t pol = policy_evict_first();
       long long it = 0;
       int seg = 0, issued = 0;
       for (long long w = wb; w < we; ++w, ++it) {
         const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
         if (seg_first(part, w, wb)) {
+          // Every lane waits, so the warp leaves the loop together on a timeout.
           if (!mbar_wait(sfree, (uint32_t)((seg & 1) ^ 1), abort_flag)) break;
-          mbar_arrive_expect_tx(sfull, kTileBytes + 1024);
-          bulk_load(sm + TcApplySmem::SIMG, p.S_img + (size_t)bh * 128 * 128, kTileBytes, sfull);
-          bulk_load(sm + TcApplySmem::Z, p.z + (size_t)bh * 128, 512, sfull);
-          bulk_load(sm + TcApplySmem::RS, p.S_rs + (size_t)bh * 128, 512, sfull);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(sfull, kTileBytes + 512 + 16);
+            bulk_load(sm + TcApplySmem::SIMG, p.S_img + (size_t)bh * 128 * 128, kTileBytes, sfull);
+            bulk_load(sm + TcApplySmem::Z, p.z + (size_t)bh * 128, 512, sfull);
+            bulk_load(sm + TcApplySmem::SCL, p.S_scale + (size_t)bh * 4, 16, sfull);
+          }
           ++seg;
         }
         const int s = (int)(it % kApQ);
         const uint32_t ph = (uint32_t)((it / kApQ) & 1);
         if (!mbar_wait(&qempty[s], ph ^ 1u, abort_flag)) break;
         const int n0 = (int)(w % tph) * kTcTile;
+        if (g.rope_on)
+          tile_rowpos(g, win, n0, lane, reinterpret_cast<uint2*>(sm + TcApplySmem::ROWPOS + s * 1024));
+        __syncwarp();
+        if (lane != 0) { ++issued; continue; }
         mbar_arrive_expect_tx(&qfull[s], kTileBytes);
         unsigned char* qt = sm + TcApplySmem::Q + s * kTileBytes;
         tma_load_3d(qt, &tmQ, &qfull[s], h * 128, n0, b, pol);
         tma_load_3d(qt + kBox, &tmQ, &qfull[s], h * 128 + 64, n0, b, pol);
         ++issued;
       }
-      if (*abort_flag) {
+      if (*abort_flag && lane == 0) {
         long long first = it - (issued < kApQ ? issued : kApQ);
         for (long long i2 = first; i2 < it; ++i2) {
           int dummy = 0;
@@ -581,9 +655,12 @@ __global__ void __launch_bounds__(kApThreads, 1)
     // ------------------------------------ transform warps: q -> q_til, den
     const int tw = warp - kApTW0;
     const int rg = lane >> 3, j = lane & 7;
-    PairInfo pi;
-    pair_info(g, win, j, pi);
-    float zr[16];
+    LaneRope lr;
+    lane_rope(g, j, lr);
+    uint32_t ch0, ch1;
+    lane_chunks(0, tw * 4 + rg, j, ch0, ch1);
+    f2_t zr[8];
+    float hscale = 1.f;
     long long it = 0;
     int seg = 0;
     for (long long w = wb; w < we; ++w, ++it) {
@@ -591,7 +668,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
       if (seg_first(part, w, wb)) {
         if (!mbar_wait(sfull, (uint32_t)(seg & 1), abort_flag)) break;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) zr[i] = zs[16 * j + i];
+        for (int i = 0; i < 8; ++i) zr[i] = f2(zs[16 * j + 2 * i], zs[16 * j + 2 * i + 1]);
+        hscale = scl_s[0];
         ++seg;
       }
       const int s = (int)(it % kApQ);
@@ -604,32 +682,36 @@ __global__ void __launch_bounds__(kApThreads, 1)
       for (int ps = 0; ps < kTcTile / kApRowsPerPass; ++ps) {
         const int r = ps * kApRowsPerPass + tw * 4 + rg;
         const int n = n0 + r;
-        uint32_t a0, a1;
-        lane_chunks(qt, r, j, a0, a1);
-        float x[16];
-        unpack16(lds128(a0), lds128(a1), x);
-        norm_relu16(x);
-        float dp = 0.f;
+        const uint32_t a0 = qt + ch0 + ps * kApRowsPerPass * 128;
+        const uint32_t a1 = qt + ch1 + ps * kApRowsPerPass * 128;
+        const float2* pA = tab;
+        int dE = 0;
+        if (g.rope_on)
+          lane_rope_row(lr, tab, reinterpret_cast<const uint2*>(sm + TcApplySmem::ROWPOS + s * 1024)[r], pA, dE);
+        f2_t x[8];
+        unpack8(lds128(a0), lds128(a1), x);
+        const float rstd = row_rstd(x);
+        f2_t dp2 = 0ull;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dp = fmaf(zr[i], x[i], dp);
+        for (int i = 0; i < 8; ++i) {
+          x[i] = f2_relu(x[i]);
+          dp2 = f2_fma(zr[i], x[i], dp2);
+        }
+        uint4 o0, o1;
+        rope_scale_pack<true>(g, lr, pA, dE, x, rstd, o0, o1);
+        sts128(a0, o0);
+        sts128(a1, o1);
+        float dp = f2_lo(dp2) + f2_hi(dp2);
         dp += __shfl_xor_sync(0xffffffffu, dp, 1);
         dp += __shfl_xor_sync(0xffffffffu, dp, 2);
         dp += __shfl_xor_sync(0xffffffffu, dp, 4);
-        const float dn = dp + g.eps;
-        const uint32_t opk = packed_pos(g, win, n < g.N ? n : n0);
-        uint4 o0, o1;
-        rope_pack16<true>(g, tab, pi, opk, x, 1.f, o0, o1);
-        sts128(a0, o0);
-        sts128(a1, o1);
+        const float dn = fmaf(dp, rstd, g.eps);      // z . q_pls + eps
         if (j == 0) {
-          den[r] = dn;
+          // The read-out sees S * scale; fold the scale into the denominator.
+          den[r] = dn * hscale;
           if (kDebug && p.den_out && n < g.N) p.den_out[((size_t)b * g.N + n) * g.Hh + h] = dn;
         }
       }
-      // The epilogue of this tile reads the row scales of S from this ring
-      // slot, which (like den) stays untouched until that epilogue is done;
-      // the shared copy at RS may meanwhile be replaced by the next head's.
-      if (lane < 16) rs_ring[(it % kApDen) * 128 + tw * 16 + lane] = rs[tw * 16 + lane];
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&qready[s]);
@@ -653,13 +735,14 @@ __global__ void __launch_bounds__(kApThreads, 1)
       const int gsl = (int)(it % kApG);
       const uint32_t gph = (uint32_t)((it / kApG) & 1);
       if (!mbar_wait(&gfull[gsl], gph, abort_flag)) break;
-      const float inv_den = 1.f / den_ring[(it % kApDen) * 128 + row];
-      const float* rsc = rs_ring + (it % kApDen) * 128;
+      // sigma(g) / den' = (0.5 tanh(g/2) + 0.5) / den' = fma(hc, tanh(g/2), hc)
+      const float hc = 0.5f / den_ring[(it % kApDen) * 128 + row];
       const uint32_t taddr = tmem + (uint32_t)(grp * 128) + ((uint32_t)(q4 * 32) << 16);
       const uint32_t gt = sbase + TcApplySmem::G + gsl * kTileBytes;
       const uint32_t grow = gt + (uint32_t)row * 128u;
       const uint32_t sw = (uint32_t)(row & 7);
-      float ss = 0.f;
+      const f2_t hc2 = f2(hc, hc), half2 = f2(0.5f, 0.5f);
+      f2_t ss2 = 0ull;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         float u[32];
@@ -674,16 +757,13 @@ __global__ void __launch_bounds__(kApThreads, 1)
           const uint32_t wv[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float g0 = bf_lo(wv[e]), g1 = bf_hi(wv[e]);
-            const float s0 = __fdividef(1.f, 1.f + __expf(-g0));
-            const float s1 = __fdividef(1.f, 1.f + __expf(-g1));
-            const int col = cb * 32 + q * 8 + 2 * e;
-            float& x0 = u[q * 8 + 2 * e];
-            float& x1 = u[q * 8 + 2 * e + 1];
-            x0 = (s0 * inv_den) * (x0 * rsc[col]);
-            x1 = (s1 * inv_den) * (x1 * rsc[col + 1]);
-            ss = fmaf(x0, x0, ss);
-            ss = fmaf(x1, x1, ss);
+            const f2_t hg = f2_mul(f2_bf(wv[e]), half2);
+            const f2_t t = f2(tanh_approx(f2_lo(hg)), tanh_approx(f2_hi(hg)));
+            const f2_t sg = f2_fma(hc2, t, hc2);   // sigmoid(g) / den'
+            const f2_t x = f2_mul(sg, f2(u[q * 8 + 2 * e], u[q * 8 + 2 * e + 1]));
+            ss2 = f2_fma(x, x, ss2);
+            u[q * 8 + 2 * e] = f2_lo(x);
+            u[q * 8 + 2 * e + 1] = f2_hi(x);
           }
         }
         if (kDebug && p.x_out && n0 + row < g.N) {
@@ -695,7 +775,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
         tmem_st32(taddr + cb * 32, u);
       }
       tmem_wait_st();
-      const float rstd = rsqrtf(ss * (1.f / 128.f) + kRmsEps);
+      const float rstd = rsqrtf((f2_lo(ss2) + f2_hi(ss2)) * (1.f / 128.f) + kRmsEps);
+      const f2_t rstd2 = f2(rstd, rstd);
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {
         float x[32];
@@ -704,12 +785,13 @@ __global__ void __launch_bounds__(kApThreads, 1)
         const uint32_t rbase = grow + (uint32_t)(cb >> 1) * kBox;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint4 o;
-          o.x = pack_bf16(x[q * 8 + 0] * rstd, x[q * 8 + 1] * rstd);
-          o.y = pack_bf16(x[q * 8 + 2] * rstd, x[q * 8 + 3] * rstd);
-          o.z = pack_bf16(x[q * 8 + 4] * rstd, x[q * 8 + 5] * rstd);
-          o.w = pack_bf16(x[q * 8 + 6] * rstd, x[q * 8 + 7] * rstd);
-          sts128(rbase + ((((uint32_t)((cb & 1) * 4 + q)) ^ sw) << 4), o);
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const f2_t y = f2_mul(f2(x[q * 8 + 2 * e], x[q * 8 + 2 * e + 1]), rstd2);
+            o[e] = pack_bf16(f2_lo(y), f2_hi(y));
+          }
+          sts128(rbase + ((((uint32_t)((cb & 1) * 4 + q)) ^ sw) << 4), make_uint4(o[0], o[1], o[2], o[3]));
         }
       }
       tc_fence_before();
@@ -794,7 +876,7 @@ inline int tc_table_entries(const Geom& g, const Partition& part) {
 inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const void* v,
                              const void* beta, const void* gate, void* out, float* S,
                              float* z, bool carry, float* part_S, float* part_z,
-                             __half* S_img, float* S_rs, float* den_dbg, float* x_dbg,
+                             __half* S_img, float* S_scale, float* den_dbg, float* x_dbg,
                              int sms, cudaStream_t stream, void* const* events) {
   auto mark = [&](int i) {
     if (!events || !events[i]) return cudaSuccess;
@@ -829,13 +911,13 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   cp.part_S = part_S; cp.part_z = part_z;
   cp.S_in = carry ? S : nullptr;
   cp.z_in = carry ? z : nullptr;
-  cp.S_out = S; cp.z_out = z; cp.S_img = S_img; cp.S_rs = S_rs;
-  dim3 cgrid(128 * 128 / kCombineElems, g.B * g.Hh);
+  cp.S_out = S; cp.z_out = z; cp.S_img = S_img; cp.S_scale = S_scale;
+  dim3 cgrid(kCombineCluster, g.B * g.Hh);
   combine_kernel<<<cgrid, kCombineThreads, 0, stream>>>(cp);
   if (cudaGetLastError() != cudaSuccess || mark(2) != cudaSuccess) return GLA_ERR_CUDA;
 
   TcApplyParams ap;
-  ap.g = g; ap.part = part; ap.S_img = S_img; ap.S_rs = S_rs; ap.z = z;
+  ap.g = g; ap.part = part; ap.S_img = S_img; ap.S_scale = S_scale; ap.z = z;
   ap.den_out = den_dbg; ap.x_out = x_dbg; ap.tab_entries = tab;
   const bool dbg = den_dbg != nullptr || x_dbg != nullptr;
   if (dbg) {

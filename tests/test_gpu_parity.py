@@ -11,7 +11,8 @@ import torch
 
 from gated_bidirectional_linear_b200 import gla, workloads
 from gpu_common import (BF16_TOL, F32_TOL, S_TOL_BF16, ZDEN_TOL, head_slice, np64,
-                        oracle_forward, rel_elem, rel_floor, rel_rms, to_device)
+                        oracle_forward, rel_elem, rel_floor, rel_rms, rel_rms_bf16out,
+                        to_device)
 import oracle.gla_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -61,11 +62,14 @@ def w480():
 def test_480p_all_outputs(w480, path):
     wl, inp, ref = w480
     got = _debug(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, path)
-    err = rel_rms(got["out"], ref["out"])
-    print(f"480p {path}: out err/rms {err:.3e}")
-    assert err <= BF16_TOL
-    assert rel_rms(got["x"], ref["x"]) <= BF16_TOL
-    assert np.max(np.abs(got["S"] - ref["S"])) / np.sqrt(np.mean(ref["S"] ** 2)) <= S_TOL_BF16
+    err_q = rel_rms_bf16out(got["out"], ref["out"])
+    err_x = rel_rms(got["x"], ref["x"])
+    print(f"480p path {path}: out err/rms {rel_rms(got['out'], ref['out']):.3e} "
+          f"(beyond bf16 rounding {err_q:.3e}), x err/rms {err_x:.3e}, "
+          f"S {rel_floor(got['S'], ref['S']):.3e}")
+    assert err_q <= BF16_TOL
+    assert err_x <= BF16_TOL
+    assert rel_floor(got["S"], ref["S"]) <= S_TOL_BF16
     assert rel_elem(got["z"], ref["z"]) <= ZDEN_TOL
     assert rel_elem(got["den"], ref["den"]) <= ZDEN_TOL
 
@@ -88,13 +92,15 @@ def _sampled_parity(name, heads):
     torch.cuda.synchronize()
     assert gla.gla_get_device_status() == gla.GLA_OK
     out = out.cpu()
-    worst = 0.0
+    worst, worst_q = 0.0, 0.0
     for b, h in heads:
         ref = oracle_forward(head_slice(inp, b, h), wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
         got = out[b:b + 1, :, h:h + 1, :].to(torch.float64).numpy()
         worst = max(worst, rel_rms(got, ref["out"]))
-    print(f"{name}: sampled heads {heads}: out err/rms {worst:.3e}")
-    assert worst <= BF16_TOL
+        worst_q = max(worst_q, rel_rms_bf16out(got, ref["out"]))
+    print(f"{name}: sampled heads {heads}: out err/rms {worst:.3e}, "
+          f"beyond bf16 rounding {worst_q:.3e}")
+    assert worst_q <= BF16_TOL
 
 
 def test_720p_sampled_heads():
@@ -137,9 +143,9 @@ def test_block_causal_sampled_heads():
         ref = O.block_causal_forward(x["q"], x["k"], x["v"], x["beta"], x["g"], wl.n_blocks,
                                      wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
         got = out[b:b + 1, :, h:h + 1, :].to(torch.float64).numpy()
-        assert rel_rms(got, ref["out"]) <= BF16_TOL
+        assert rel_rms_bf16out(got, ref["out"]) <= BF16_TOL
         S = state[b, h].double().numpy()
-        assert np.max(np.abs(S - ref["S"][0, 0])) / np.sqrt(np.mean(ref["S"] ** 2)) <= S_TOL_BF16
+        assert rel_floor(S, ref["S"][0, 0]) <= S_TOL_BF16
         assert rel_elem(z[b, h].double().numpy(), ref["z"][0, 0]) <= ZDEN_TOL
 
 
@@ -183,10 +189,11 @@ def test_edge_shapes(case):
             assert rel_floor(got["out"], ref["out"]) <= F32_TOL
             assert rel_floor(got["S"], ref["S"]) <= F32_TOL
         else:
-            assert rel_rms(got["out"], ref["out"]) <= BF16_TOL
+            assert rel_rms_bf16out(got["out"], ref["out"]) <= BF16_TOL
             assert rel_rms(got["x"], ref["x"]) <= BF16_TOL
-            assert np.max(np.abs(got["S"] - ref["S"])) / np.sqrt(np.mean(ref["S"] ** 2)) <= S_TOL_BF16
-        assert rel_elem(got["z"], ref["z"]) <= ZDEN_TOL
+            assert rel_floor(got["S"], ref["S"]) <= S_TOL_BF16
+        assert rel_floor(got["z"], ref["z"]) <= ZDEN_TOL
+        assert rel_elem(got["den"], ref["den"]) <= ZDEN_TOL
         assert np.all(got["den"] >= 1e-6 * (1 - 1e-6))
 
 
