@@ -420,6 +420,86 @@ gla_status gla_forward_host(const void* q_h, const void* k_h, const void* v_h,
   return GLA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.  The scratch lives in a file-scope device array;
+// host code only ever uses its device address, looked up once per device.
+
+}  // extern "C"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GLA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device (0 on failure).
+unsigned char* noalloc_scratch() {
+  static unsigned char* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  return addr[dev];
+}
+
+// Scratch layout sized for the grid this GPU actually runs (at most `grid`
+// state CTAs, `zparts` z partials per slot) rather than the worst case.
+WsLayout noalloc_layout(int BH, int d, int grid, int zparts) {
+  WsLayout L;
+  L.slots = grid + BH;
+  size_t off = 0;
+  L.part_S = off; off = align_up(off + (size_t)L.slots * d * d * 4, kAlign);
+  L.part_z = off; off = align_up(off + (size_t)L.slots * zparts * d * 4, kAlign);
+  L.S = off; off = align_up(off + (size_t)BH * d * d * 4, kAlign);
+  L.z = off; off = align_up(off + (size_t)BH * d * 4, kAlign);
+  L.S_img = off;
+  if (d == 128) off = align_up(off + (size_t)BH * d * d * 2, kAlign);
+  L.S_scale = off;
+  if (d == 128) off = align_up(off + (size_t)BH * 4 * 4, kAlign);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+gla_status gla_forward_noalloc(const void* q, const void* k, const void* v, const void* beta,
+                               const void* g, int batch, int heads, int head_dim, int T, int H,
+                               int W, float rope_theta, float eps, int dtype, void* out,
+                               void* stream) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W)) return GLA_ERR_INVALID_ARG;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+  if (!(eps > 0.f) || !isfinite(eps) || !isfinite(rope_theta)) return GLA_ERR_INVALID_ARG;
+  const void* ptrs[6] = {q, k, v, beta, g, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
+  Call c;
+  c.g = make_geom(batch, heads, head_dim, T, H, W, 0, rope_theta, eps);
+  const int sms = device_sm_count();
+  if (sms <= 0) return GLA_ERR_CUDA;
+  c.dtype = dtype;
+  c.path = resolve_path(GLA_PATH_AUTO, dtype, head_dim, &c.g, sms);
+  const bool tensor = c.path == GLA_PATH_TENSOR;
+  const Partition part = tensor ? make_partition(batch * heads, c.g.N, kTcTile, sms)
+                                : make_partition(batch * heads, c.g.N, kSimtTile, 2 * sms);
+  const WsLayout L = noalloc_layout(batch * heads, head_dim, part.grid, tensor ? kStTW : 1);
+  if (L.total > GLA_NOALLOC_SCRATCH_BYTES) return GLA_ERR_WORKSPACE;
+  unsigned char* scratch = noalloc_scratch();
+  if (!scratch) return GLA_ERR_CUDA;
+  c.q = q; c.k = k; c.v = v; c.beta = beta; c.gate = g; c.out = out;
+  c.ws = scratch;
+  c.L = L;
+  c.S = reinterpret_cast<float*>(c.ws + L.S);
+  c.z = reinterpret_cast<float*>(c.ws + L.z);
+  c.carry = false;
+  c.stream = static_cast<cudaStream_t>(stream);
+  c.S_dbg = c.z_dbg = c.den_dbg = c.x_dbg = nullptr;
+  c.events = nullptr;
+  return run_call(c);
+}
+
 gla_status gla_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return GLA_ERR_CUDA;

@@ -38,6 +38,7 @@ _SIGS = {
     "gla_block_causal_step_ex": (_i, [_vp] * 7 + [_i] * 7
                                  + [_f, _f, _i, _vp, _vp, _sz, _vp, _i]),
     "gla_forward_host": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
+    "gla_forward_noalloc": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp]),
     "gla_get_device_status": (_i, [_vp]),
     "gla_plan": (_i, [_i] * 9 + [ctypes.POINTER(_i)] * 3),
 }
@@ -212,6 +213,22 @@ def gla_forward_host(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, ou
                                 H, W, rope_theta, eps, code, _ptr(out), _ptr(arena),
                                 arena.numel(), _stream(stream))
     _check(st, "gla_forward_host")
+    return out
+
+
+def gla_forward_noalloc(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, out=None,
+                        stream=None):
+    """gla_forward without a workspace argument, for callers that cannot
+    allocate device memory: the scratch comes from an array built into
+    libgla.so (GLA_NOALLOC_SCRATCH_BYTES).  Calls share that array, so keep
+    them ordered on one stream."""
+    B, Hh, d = _dims(q, T, H, W)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib().gla_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
+                                   H, W, rope_theta, eps, code, _ptr(out), _stream(stream))
+    _check(st, "gla_forward_noalloc")
     return out
 
 

@@ -187,6 +187,33 @@ GLA_API gla_status gla_forward_host(const void* q_h, const void* k_h, const void
                             int dtype, void* out_h, void* arena, size_t arena_bytes,
                             void* stream);
 
+/* Size of the scratch array built into the library for gla_forward_noalloc. */
+#define GLA_NOALLOC_SCRATCH_BYTES (24u << 20)
+
+/* gla_forward for callers that cannot allocate device memory: code running
+ * where cudaMalloc is unavailable or forbidden (inside a memory-pool-managed
+ * runtime that owns every allocation, in a plugin that must not grow the
+ * process footprint at call time, or on a path that may not synchronise the
+ * device, which cudaMalloc can do).  The operator's scratch space (split-N
+ * partial states, the combined state and its fp16 image) comes from one
+ * array of GLA_NOALLOC_SCRATCH_BYTES compiled into this library; every GPU
+ * that loads the library holds that array until the process exits.  The
+ * caller still passes the inputs and `out`.  No counterpart on the pages: it
+ * is a packaging choice of this library.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call shares the one array and leaves its contents behind:
+ * calls whose kernels overlap on the GPU (different streams, or different
+ * host threads on the same device without ordering) race on it and give
+ * wrong results, so order them on one stream.  Nothing in the array needs to
+ * start at zero.  Problems whose scratch would exceed the array return
+ * GLA_ERR_WORKSPACE with nothing launched; it allocates nothing, ever. */
+GLA_API gla_status gla_forward_noalloc(const void* q, const void* k, const void* v,
+                                       const void* beta, const void* g, int batch, int heads,
+                                       int head_dim, int T, int H, int W, float rope_theta,
+                                       float eps, int dtype, void* out, void* stream);
+
 /* Synchronises `stream`, then reports and clears the library's device error
  * word: GLA_ERR_TIMEOUT if a kernel gave up a bounded wait since the last
  * call, GLA_ERR_CUDA if the synchronisation itself failed, else GLA_OK. */
