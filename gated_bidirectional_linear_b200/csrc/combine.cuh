@@ -26,7 +26,7 @@ namespace gla {
 
 constexpr int kCombineCluster = 8;
 constexpr int kMaxZPartsCombined = 4 * kCombineCluster;   // z partials per slot it can add
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 256;   // >= d, so one thread per z element
 
 struct CombineParams {
   Partition part;
@@ -58,6 +58,10 @@ __device__ __forceinline__ void add4(float4& s, const float4 t) {
 __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombineThreads)
     combine_kernel(CombineParams p) {
   namespace cg = cooperative_groups;
+  // Launched as a programmatic dependent of the state reduction: wait for its
+  // partials, and let the read-out kernel start its own prologue meanwhile.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cg::cluster_group cluster = cg::this_cluster();
   __shared__ float red[kCombineThreads / 32];
   __shared__ float cta_max;
@@ -72,61 +76,65 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
   const int chunk = (int)(dd / kCombineCluster);        // 2048 for d = 128
   const int e_base = rank * chunk;
 
-  // Each thread owns up to two float4 groups: e = e_base + 4*tid + 1024*k.
+  // Each thread owns up to two float4 groups of S (e = e_base + 4*tid + 1024*k)
+  // and, for d <= 128, one element e = tid of the z partials this rank adds
+  // (partials rank, rank + 8, ... of each slot).  All loads of a batch of
+  // slots are issued before any is added, then added in slot order.
+  constexpr int kBatch = 4;
   float4 acc[2];
-  float m = 0.f;
+  float zacc = 0.f;
+  bool live[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
+    live[k] = e < e_base + chunk;
     acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (e >= e_base + chunk) continue;
-    if (p.S_in) acc[k] = *reinterpret_cast<const float4*>(p.S_in + bh * dd + e);
-    int c = c_lo;
-    // Issue four independent loads at a time; add them in slot order.
-    for (; c + 3 <= c_hi; c += 4) {
-      const float4 t0 = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + bh) * dd + e);
-      const float4 t1 = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + 1 + bh) * dd + e);
-      const float4 t2 = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + 2 + bh) * dd + e);
-      const float4 t3 = *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + 3 + bh) * dd + e);
-      add4(acc[k], t0); add4(acc[k], t1); add4(acc[k], t2); add4(acc[k], t3);
+    if (live[k] && p.S_in) acc[k] = *reinterpret_cast<const float4*>(p.S_in + bh * dd + e);
+  }
+  const bool zlive = (int)threadIdx.x < d;
+  for (int c0 = c_lo; c0 <= c_hi; c0 += kBatch) {
+    float4 t[kBatch][2];
+    float zt[kBatch][4];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int c = c0 + b;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
+        t[b][k] = (c <= c_hi && live[k])
+                      ? *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + bh) * dd + e)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int zp = rank + kCombineCluster * q;
+        zt[b][q] = (c <= c_hi && zlive && zp < p.zparts)
+                       ? p.part_z[(((size_t)c + bh) * p.zparts + zp) * d + threadIdx.x]
+                       : 0.f;
+      }
     }
-    for (; c <= c_hi; ++c)
-      add4(acc[k], *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + bh) * dd + e));
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      if (c0 + b > c_hi) break;
+      add4(acc[0], t[b][0]);
+      add4(acc[1], t[b][1]);
+      zacc += zt[b][0]; zacc += zt[b][1]; zacc += zt[b][2]; zacc += zt[b][3];
+    }
+  }
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    if (!live[k]) continue;
+    const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
     *reinterpret_cast<float4*>(p.S_out + bh * dd + e) = acc[k];
     m = fmaxf(m, fmaxf(fmaxf(fabsf(acc[k].x), fabsf(acc[k].y)),
                        fmaxf(fabsf(acc[k].z), fabsf(acc[k].w))));
   }
 
-  // z: rank r sums the z partials r, r + 8, ... of every contributing slot
-  // (slot-major, in order); rank 0 then adds the ranks' sums in rank order.
+  // z: rank 0 adds the ranks' sums in rank order; the head maximum of |S|
+  // travels in the same exchange.
   __shared__ float zsum[128];
-  for (int e = threadIdx.x; e < d; e += kCombineThreads) {
-    float s = 0.f;
-    for (int c = c_lo; c <= c_hi; ++c) {
-      const float* zc = p.part_z + ((size_t)c + bh) * p.zparts * d + e;
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int zp = rank + kCombineCluster * k;
-        if (zp < p.zparts) t[k] = zc[(size_t)zp * d];
-      }
-      s += t[0]; s += t[1]; s += t[2]; s += t[3];
-    }
-    zsum[e] = s;
-  }
-  cluster.sync();
-  if (rank == 0) {
-    for (int e = threadIdx.x; e < d; e += kCombineThreads) {
-      float s = p.z_in ? p.z_in[(size_t)bh * d + e] : 0.f;
-      for (int r = 0; r < kCombineCluster; ++r) s += *cluster.map_shared_rank(&zsum[e], r);
-      p.z_out[(size_t)bh * d + e] = s;
-    }
-  }
-  cluster.sync();   // zsum of every rank stays valid until rank 0 has read it
-
-  if (p.S_img == nullptr) return;     // uniform over the whole grid
-
-  // Head maximum: warp, CTA, then the cluster through distributed smem.
+  if (zlive) zsum[threadIdx.x] = zacc;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -137,10 +145,17 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
     cta_max = mm;
   }
   cluster.sync();
+  if (rank == 0 && zlive) {
+    float zs = p.z_in ? p.z_in[(size_t)bh * d + threadIdx.x] : 0.f;
+    for (int r = 0; r < kCombineCluster; ++r) zs += *cluster.map_shared_rank(&zsum[threadIdx.x], r);
+    p.z_out[(size_t)bh * d + threadIdx.x] = zs;
+  }
   float hm = 0.f;
-  for (int r = 0; r < kCombineCluster; ++r)
-    hm = fmaxf(hm, *cluster.map_shared_rank(&cta_max, r));
-  cluster.sync();   // no CTA leaves while others still read its cta_max
+  if (p.S_img != nullptr)
+    for (int r = 0; r < kCombineCluster; ++r) hm = fmaxf(hm, *cluster.map_shared_rank(&cta_max, r));
+  cluster.sync();   // every rank's zsum / cta_max stays valid until all have read
+
+  if (p.S_img == nullptr) return;     // uniform over the whole grid
 
   // hm = f * 2^E with f in [0.5, 1): scale by 2^(14 - E).
   int E = (int)((__float_as_uint(hm) >> 23) & 0xFFu) - 126;

@@ -100,23 +100,55 @@ inline Partition make_partition(int BH, int N, int tile, int max_grid) {
 // --------------------------------------------------------------- RoPE table
 //
 // Each CTA keeps cos/sin of the rotations it needs in shared memory, as float2
-// (cos, sin) entries, position-major inside each axis so that the pairs of one
-// position are adjacent:
-//   time axis:   [Lt frames][pt pairs]  (frames t_lo .. t_lo+Lt-1, wrapping
-//                                        modulo T when the CTA's tokens cross
-//                                        from the end of one head's sequence
-//                                        to the start of the next)
-//   height axis: [H][ph]
-//   width axis:  [W][pw]
-// Angles are formed and evaluated in double precision, then rounded to fp32.
+// (cos, sin) entries, position-major inside each axis:
+//   time axis:   Lt rows (frames t_lo .. t_lo+Lt-1, wrapping modulo T when
+//                the CTA's tokens cross from the end of one head's sequence to
+//                the start of the next)
+//   height axis: H rows;  width axis: W rows.
+// Pair p (global index 0 .. d/2-1) of axis a sits at column
+//   idx(p) = (p - start_a) + (p >> 3) - (start_a >> 3)
+// of its row: one padding entry after every 8 global pairs, so the 8 pairs a
+// tensor-path lane handles are contiguous while lanes land on different banks.
+// Row strides and axis bases (rope_layout) are chosen so that the transform
+// warps' lookups are free of shared-memory bank conflicts.  Angles are formed
+// and reduced in double precision; cos/sin are evaluated in fp32.
 
 struct RopeWindow {
   int t_lo;   // first local frame held
   int Lt;     // frames held (<= T)
 };
 
-__host__ __device__ inline int rope_table_entries(const Geom& g, int Lt) {
-  return g.pt * Lt + g.ph * g.H + g.pw * g.W;
+struct RopeLayout {
+  int start[3];    // first global pair of each axis
+  int stride[3];   // entries per row
+  int base[3];     // first entry of each axis
+  int entries;     // table size
+};
+
+__host__ __device__ inline int rope_idx(const RopeLayout& L, int a, int p) {
+  return (p - L.start[a]) + (p >> 3) - (L.start[a] >> 3);
+}
+
+__host__ __device__ inline RopeLayout rope_layout(const Geom& g, int Lt) {
+  RopeLayout L;
+  const int np[3] = {g.pt, g.ph, g.pw};
+  L.start[0] = 0;
+  L.start[1] = g.pt;
+  L.start[2] = g.pt + g.ph;
+  for (int a = 0; a < 3; ++a) {
+    const int last = L.start[a] + np[a] - 1;
+    const int width = np[a] > 0 ? (last - L.start[a]) + (last >> 3) - (L.start[a] >> 3) + 1 : 0;
+    // time rows: a multiple of 16 entries; height/width rows: 8 mod 16.
+    L.stride[a] = a == 0 ? (width + 15) / 16 * 16 : ((width + 7) / 16) * 16 + 8;
+  }
+  const int rows[3] = {Lt, g.H, g.W};
+  int off = 0;
+  for (int a = 0; a < 3; ++a) {
+    L.base[a] = off;
+    off = (off + rows[a] * L.stride[a] + 15) / 16 * 16;
+  }
+  L.entries = off;
+  return L;
 }
 
 // Frames touched by the items [w0, w1] (inclusive) of a partition.
@@ -143,47 +175,56 @@ __host__ __device__ inline RopeWindow rope_window(const Geom& g, const Partition
   return r;
 }
 
+__host__ __device__ inline int rope_table_entries(const Geom& g, int Lt) {
+  return rope_layout(g, Lt).entries;
+}
+
 __device__ inline void rope_build(float2* tab, const Geom& g, RopeWindow win, int tid,
                                   int nthr) {
   if (!g.rope_on) return;
-  const int nt = g.pt * win.Lt, nh = g.ph * g.H, nw = g.pw * g.W;
-  const double log_theta = log((double)g.theta);
-  for (int e = tid; e < nt + nh + nw; e += nthr) {
-    int i, p;
-    double pos;
-    if (e < nt) {
-      i = e % g.pt;
-      p = g.pt;
-      int f = win.t_lo + e / g.pt;
+  // Thread tid handles rotation pair (tid mod P) of its axis at every
+  // (nthr / P)-th position: one exp per thread, then per entry the angle
+  // pos * freq in double, reduced to [-pi, pi] in double, and fp32 sincosf.
+  const RopeLayout L = rope_layout(g, win.Lt);
+  const int P = g.pt + g.ph + g.pw;
+  const int pr = tid % P;
+  const int lane0 = tid / P, step = nthr / P;
+  if (lane0 >= step) return;
+  const int axis = pr < g.pt ? 0 : (pr < g.pt + g.ph ? 1 : 2);
+  const int np = axis == 0 ? g.pt : (axis == 1 ? g.ph : g.pw);
+  const int i = pr - L.start[axis];
+  const int rows = axis == 0 ? win.Lt : (axis == 1 ? g.H : g.W);
+  const int col = rope_idx(L, axis, pr);
+  const double freq = exp(-((double)i / (double)np) * log((double)g.theta));
+  const double two_pi = 6.283185307179586476925286766559;
+  for (int pos = lane0; pos < rows; pos += step) {
+    double x;
+    if (axis == 0) {
+      int f = win.t_lo + pos;
       if (f >= g.T) f -= g.T;
-      pos = (double)(g.t0 + f);
-    } else if (e < nt + nh) {
-      i = (e - nt) % g.ph;
-      p = g.ph;
-      pos = (double)((e - nt) / g.ph);
+      x = (double)(g.t0 + f);
     } else {
-      i = (e - nt - nh) % g.pw;
-      p = g.pw;
-      pos = (double)((e - nt - nh) / g.pw);
+      x = (double)pos;
     }
-    const double ang = pos * exp(-((double)i / (double)p) * log_theta);
-    double s, c;
-    sincos(ang, &s, &c);
-    tab[e] = make_float2((float)c, (float)s);
+    double ang = x * freq;
+    ang -= two_pi * rint(ang * (1.0 / two_pi));
+    float sn, cs;
+    sincosf((float)ang, &sn, &cs);
+    tab[L.base[axis] + pos * L.stride[axis] + col] = make_float2(cs, sn);
   }
 }
 
 // Index of the (cos, sin) entry of rotation pair `pr` (0 .. d/2-1) for a token
 // at local frame f, row hh, column ww.
-__device__ inline int rope_index(const Geom& g, RopeWindow win, int pr, int f, int hh,
-                                 int ww) {
+__device__ inline int rope_index(const Geom& g, RopeWindow win, const RopeLayout& L, int pr,
+                                 int f, int hh, int ww) {
   if (pr < g.pt) {
     int tl = f - win.t_lo;
     if (tl < 0) tl += g.T;
-    return tl * g.pt + pr;
+    return L.base[0] + tl * L.stride[0] + rope_idx(L, 0, pr);
   }
-  if (pr < g.pt + g.ph) return g.pt * win.Lt + hh * g.ph + (pr - g.pt);
-  return g.pt * win.Lt + g.ph * g.H + ww * g.pw + (pr - g.pt - g.ph);
+  if (pr < g.pt + g.ph) return L.base[1] + hh * L.stride[1] + rope_idx(L, 1, pr);
+  return L.base[2] + ww * L.stride[2] + rope_idx(L, 2, pr);
 }
 
 // ------------------------------------------------------------------ dtypes

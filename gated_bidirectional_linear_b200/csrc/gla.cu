@@ -133,9 +133,9 @@ inline cudaError_t mark(const Call& c, int i) {
 // its tile rings; grids whose table does not fit use the CUDA-core path.
 bool tensor_fits(const Geom& g, int sms) {
   if (g.H >= (1 << kPosBits) || g.W >= (1 << kPosBits) || g.T >= (1 << kPosBits)) return false;
-  const Partition part = make_partition(g.B * g.Hh, g.N, kTcTile, sms);
-  const int tab = tc_table_entries(g, part);
-  return tc_state_smem(tab) <= kMaxSmem && tc_apply_smem(tab) <= kMaxSmem;
+  const int stab = tc_table_entries(g, tc_state_partition(g, sms));
+  const int tab = tc_table_entries(g, tc_apply_partition(g, sms));
+  return tc_state_smem(stab) <= kMaxSmem && tc_apply_smem(tab) <= kMaxSmem;
 }
 
 int resolve_path(int requested, int dtype, int d, const Geom* g = nullptr, int sms = 0) {
@@ -482,7 +482,7 @@ gla_status gla_forward_noalloc(const void* q, const void* k, const void* v, cons
   c.dtype = dtype;
   c.path = resolve_path(GLA_PATH_AUTO, dtype, head_dim, &c.g, sms);
   const bool tensor = c.path == GLA_PATH_TENSOR;
-  const Partition part = tensor ? make_partition(batch * heads, c.g.N, kTcTile, sms)
+  const Partition part = tensor ? tc_state_partition(c.g, sms)
                                 : make_partition(batch * heads, c.g.N, kSimtTile, 2 * sms);
   const WsLayout L = noalloc_layout(batch * heads, head_dim, part.grid, tensor ? kStTW : 1);
   if (L.total > GLA_NOALLOC_SCRATCH_BYTES) return GLA_ERR_WORKSPACE;
@@ -523,8 +523,9 @@ gla_status gla_plan(int batch, int heads, int head_dim, int T, int H, int W, int
   const int resolved = resolve_path(path, dtype, head_dim, &g, num_sms);
   if (resolved < 0) return GLA_ERR_UNSUPPORTED;
   const int N = T * H * W;
+  (void)N;
   Partition p = resolved == GLA_PATH_TENSOR
-                    ? make_partition(batch * heads, N, kTcTile, num_sms)
+                    ? tc_state_partition(g, num_sms)
                     : make_partition(batch * heads, N, kSimtTile, 2 * num_sms);
   *grid = p.grid;
   *tile_tokens = p.tile;

@@ -90,6 +90,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// ------------------------------------------------ programmatic dependent launch
+
+// Let the next kernel of the stream (launched with programmatic stream
+// serialization) start its prologue while this grid is still running.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Block until the preceding grid of the stream has completed and its memory
+// operations are visible.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------- TMA / bulk
 
 __device__ __forceinline__ uint64_t policy_evict_first() {

@@ -29,7 +29,8 @@ struct SimtStateParams {
 // warp: lane l holds elements l + 32 m.  Returns in x_pls / x_til.
 template <int D, typename Tin>
 __device__ inline void row_features(const Tin* row, const Geom& g, const float2* tab,
-                                    RopeWindow win, int f, int hh, int ww, int lane,
+                                    RopeWindow win, const RopeLayout& L, int f, int hh, int ww,
+                                    int lane,
                                     float (&x_pls)[D / 32], float (&x_til)[D / 32],
                                     bool valid) {
   constexpr int M = D / 32;
@@ -49,7 +50,7 @@ __device__ inline void row_features(const Tin* row, const Geom& g, const float2*
     const float other = __shfl_xor_sync(0xffffffffu, x_pls[m], 1);
     if (g.rope_on && valid) {
       const int e = lane + 32 * m;
-      const float2 cs = tab[rope_index(g, win, e >> 1, f, hh, ww)];
+      const float2 cs = tab[rope_index(g, win, L, e >> 1, f, hh, ww)];
       x_til[m] = (e & 1) ? fmaf(other, cs.y, x_pls[m] * cs.x)     // x0 s + x1 c
                          : fmaf(-other, cs.y, x_pls[m] * cs.x);   // x0 c - x1 s
     } else {
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_state_kernel(SimtStateParam
   const int c = blockIdx.x;
   const long long w_begin = part_begin(part, c), w_end = part_begin(part, c + 1);
   const RopeWindow win = rope_window(g, part, w_begin, w_end - 1);
+  const RopeLayout L = rope_layout(g, win.Lt);
   rope_build(tab, g, win, tid, blockDim.x);
 
   const Tin* kin = static_cast<const Tin*>(p.k);
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_state_kernel(SimtStateParam
                   ww = valid ? n % g.W : 0;
         const size_t row = (((size_t)b * g.N + (valid ? n : 0)) * g.Hh + h);
         float xp[M], xt[M];
-        row_features<D, Tin>(kin + row * D, g, tab, win, f, hh, ww, lane, xp, xt, valid);
+        row_features<D, Tin>(kin + row * D, g, tab, win, L, f, hh, ww, lane, xp, xt, valid);
         const float be = valid ? to_f32<Tin>(bin[row]) : 0.f;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
@@ -180,6 +182,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_apply_kernel(SimtApplyParam
   tp.BH = 1; tp.tile = kSimtApplyTile; tp.tiles_per_head = (g.N + kSimtApplyTile - 1) / kSimtApplyTile;
   tp.items = tp.tiles_per_head; tp.grid = 1;
   const RopeWindow win = rope_window(g, tp, blockIdx.x, blockIdx.x);
+  const RopeLayout L = rope_layout(g, win.Lt);
   rope_build(tab, g, win, tid, blockDim.x);
 
   const float* Sg = p.S + (size_t)bh * D * D;
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_apply_kernel(SimtApplyParam
     const int f = n / HW, hh = (n / g.W) % g.H, ww = n % g.W;
     const size_t row = (((size_t)b * g.N + n) * g.Hh + h);
     float xp[M], xt[M];
-    row_features<D, Tin>(qin + row * D, g, tab, win, f, hh, ww, lane, xp, xt, true);
+    row_features<D, Tin>(qin + row * D, g, tab, win, L, f, hh, ww, lane, xp, xt, true);
     float dsum = 0.f;
 #pragma unroll
     for (int m = 0; m < M; ++m) dsum = fmaf(zs[lane + 32 * m], xp[m], dsum);

@@ -26,27 +26,33 @@
 
 namespace gla {
 
-constexpr int kTcTile = 128;                 // tokens per tile
+constexpr int kTcTile = 128;                 // tokens per read-out tile (MMA M)
 constexpr uint32_t kBox = 16384;             // one TMA box: 128 rows x 128 bytes
-constexpr uint32_t kTileBytes = 2 * kBox;    // 128 tokens x 128 channels bf16
+constexpr uint32_t kTileBytes = 2 * kBox;    // 128 tokens x 128 channels, 16-bit
+constexpr int kStTile = 96;                  // tokens per state tile (MMA K)
+constexpr uint32_t kStBox = kStTile * 128;   // 96 rows x 128 bytes
+constexpr uint32_t kStTileBytes = 2 * kStBox;
 constexpr int kPosBits = 11;                 // packed (t, h, w) offsets, < 2048 each
 
 // --------------------------------------------------------------- state kernel
 
-constexpr int kStStages = 3;
+constexpr int kStStages = 4;
 constexpr int kStTW = 12;                    // transform warps; the first four
                                              // also drain finished S partials
 constexpr int kStTW0 = 2;                    // first transform warp
 constexpr int kStThreads = (kStTW0 + kStTW) * 32;
 static_assert(kStTW <= kMaxZPartsCombined, "combine adds at most this many z partials");
 static_assert((kStTW * 4) % 8 == 0, "rows per pass keep the 8-row swizzle phase");
+static_assert(kStTile % (kStTW * 4) == 0, "whole passes per state tile");
+static_assert(kStTile % 16 == 0 && kStBox % 1024 == 0, "MMA K steps and swizzle atoms");
 constexpr int kStRowsPerPass = kStTW * 4;
 
 struct TcStateSmem {
   static constexpr uint32_t K = 0;
-  static constexpr uint32_t V = kStStages * kTileBytes;
-  static constexpr uint32_t ROWPOS = 2 * kStStages * kTileBytes;      // [stage][128] uint2
-  static constexpr uint32_t BAR = ROWPOS + kStStages * 1024;          // barriers
+  static constexpr uint32_t V = kStStages * kStTileBytes;
+  static constexpr uint32_t ROWPOS = 2 * kStStages * kStTileBytes;    // [stage][96] uint2
+  static constexpr uint32_t BETA = ROWPOS + kStStages * kStTile * 8;  // [stage][96] f32
+  static constexpr uint32_t BAR = BETA + kStStages * kStTile * 4;     // barriers
   static constexpr uint32_t NBAR = 3 * kStStages + 5;
   static constexpr uint32_t MISC = BAR + NBAR * 8;                     // tmem base, abort
   static constexpr uint32_t TAB = (MISC + 16 + 15) & ~15u;              // RoPE table
@@ -72,12 +78,13 @@ __device__ __forceinline__ bool seg_last(const Partition& p, long long w, long l
 // producer warp stores the byte offsets, inside the RoPE table, of the token's
 // time, height and width rows: (offT | offH << 16, offW).  The table is at
 // most 22.5 KB, so 16 bits hold each offset.
+template <int kRows>
 __device__ __forceinline__ void tile_rowpos(const Geom& g, RopeWindow win, int n0, int lane,
                                             uint2* rowpos) {
   const uint32_t HW = g.div_HW.d, W = g.div_W.d;
-  const uint32_t baseH = (uint32_t)(g.pt * win.Lt), baseW = baseH + (uint32_t)(g.ph * g.H);
+  const RopeLayout L = rope_layout(g, win.Lt);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < kRows / 32; ++k) {
     const int r = lane + 32 * k;
     int n = n0 + r;
     if (n >= g.N) n = n0;
@@ -87,17 +94,18 @@ __device__ __forceinline__ void tile_rowpos(const Geom& g, RopeWindow win, int n
     const uint32_t ww = rem - hh * W;
     int tl = (int)f - win.t_lo;
     if (tl < 0) tl += g.T;
-    const uint32_t offT = 8u * (uint32_t)(tl * g.pt);
-    const uint32_t offH = 8u * (baseH + hh * (uint32_t)g.ph);
-    const uint32_t offW = 8u * (baseW + ww * (uint32_t)g.pw);
+    const uint32_t offT = 8u * (uint32_t)(L.base[0] + tl * L.stride[0]);
+    const uint32_t offH = 8u * (uint32_t)(L.base[1] + (int)hh * L.stride[1]);
+    const uint32_t offW = 8u * (uint32_t)(L.base[2] + (int)ww * L.stride[2]);
     rowpos[r] = make_uint2(offT | (offH << 16), offW);
   }
 }
 
 // Per-lane view of the RoPE table.  Lane j of a row group handles channels
 // 16j .. 16j+15, i.e. rotation pairs 8j .. 8j+7; for d = 128 every axis has at
-// least 21 pairs, so those 8 pairs lie on at most two axes A and B.  With the
-// position-major table, pair i of the lane sits at byte
+// least 21 pairs, so those 8 pairs lie on at most two axes A and B.  In the
+// table, pair 8j + i of axis X sits at column idx = 8j + i - start + j -
+// (start >> 3) of its row, so slot i of the lane is at byte
 //   offA(row) + inA + 8 i   (pairs on axis A)
 //   offB(row) + inB + 8 i   (pairs on axis B, useB[i] = 1)
 // where offX(row) is the row's metadata for axis X.
@@ -115,8 +123,8 @@ __device__ __forceinline__ void lane_rope(const Geom& g, int j, LaneRope& lr) {
   const int p0 = 8 * j;
   const int start[3] = {0, g.pt, g.pt + g.ph};
   const int aA = axis_of(g, p0), aB = axis_of(g, p0 + 7);
-  lr.inA = 8 * (p0 - start[aA]);
-  lr.inB = 8 * (p0 - start[aB]);
+  lr.inA = 8 * (p0 - start[aA] + j - (start[aA] >> 3));
+  lr.inB = 8 * (p0 - start[aB] + j - (start[aB] >> 3));
   lr.wA = aA == 2 ? 1 : 0;
   lr.shA = aA == 1 ? 16 : 0;
   lr.wB = aB == 2 ? 1 : 0;
@@ -125,22 +133,22 @@ __device__ __forceinline__ void lane_rope(const Geom& g, int j, LaneRope& lr) {
   for (int i = 0; i < 8; ++i) lr.useB[i] = axis_of(g, p0 + i) != aA ? 1 : 0;
 }
 
-// Table pointer of the lane's pair 0 for a row, and the entry distance from
-// its axis-A run to its axis-B run.
-__device__ __forceinline__ void lane_rope_row(const LaneRope& lr, const float2* tab, uint2 m,
-                                              const float2*& pA, int& dE) {
+// Shared-memory address of the lane's pair-0 table entry for a row, and the
+// byte distance from its axis-A run to its axis-B run.
+__device__ __forceinline__ void lane_rope_row(const LaneRope& lr, uint32_t tab_s, uint2 m,
+                                              uint32_t& aA, int& dB) {
   const uint32_t offA = ((lr.wA ? m.y : m.x) >> lr.shA) & 0xFFFFu;
   const uint32_t offB = ((lr.wB ? m.y : m.x) >> lr.shB) & 0xFFFFu;
   const int bA = (int)offA + lr.inA, bB = (int)offB + lr.inB;
-  pA = reinterpret_cast<const float2*>(reinterpret_cast<const char*>(tab) + bA);
-  dE = (bB - bA) >> 3;
+  aA = tab_s + (uint32_t)bA;
+  dB = bB - bA;
 }
 
 // Shared-memory addresses of the two 16-byte chunks a lane owns in row r of a
 // 128x128 16-bit tile stored as two 128-byte-swizzled boxes.
-__device__ __forceinline__ void lane_chunks(uint32_t tile, int r, int j, uint32_t& a0,
-                                            uint32_t& a1) {
-  const uint32_t row = tile + (uint32_t)(j >> 2) * kBox + (uint32_t)r * 128u;
+__device__ __forceinline__ void lane_chunks(uint32_t tile, uint32_t box, int r, int j,
+                                            uint32_t& a0, uint32_t& a1) {
+  const uint32_t row = tile + (uint32_t)(j >> 2) * box + (uint32_t)r * 128u;
   const uint32_t c0 = (uint32_t)((2 * j) & 7);
   a0 = row + (((c0) ^ (uint32_t)(r & 7)) << 4);
   a1 = row + (((c0 + 1) ^ (uint32_t)(r & 7)) << 4);
@@ -152,46 +160,72 @@ __device__ __forceinline__ void unpack8(uint4 a, uint4 b, f2_t (&x)[8]) {
   x[4] = f2_bf(b.x); x[5] = f2_bf(b.y); x[6] = f2_bf(b.z); x[7] = f2_bf(b.w);
 }
 
+// Lane layout of the transform warps: a warp holds 4 rows x 8 lanes.  Lane
+// bits 0-1 pick the chunk pair inside a 64-channel box, bit 3 the box (so
+// j = chunk-pair index 0..7), bits 2 and 4 the row.  Each group of 8
+// consecutive lanes -- the unit in which the hardware serves 16-byte shared
+// accesses -- then touches 8 different 16-byte bank groups of the swizzled
+// tile, and the 8 lanes of a row are closed under xor 1, 2, 8.
+__device__ __forceinline__ int tw_row(int lane) { return ((lane >> 2) & 1) | (((lane >> 4) & 1) << 1); }
+__device__ __forceinline__ int tw_chunk(int lane) { return (lane & 3) | (((lane >> 3) & 1) << 2); }
+
+__device__ __forceinline__ float row_sum(float s) {
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 8);
+  return s;
+}
+
 // 1/RMS of a row whose 128 elements are spread over the 8 lanes of a group.
 __device__ __forceinline__ float row_rstd(const f2_t (&x)[8]) {
   f2_t ss = 0ull;
 #pragma unroll
   for (int i = 0; i < 8; ++i) ss = f2_fma(x[i], x[i], ss);
-  float s = f2_lo(ss) + f2_hi(ss);
-  s += __shfl_xor_sync(0xffffffffu, s, 1);
-  s += __shfl_xor_sync(0xffffffffu, s, 2);
-  s += __shfl_xor_sync(0xffffffffu, s, 4);
-  return rsqrtf(s * (1.f / 128.f) + kRmsEps);
+  return rsqrtf(row_sum(f2_lo(ss) + f2_hi(ss)) * (1.f / 128.f) + kRmsEps);
 }
 
 __device__ __forceinline__ f2_t f2_relu(f2_t x) {
   return f2(fmaxf(f2_lo(x), 0.f), fmaxf(f2_hi(x), 0.f));
 }
 
+// (cos, sin) of pair I of the lane: one shared load at an immediate offset.
+#define GLA_TAB_LOAD(I, base, out)                                              \
+  asm volatile("ld.shared.b64 %0, [%1+%2];" : "=l"(out) : "r"(base), "n"(8 * (I)))
+
 // Rotate the lane's 8 ReLU'd pairs r (still unnormalised), scaled by `scl`:
 // y = scl * RoPE(r), packed to bf16 (kHalf = false) or fp16.
 template <bool kHalf>
 __device__ __forceinline__ void rope_scale_pack(const Geom& g, const LaneRope& lr,
-                                                const float2* pA, int dE,
+                                                uint32_t aA, int dB,
                                                 const f2_t (&r)[8], float scl, uint4& o0,
                                                 uint4& o1) {
   uint32_t w[8];
   const f2_t scl2 = f2(scl, scl);
+  if (g.rope_on) {
+    f2_t e[8];
+    GLA_TAB_LOAD(0, aA + (uint32_t)(lr.useB[0] * dB), e[0]);
+    GLA_TAB_LOAD(1, aA + (uint32_t)(lr.useB[1] * dB), e[1]);
+    GLA_TAB_LOAD(2, aA + (uint32_t)(lr.useB[2] * dB), e[2]);
+    GLA_TAB_LOAD(3, aA + (uint32_t)(lr.useB[3] * dB), e[3]);
+    GLA_TAB_LOAD(4, aA + (uint32_t)(lr.useB[4] * dB), e[4]);
+    GLA_TAB_LOAD(5, aA + (uint32_t)(lr.useB[5] * dB), e[5]);
+    GLA_TAB_LOAD(6, aA + (uint32_t)(lr.useB[6] * dB), e[6]);
+    GLA_TAB_LOAD(7, aA + (uint32_t)(lr.useB[7] * dB), e[7]);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float r0 = f2_lo(r[i]), r1 = f2_hi(r[i]);
-    float y0, y1;
-    if (g.rope_on) {
-      const float2 e = pA[lr.useB[i] * dE + i];
-      const f2_t cs = f2_mul(f2(e.x, e.y), scl2);
+    for (int i = 0; i < 8; ++i) {
+      const float r0 = f2_lo(r[i]), r1 = f2_hi(r[i]);
+      const f2_t cs = f2_mul(e[i], scl2);
       const float c = f2_lo(cs), sn = f2_hi(cs);
-      y0 = fmaf(-r1, sn, r0 * c);
-      y1 = fmaf(r1, c, r0 * sn);
-    } else {
-      y0 = r0 * scl;
-      y1 = r1 * scl;
+      const float y0 = fmaf(-r1, sn, r0 * c);
+      const float y1 = fmaf(r1, c, r0 * sn);
+      w[i] = kHalf ? pack_f16(y0, y1) : pack_bf16(y0, y1);
     }
-    w[i] = kHalf ? pack_f16(y0, y1) : pack_bf16(y0, y1);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const f2_t y = f2_mul(r[i], scl2);
+      w[i] = kHalf ? pack_f16(f2_lo(y), f2_hi(y)) : pack_bf16(f2_lo(y), f2_hi(y));
+    }
   }
   o0 = make_uint4(w[0], w[1], w[2], w[3]);
   o1 = make_uint4(w[4], w[5], w[6], w[7]);
@@ -224,7 +258,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 2);     // TMA bytes + the producer's beta / metadata arrival
       mbar_init(&kready[s], kStTW);
       mbar_init(&empty[s], 1);
     }
@@ -241,6 +275,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
     tmem_relinquish();
   }
   if (warp >= kStTW0) rope_build(tab, g, win, threadIdx.x - kStTW0 * 32, kStTW * 32);
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -249,9 +284,11 @@ __global__ void __launch_bounds__(kStThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // All lanes compute the tile's row metadata; lane 0 issues the copies.
+    // All lanes fetch beta and compute the tile's row metadata; lane 0 issues
+    // the copies.
     {
       const uint64_t pol = policy_evict_first();
+      const uint64_t pol_beta = policy_evict_last();
       long long it = 0;
       int issued = 0;
       for (long long w = wb; w < we; ++w, ++it) {
@@ -259,17 +296,34 @@ __global__ void __launch_bounds__(kStThreads, 1)
         const uint32_t ph = (uint32_t)((it / kStStages) & 1);
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
         const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
-        const int n0 = (int)(w % tph) * kTcTile;
+        const int n0 = (int)(w % tph) * kStTile;
+        // Lane 0 starts the tile copies first; then the warp fetches beta and
+        // the row metadata while they are in flight, and arrives once more.
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], 2 * kStTileBytes);
+          unsigned char* kt = sm + TcStateSmem::K + s * kStTileBytes;
+          unsigned char* vt = sm + TcStateSmem::V + s * kStTileBytes;
+          tma_load_3d(kt, &tmK, &full[s], h * 128, n0, b, pol);
+          tma_load_3d(kt + kStBox, &tmK, &full[s], h * 128 + 64, n0, b, pol);
+          tma_load_3d(vt, &tmV, &full[s], h * 128, n0, b, pol);
+          tma_load_3d(vt + kStBox, &tmV, &full[s], h * 128 + 64, n0, b, pol);
+        }
+        float* bs = reinterpret_cast<float*>(sm + TcStateSmem::BETA + s * kStTile * 4);
+#pragma unroll
+        for (int k2 = 0; k2 < kStTile / 32; ++k2) {
+          const int n = n0 + lane + 32 * k2;
+          float bv = 0.f;
+          if (n < g.N) {
+            const uint16_t raw = ld_u16_policy(p.beta + ((size_t)b * g.N + n) * g.Hh + h, pol_beta);
+            bv = __uint_as_float((uint32_t)raw << 16);
+          }
+          bs[lane + 32 * k2] = bv;
+        }
         if (g.rope_on)
-          tile_rowpos(g, win, n0, lane, reinterpret_cast<uint2*>(sm + TcStateSmem::ROWPOS + s * 1024));
+          tile_rowpos<kStTile>(g, win, n0, lane,
+                               reinterpret_cast<uint2*>(sm + TcStateSmem::ROWPOS + s * kStTile * 8));
         __syncwarp();
-        if (lane != 0) { ++issued; continue; }
-        mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);        unsigned char* kt = sm + TcStateSmem::K + s * kTileBytes;
-        unsigned char* vt = sm + TcStateSmem::V + s * kTileBytes;
-        tma_load_3d(kt, &tmK, &full[s], h * 128, n0, b, pol);
-        tma_load_3d(kt + kBox, &tmK, &full[s], h * 128 + 64, n0, b, pol);
-        tma_load_3d(vt, &tmV, &full[s], h * 128, n0, b, pol);
-        tma_load_3d(vt + kBox, &tmV, &full[s], h * 128 + 64, n0, b, pol);
+        if (lane == 0) mbar_arrive(&full[s]);
         ++issued;
       }
       if (*abort_flag && lane == 0) {
@@ -297,12 +351,12 @@ __global__ void __launch_bounds__(kStThreads, 1)
           break;
         if (!mbar_wait(&kready[s], ph, abort_flag)) break;
         tc_fence_after();
-        const uint32_t kt = sbase + TcStateSmem::K + s * kTileBytes;
-        const uint32_t vt = sbase + TcStateSmem::V + s * kTileBytes;
+        const uint32_t kt = sbase + TcStateSmem::K + s * kStTileBytes;
+        const uint32_t vt = sbase + TcStateSmem::V + s * kStTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = sdesc_sw128(vt + kk * 2048, kBox, 1024);
-          const uint64_t bd = sdesc_sw128(kt + kk * 2048, kBox, 1024);
+        for (int kk = 0; kk < kStTile / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(vt + kk * 2048, kStBox, 1024);
+          const uint64_t bd = sdesc_sw128(kt + kk * 2048, kStBox, 1024);
           umma_f16kind(tmem + ab * 128, ad, bd, idesc, (first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&empty[s]);
@@ -319,14 +373,14 @@ __global__ void __launch_bounds__(kStThreads, 1)
   } else {
     // ------------------------------------------- transform warps: k -> beta k_til
     const int tw = warp - kStTW0;
-    const int rg = lane >> 3, j = lane & 7;
+    const int rg = tw_row(lane), j = tw_chunk(lane);
     LaneRope lr;
     lane_rope(g, j, lr);
-    const uint64_t pol_beta = policy_evict_last();
+    const uint32_t tab_s = smem_u32(tab);
     // This lane's two 16-byte chunks in row (tw*4 + rg) of a tile; rows of later
     // passes add whole multiples of 8 rows, which keeps the swizzle phase.
     uint32_t ch0, ch1;
-    lane_chunks(0, tw * 4 + rg, j, ch0, ch1);
+    lane_chunks(0, kStBox, tw * 4 + rg, j, ch0, ch1);
     f2_t zacc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) zacc[i] = 0ull;
@@ -337,31 +391,19 @@ __global__ void __launch_bounds__(kStThreads, 1)
       const int s = (int)(it % kStStages);
       const uint32_t ph = (uint32_t)((it / kStStages) & 1);
       const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
-      const int n0 = (int)(w % tph) * kTcTile;
-      constexpr int kPasses = (kTcTile + kStRowsPerPass - 1) / kStRowsPerPass;
-      static_assert(kPasses <= 4, "beta prefetch holds four rows");
-      float be[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ps = 0; ps < kPasses; ++ps) {
-        const int n = n0 + ps * kStRowsPerPass + tw * 4 + rg;
-        if (n < g.N && ps * kStRowsPerPass + tw * 4 < kTcTile) {
-          const uint16_t raw = ld_u16_policy(p.beta + ((size_t)b * g.N + n) * g.Hh + h, pol_beta);
-          be[ps] = __uint_as_float((uint32_t)raw << 16);
-        }
-      }
+      constexpr int kPasses = kStTile / kStRowsPerPass;
       if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
-      const uint32_t kt = sbase + TcStateSmem::K + s * kTileBytes;
+      const uint32_t kt = sbase + TcStateSmem::K + s * kStTileBytes;
 #pragma unroll 1
       for (int ps = 0; ps < kPasses; ++ps) {
         const int r = ps * kStRowsPerPass + tw * 4 + rg;
-        if (ps * kStRowsPerPass + tw * 4 >= kTcTile) break;
-        const float bcur = ps == 0 ? be[0] : (ps == 1 ? be[1] : (ps == 2 ? be[2] : be[3]));
+        const float bcur = reinterpret_cast<const float*>(sm + TcStateSmem::BETA + s * kStTile * 4)[r];
         const uint32_t a0 = kt + ch0 + ps * kStRowsPerPass * 128;
         const uint32_t a1 = kt + ch1 + ps * kStRowsPerPass * 128;
-        const float2* pA = tab;
-        int dE = 0;
+        uint32_t aA = 0;
+        int dB = 0;
         if (g.rope_on)
-          lane_rope_row(lr, tab, reinterpret_cast<const uint2*>(sm + TcStateSmem::ROWPOS + s * 1024)[r], pA, dE);
+          lane_rope_row(lr, tab_s, reinterpret_cast<const uint2*>(sm + TcStateSmem::ROWPOS + s * kStTile * 8)[r], aA, dB);
         f2_t x[8];
         unpack8(lds128(a0), lds128(a1), x);
         const float rstd = row_rstd(x);
@@ -372,7 +414,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
           zacc[i] = f2_fma(x[i], rstd2, zacc[i]);   // z += k_pls
         }
         uint4 o0, o1;
-        rope_scale_pack<false>(g, lr, pA, dE, x, rstd * bcur, o0, o1);
+        rope_scale_pack<false>(g, lr, aA, dB, x, rstd * bcur, o0, o1);
         sts128(a0, o0);
         sts128(a1, o1);
       }
@@ -390,8 +432,8 @@ __global__ void __launch_bounds__(kStThreads, 1)
           zf[2 * i + 1] = f2_hi(zacc[i]);
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          zf[i] += __shfl_xor_sync(0xffffffffu, zf[i], 8);
+        for (int i = 0; i < 16; ++i) {          // add the warp's four rows
+          zf[i] += __shfl_xor_sync(0xffffffffu, zf[i], 4);
           zf[i] += __shfl_xor_sync(0xffffffffu, zf[i], 16);
         }
         if (rg == 0) {
@@ -546,6 +588,9 @@ __global__ void __launch_bounds__(kApThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------- producer: S image + q
     // All lanes compute the tile's row metadata; lane 0 issues the copies.
+    // The S image, z and scale come from the combine kernel, which may still
+    // be running (programmatic dependent launch): wait for it first.
+    pdl_wait();
     {
       const uint64_t pol = policy_evict_first();
       long long it = 0;
@@ -568,7 +613,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
         if (!mbar_wait(&qempty[s], ph ^ 1u, abort_flag)) break;
         const int n0 = (int)(w % tph) * kTcTile;
         if (g.rope_on)
-          tile_rowpos(g, win, n0, lane, reinterpret_cast<uint2*>(sm + TcApplySmem::ROWPOS + s * 1024));
+          tile_rowpos<kTcTile>(g, win, n0, lane, reinterpret_cast<uint2*>(sm + TcApplySmem::ROWPOS + s * 1024));
         __syncwarp();
         if (lane != 0) { ++issued; continue; }
         mbar_arrive_expect_tx(&qfull[s], kTileBytes);
@@ -654,11 +699,12 @@ __global__ void __launch_bounds__(kApThreads, 1)
   } else if (warp < kApEW0) {
     // ------------------------------------ transform warps: q -> q_til, den
     const int tw = warp - kApTW0;
-    const int rg = lane >> 3, j = lane & 7;
+    const int rg = tw_row(lane), j = tw_chunk(lane);
     LaneRope lr;
     lane_rope(g, j, lr);
+    const uint32_t tab_s = smem_u32(tab);
     uint32_t ch0, ch1;
-    lane_chunks(0, tw * 4 + rg, j, ch0, ch1);
+    lane_chunks(0, kBox, tw * 4 + rg, j, ch0, ch1);
     f2_t zr[8];
     float hscale = 1.f;
     long long it = 0;
@@ -684,10 +730,10 @@ __global__ void __launch_bounds__(kApThreads, 1)
         const int n = n0 + r;
         const uint32_t a0 = qt + ch0 + ps * kApRowsPerPass * 128;
         const uint32_t a1 = qt + ch1 + ps * kApRowsPerPass * 128;
-        const float2* pA = tab;
-        int dE = 0;
+        uint32_t aA = 0;
+        int dB = 0;
         if (g.rope_on)
-          lane_rope_row(lr, tab, reinterpret_cast<const uint2*>(sm + TcApplySmem::ROWPOS + s * 1024)[r], pA, dE);
+          lane_rope_row(lr, tab_s, reinterpret_cast<const uint2*>(sm + TcApplySmem::ROWPOS + s * 1024)[r], aA, dB);
         f2_t x[8];
         unpack8(lds128(a0), lds128(a1), x);
         const float rstd = row_rstd(x);
@@ -698,13 +744,11 @@ __global__ void __launch_bounds__(kApThreads, 1)
           dp2 = f2_fma(zr[i], x[i], dp2);
         }
         uint4 o0, o1;
-        rope_scale_pack<true>(g, lr, pA, dE, x, rstd, o0, o1);
+        rope_scale_pack<true>(g, lr, aA, dB, x, rstd, o0, o1);
         sts128(a0, o0);
         sts128(a1, o1);
         float dp = f2_lo(dp2) + f2_hi(dp2);
-        dp += __shfl_xor_sync(0xffffffffu, dp, 1);
-        dp += __shfl_xor_sync(0xffffffffu, dp, 2);
-        dp += __shfl_xor_sync(0xffffffffu, dp, 4);
+        dp = row_sum(dp);
         const float dn = fmaf(dp, rstd, g.eps);      // z . q_pls + eps
         if (j == 0) {
           // The read-out sees S * scale; fold the scale into the denominator.
@@ -839,13 +883,13 @@ inline EncodeTiledFn encode_fn() {
 }
 
 // [B][N][Hh][128] bf16 activations as a 3D map (channel, token, batch) with
-// boxes of 64 channels x 128 tokens, 128-byte swizzle, zero fill past N.
-inline bool make_act_map(CUtensorMap* m, const void* ptr, const Geom& g) {
+// boxes of 64 channels x `rows` tokens, 128-byte swizzle, zero fill past N.
+inline bool make_act_map(CUtensorMap* m, const void* ptr, const Geom& g, uint32_t rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)g.Hh * 128, (cuuint64_t)g.N, (cuuint64_t)g.B};
   cuuint64_t strides[2] = {(cuuint64_t)g.Hh * 128 * 2, (cuuint64_t)g.N * g.Hh * 128 * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -861,7 +905,16 @@ inline size_t tc_apply_smem(int tab_entries) {
 }
 constexpr size_t kMaxSmem = 232448;
 
-// Per-CTA RoPE table size of the tensor partition (max over CTAs).
+// The state reduction and the read-out split the same items differently
+// (96- and 128-token tiles); each CTA count is at most the SM count.
+inline Partition tc_state_partition(const Geom& g, int sms) {
+  return make_partition(g.B * g.Hh, g.N, kStTile, sms);
+}
+inline Partition tc_apply_partition(const Geom& g, int sms) {
+  return make_partition(g.B * g.Hh, g.N, kTcTile, sms);
+}
+
+// Per-CTA RoPE table size of a tensor partition (max over CTAs).
 inline int tc_table_entries(const Geom& g, const Partition& part) {
   if (!g.rope_on) return 1;
   int mx = 1;
@@ -885,53 +938,72 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   if (sms <= 0) return GLA_ERR_CUDA;
   if (g.H >= (1 << kPosBits) || g.W >= (1 << kPosBits) || g.T >= (1 << kPosBits))
     return GLA_ERR_UNSUPPORTED;
-  const Partition part = make_partition(g.B * g.Hh, g.N, kTcTile, sms);
-  const int tab = tc_table_entries(g, part);
-  const size_t smem_st = tc_state_smem(tab), smem_ap = tc_apply_smem(tab);
+  const Partition spart = tc_state_partition(g, sms);
+  const Partition part = tc_apply_partition(g, sms);
+  const int stab = tc_table_entries(g, spart), tab = tc_table_entries(g, part);
+  const size_t smem_st = tc_state_smem(stab), smem_ap = tc_apply_smem(tab);
   if (smem_st > kMaxSmem || smem_ap > kMaxSmem) return GLA_ERR_UNSUPPORTED;
 
   CUtensorMap mK, mV, mQ, mG, mO;
-  if (!make_act_map(&mK, k, g) || !make_act_map(&mV, v, g) || !make_act_map(&mQ, q, g) ||
-      !make_act_map(&mG, gate, g) || !make_act_map(&mO, out, g))
+  if (!make_act_map(&mK, k, g, kStTile) || !make_act_map(&mV, v, g, kStTile) ||
+      !make_act_map(&mQ, q, g, kTcTile) || !make_act_map(&mG, gate, g, kTcTile) ||
+      !make_act_map(&mO, out, g, kTcTile))
     return GLA_ERR_CUDA;
 
   TcStateParams sp;
-  sp.g = g; sp.part = part;
+  sp.g = g; sp.part = spart;
   sp.beta = static_cast<const __nv_bfloat16*>(beta);
-  sp.part_S = part_S; sp.part_z = part_z; sp.tab_entries = tab;
+  sp.part_S = part_S; sp.part_z = part_z; sp.tab_entries = stab;
   if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem_st) != cudaSuccess)
     return GLA_ERR_CUDA;
   if (mark(0) != cudaSuccess) return GLA_ERR_CUDA;
-  tc_state_kernel<<<part.grid, kStThreads, smem_st, stream>>>(mK, mV, sp);
+  tc_state_kernel<<<spart.grid, kStThreads, smem_st, stream>>>(mK, mV, sp);
   if (cudaGetLastError() != cudaSuccess || mark(1) != cudaSuccess) return GLA_ERR_CUDA;
 
   CombineParams cp;
-  cp.part = part; cp.d = 128; cp.zparts = kStTW;
+  cp.part = spart; cp.d = 128; cp.zparts = kStTW;
   cp.part_S = part_S; cp.part_z = part_z;
   cp.S_in = carry ? S : nullptr;
   cp.z_in = carry ? z : nullptr;
   cp.S_out = S; cp.z_out = z; cp.S_img = S_img; cp.S_scale = S_scale;
-  dim3 cgrid(kCombineCluster, g.B * g.Hh);
-  combine_kernel<<<cgrid, kCombineThreads, 0, stream>>>(cp);
-  if (cudaGetLastError() != cudaSuccess || mark(2) != cudaSuccess) return GLA_ERR_CUDA;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cc = {};
+  cc.gridDim = dim3(kCombineCluster, g.B * g.Hh);
+  cc.blockDim = dim3(kCombineThreads);
+  cc.dynamicSmemBytes = 0;
+  cc.stream = stream;
+  cc.attrs = pdl;
+  cc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cc, combine_kernel, cp) != cudaSuccess || mark(2) != cudaSuccess)
+    return GLA_ERR_CUDA;
 
   TcApplyParams ap;
   ap.g = g; ap.part = part; ap.S_img = S_img; ap.S_scale = S_scale; ap.z = z;
   ap.den_out = den_dbg; ap.x_out = x_dbg; ap.tab_entries = tab;
   const bool dbg = den_dbg != nullptr || x_dbg != nullptr;
+  cudaLaunchConfig_t ac = {};
+  ac.gridDim = dim3(part.grid);
+  ac.blockDim = dim3(kApThreads);
+  ac.dynamicSmemBytes = smem_ap;
+  ac.stream = stream;
+  ac.attrs = pdl;
+  ac.numAttrs = 1;
+  cudaError_t e;
   if (dbg) {
     if (cudaFuncSetAttribute(tc_apply_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_ap) != cudaSuccess)
       return GLA_ERR_CUDA;
-    tc_apply_kernel<true><<<part.grid, kApThreads, smem_ap, stream>>>(mQ, mG, mO, ap);
+    e = cudaLaunchKernelEx(&ac, tc_apply_kernel<true>, mQ, mG, mO, ap);
   } else {
     if (cudaFuncSetAttribute(tc_apply_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_ap) != cudaSuccess)
       return GLA_ERR_CUDA;
-    tc_apply_kernel<false><<<part.grid, kApThreads, smem_ap, stream>>>(mQ, mG, mO, ap);
+    e = cudaLaunchKernelEx(&ac, tc_apply_kernel<false>, mQ, mG, mO, ap);
   }
-  if (cudaGetLastError() != cudaSuccess || mark(3) != cudaSuccess) return GLA_ERR_CUDA;
+  if (e != cudaSuccess || mark(3) != cudaSuccess) return GLA_ERR_CUDA;
   return GLA_OK;
 }
 

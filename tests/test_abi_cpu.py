@@ -106,12 +106,13 @@ def test_host_entry_rejects_bad_arguments():
 
 
 def test_plan_paths():
-    assert gla.gla_plan(2, 20, 128, 16, 23, 40, 1, 0, 148) == (148, 128, gla.GLA_PATH_TENSOR)
+    # tensor path: the state reduction walks 96-token tiles
+    assert gla.gla_plan(2, 20, 128, 16, 23, 40, 1, 0, 148) == (148, 96, gla.GLA_PATH_TENSOR)
     assert gla.gla_plan(1, 2, 32, 2, 4, 4, 0, 0, 148) == (2, 64, gla.GLA_PATH_SIMT)
     assert gla.gla_plan(2, 20, 128, 16, 23, 40, 1, gla.GLA_PATH_SIMT, 148)[2] == gla.GLA_PATH_SIMT
-    # 20 heads x 22 tiles of 128 tokens = 440 items >= 148 CTAs
+    # 20 heads x 29 tiles of 96 tokens = 580 items >= 148 CTAs
     assert gla.gla_plan(1, 20, 128, 3, 23, 40, 1, 0, 148)[0] == 148
-    # fewer items than SMs: one CTA per item
-    assert gla.gla_plan(1, 2, 128, 1, 1, 100, 1, 0, 148)[0] == 2
+    # fewer items than SMs: one CTA per item (2 heads x 2 tiles of 96 tokens)
+    assert gla.gla_plan(1, 2, 128, 1, 1, 100, 1, 0, 148)[0] == 4
     with pytest.raises(gla.GlaError):
         gla.gla_plan(1, 2, 32, 2, 4, 4, 0, gla.GLA_PATH_TENSOR, 148)
