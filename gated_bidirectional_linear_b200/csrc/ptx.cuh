@@ -141,6 +141,10 @@ __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
@@ -331,14 +335,10 @@ __device__ __forceinline__ f2_t f2(float lo, float hi) {
   return r;
 }
 __device__ __forceinline__ float f2_lo(f2_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
+  return __uint_as_float((uint32_t)(v & 0xFFFFFFFFull));
 }
 __device__ __forceinline__ float f2_hi(f2_t v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
+  return __uint_as_float((uint32_t)(v >> 32));
 }
 __device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
   f2_t d;

@@ -67,6 +67,46 @@ struct TcStateParams {
   int tab_entries;
 };
 
+// A CTA's items in order, advanced without divisions: head bh (batch b and
+// head h), tile ti inside the head, and whether the item opens (first) or
+// closes (last) one of the CTA's head segments.
+struct ItemWalk {
+  int tph, Hh, bh, b, h, ti, left;
+  bool first, last;
+  __device__ __forceinline__ ItemWalk(long long wb, long long we, int tph_, int Hh_)
+      : tph(tph_), Hh(Hh_) {
+    bh = (int)(wb / tph);
+    ti = (int)(wb - (long long)bh * tph);
+    b = bh / Hh;
+    h = bh - b * Hh;
+    left = (int)(we - wb);
+    first = true;
+    last = ti == tph - 1 || left == 1;
+  }
+  __device__ __forceinline__ bool more() const { return left > 0; }
+  __device__ __forceinline__ void next() {
+    --left;
+    first = false;
+    if (++ti == tph) {
+      ti = 0;
+      ++bh;
+      if (++h == Hh) { h = 0; ++b; }
+      first = true;
+    }
+    last = ti == tph - 1 || left == 1;
+  }
+};
+
+// Slot and phase parity of a ring of N buffers.
+template <int N>
+struct RingPos {
+  int s = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void next() {
+    if (++s == N) { s = 0; ph ^= 1u; }
+  }
+};
+
 __device__ __forceinline__ bool seg_first(const Partition& p, long long w, long long wb) {
   return w == wb || (w % p.tiles_per_head) == 0;
 }
@@ -291,12 +331,13 @@ __global__ void __launch_bounds__(kStThreads, 1)
       const uint64_t pol_beta = policy_evict_last();
       long long it = 0;
       int issued = 0;
-      for (long long w = wb; w < we; ++w, ++it) {
-        const int s = (int)(it % kStStages);
-        const uint32_t ph = (uint32_t)((it / kStStages) & 1);
-        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) break;
-        const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
-        const int n0 = (int)(w % tph) * kStTile;
+      ItemWalk iw(wb, we, tph, g.Hh);
+      RingPos<kStStages> rp;
+      for (; iw.more(); iw.next(), rp.next(), ++it) {
+        const int s = rp.s;
+        if (!mbar_wait(&empty[s], rp.ph ^ 1u, abort_flag)) break;
+        const int b = iw.b, h = iw.h;
+        const int n0 = iw.ti * kStTile;
         // Lane 0 starts the tile copies first; then the warp fetches beta and
         // the row metadata while they are in flight, and arrives once more.
         if (lane == 0) {
@@ -340,12 +381,13 @@ __global__ void __launch_bounds__(kStThreads, 1)
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(128, 128, true, true);
-      long long it = 0;
       int seg = 0;
-      for (long long w = wb; w < we; ++w, ++it) {
-        const int s = (int)(it % kStStages);
-        const uint32_t ph = (uint32_t)((it / kStStages) & 1);
-        const bool first = seg_first(part, w, wb), last = seg_last(part, w, we);
+      ItemWalk iw(wb, we, tph, g.Hh);
+      RingPos<kStStages> rp;
+      for (; iw.more(); iw.next(), rp.next()) {
+        const int s = rp.s;
+        const uint32_t ph = rp.ph;
+        const bool first = iw.first, last = iw.last;
         const int ab = seg & 1;
         if (first && !mbar_wait(&accempty[ab], (uint32_t)(((seg >> 1) & 1) ^ 1), abort_flag))
           break;
@@ -384,13 +426,14 @@ __global__ void __launch_bounds__(kStThreads, 1)
     f2_t zacc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) zacc[i] = 0ull;
-    long long it = 0;
     int seg = 0;
     bool ok = true;
-    for (long long w = wb; w < we && ok; ++w, ++it) {
-      const int s = (int)(it % kStStages);
-      const uint32_t ph = (uint32_t)((it / kStStages) & 1);
-      const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
+    ItemWalk iw(wb, we, tph, g.Hh);
+    RingPos<kStStages> rp;
+    for (; iw.more() && ok; iw.next(), rp.next()) {
+      const int s = rp.s;
+      const uint32_t ph = rp.ph;
+      const int bh = iw.bh;
       constexpr int kPasses = kStTile / kStRowsPerPass;
       if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
       const uint32_t kt = sbase + TcStateSmem::K + s * kStTileBytes;
@@ -422,7 +465,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&kready[s]);
 
-      if (seg_last(part, w, we)) {
+      if (iw.last) {
         // z of this head segment: sum the warp's four row groups, then store
         // one partial per warp (the combine adds them in warp order).
         float zf[16];
@@ -487,10 +530,11 @@ constexpr int kApQ = 2;                      // q ring
 constexpr int kApG = 3;                      // g / out ring
 constexpr int kApAcc = 2;                    // TMEM accumulators
 constexpr int kApDen = kApQ + kApAcc;        // den ring
-constexpr int kApTW = 8;
-constexpr int kApTW0 = 3;                    // transform warps 3..10
-constexpr int kApEW0 = kApTW0 + kApTW;       // epilogue warps 11..18
-constexpr int kApEW = 4 * kApAcc;
+constexpr int kApTW = 12;
+constexpr int kApTW0 = 3;                    // transform warps 3..14
+constexpr int kApEW0 = kApTW0 + kApTW;       // epilogue warps 15..18
+constexpr int kApEWGroups = 1;               // groups of 4 epilogue warps
+constexpr int kApEW = 4 * kApEWGroups;
 constexpr int kApThreads = (kApEW0 + kApEW) * 32;
 constexpr int kApRowsPerPass = kApTW * 4;
 
@@ -595,9 +639,11 @@ __global__ void __launch_bounds__(kApThreads, 1)
       const uint64_t pol = policy_evict_first();
       long long it = 0;
       int seg = 0, issued = 0;
-      for (long long w = wb; w < we; ++w, ++it) {
-        const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
-        if (seg_first(part, w, wb)) {
+      ItemWalk iw(wb, we, tph, g.Hh);
+      RingPos<kApQ> rq;
+      for (; iw.more(); iw.next(), rq.next(), ++it) {
+        const int bh = iw.bh, b = iw.b, h = iw.h;
+        if (iw.first) {
           // Every lane waits, so the warp leaves the loop together on a timeout.
           if (!mbar_wait(sfree, (uint32_t)((seg & 1) ^ 1), abort_flag)) break;
           if (lane == 0) {
@@ -608,10 +654,9 @@ __global__ void __launch_bounds__(kApThreads, 1)
           }
           ++seg;
         }
-        const int s = (int)(it % kApQ);
-        const uint32_t ph = (uint32_t)((it / kApQ) & 1);
-        if (!mbar_wait(&qempty[s], ph ^ 1u, abort_flag)) break;
-        const int n0 = (int)(w % tph) * kTcTile;
+        const int s = rq.s;
+        if (!mbar_wait(&qempty[s], rq.ph ^ 1u, abort_flag)) break;
+        const int n0 = iw.ti * kTcTile;
         if (g.rope_on)
           tile_rowpos<kTcTile>(g, win, n0, lane, reinterpret_cast<uint2*>(sm + TcApplySmem::ROWPOS + s * 1024));
         __syncwarp();
@@ -639,12 +684,13 @@ __global__ void __launch_bounds__(kApThreads, 1)
       const uint64_t pol = policy_evict_first();
       long long it = 0;
       int issued = 0;
-      for (long long w = wb; w < we; ++w, ++it) {
-        const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
-        const int s = (int)(it % kApG);
-        const uint32_t ph = (uint32_t)((it / kApG) & 1);
-        if (!mbar_wait(&gempty[s], ph ^ 1u, abort_flag)) break;
-        const int n0 = (int)(w % tph) * kTcTile;
+      ItemWalk iw(wb, we, tph, g.Hh);
+      RingPos<kApG> rg_;
+      for (; iw.more(); iw.next(), rg_.next(), ++it) {
+        const int b = iw.b, h = iw.h;
+        const int s = rg_.s;
+        if (!mbar_wait(&gempty[s], rg_.ph ^ 1u, abort_flag)) break;
+        const int n0 = iw.ti * kTcTile;
         mbar_arrive_expect_tx(&gfull[s], kTileBytes);
         unsigned char* gt = sm + TcApplySmem::G + s * kTileBytes;
         tma_load_3d(gt, &tmG, &gfull[s], h * 128, n0, b, pol);
@@ -664,18 +710,18 @@ __global__ void __launch_bounds__(kApThreads, 1)
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(128, 128, false, false);
-      long long it = 0;
       int seg = 0;
       const uint32_t simg = sbase + TcApplySmem::SIMG;
-      for (long long w = wb; w < we; ++w, ++it) {
-        const bool first = seg_first(part, w, wb), last = seg_last(part, w, we);
+      ItemWalk iw(wb, we, tph, g.Hh);
+      RingPos<kApAcc> ra;
+      RingPos<kApQ> rq;
+      for (; iw.more(); iw.next(), ra.next(), rq.next()) {
+        const bool first = iw.first, last = iw.last;
         if (first && !mbar_wait(sfull, (uint32_t)(seg & 1), abort_flag)) break;
-        const int ab = (int)(it % kApAcc);
-        const uint32_t aph = (uint32_t)((it / kApAcc) & 1);
-        if (!mbar_wait(&accempty[ab], aph ^ 1u, abort_flag)) break;
-        const int s = (int)(it % kApQ);
-        const uint32_t ph = (uint32_t)((it / kApQ) & 1);
-        if (!mbar_wait(&qready[s], ph, abort_flag)) break;
+        const int ab = ra.s;
+        if (!mbar_wait(&accempty[ab], ra.ph ^ 1u, abort_flag)) break;
+        const int s = rq.s;
+        if (!mbar_wait(&qready[s], rq.ph, abort_flag)) break;
         tc_fence_after();
         const uint32_t qt = sbase + TcApplySmem::Q + s * kTileBytes;
 #pragma unroll
@@ -707,25 +753,27 @@ __global__ void __launch_bounds__(kApThreads, 1)
     lane_chunks(0, kBox, tw * 4 + rg, j, ch0, ch1);
     f2_t zr[8];
     float hscale = 1.f;
-    long long it = 0;
     int seg = 0;
-    for (long long w = wb; w < we; ++w, ++it) {
-      const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
-      if (seg_first(part, w, wb)) {
+    ItemWalk iw(wb, we, tph, g.Hh);
+    RingPos<kApQ> rq;
+    RingPos<kApDen> rd;
+    for (; iw.more(); iw.next(), rq.next(), rd.next()) {
+      const int b = iw.b, h = iw.h;
+      if (iw.first) {
         if (!mbar_wait(sfull, (uint32_t)(seg & 1), abort_flag)) break;
 #pragma unroll
         for (int i = 0; i < 8; ++i) zr[i] = f2(zs[16 * j + 2 * i], zs[16 * j + 2 * i + 1]);
         hscale = scl_s[0];
         ++seg;
       }
-      const int s = (int)(it % kApQ);
-      const uint32_t ph = (uint32_t)((it / kApQ) & 1);
-      if (!mbar_wait(&qfull[s], ph, abort_flag)) break;
-      const int n0 = (int)(w % tph) * kTcTile;
+      const int s = rq.s;
+      if (!mbar_wait(&qfull[s], rq.ph, abort_flag)) break;
+      const int n0 = iw.ti * kTcTile;
       const uint32_t qt = sbase + TcApplySmem::Q + s * kTileBytes;
-      float* den = den_ring + (it % kApDen) * 128;
+      float* den = den_ring + rd.s * 128;
 #pragma unroll 1
-      for (int ps = 0; ps < kTcTile / kApRowsPerPass; ++ps) {
+      for (int ps = 0; ps < (kTcTile + kApRowsPerPass - 1) / kApRowsPerPass; ++ps) {
+        if (ps * kApRowsPerPass + tw * 4 >= kTcTile) break;
         const int r = ps * kApRowsPerPass + tw * 4 + rg;
         const int n = n0 + r;
         const uint32_t a0 = qt + ch0 + ps * kApRowsPerPass * 128;
@@ -763,25 +811,29 @@ __global__ void __launch_bounds__(kApThreads, 1)
   } else {
     // ---------------------- epilogue warps: gate, denominator, RMSNorm, store
     const int ew = warp - kApEW0;
-    const int grp = ew >> 2;            // accumulator this group drains
+    const int grp = ew >> 2;            // this group takes every kApEWGroups-th tile
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const bool storer = (ew & 3) == 0 && lane == 0;
     const uint64_t pol = policy_evict_first();
-    long long it = 0;
-    for (long long w = wb; w < we; ++w, ++it) {
-      if ((int)(it % kApAcc) != grp) continue;
-      const int bh = (int)(w / tph), b = bh / g.Hh, h = bh % g.Hh;
-      const int n0 = (int)(w % tph) * kTcTile;
-      const uint32_t aph = (uint32_t)((it / kApAcc) & 1);
-      if (!mbar_wait(&accfull[grp], aph, abort_flag)) break;
+    int prev_gsl = -1;                  // g slot whose store may still be reading
+    ItemWalk iw(wb, we, tph, g.Hh);
+    RingPos<kApAcc> ra;
+    RingPos<kApG> rg_;
+    RingPos<kApDen> rd;
+    RingPos<kApEWGroups> rsel;
+    for (; iw.more(); iw.next(), ra.next(), rg_.next(), rd.next(), rsel.next()) {
+      if (rsel.s != grp) continue;
+      const int b = iw.b, h = iw.h;
+      const int n0 = iw.ti * kTcTile;
+      const int ab = ra.s;
+      if (!mbar_wait(&accfull[ab], ra.ph, abort_flag)) break;
       tc_fence_after();
-      const int gsl = (int)(it % kApG);
-      const uint32_t gph = (uint32_t)((it / kApG) & 1);
-      if (!mbar_wait(&gfull[gsl], gph, abort_flag)) break;
+      const int gsl = rg_.s;
+      if (!mbar_wait(&gfull[gsl], rg_.ph, abort_flag)) break;
       // sigma(g) / den' = (0.5 tanh(g/2) + 0.5) / den' = fma(hc, tanh(g/2), hc)
-      const float hc = 0.5f / den_ring[(it % kApDen) * 128 + row];
-      const uint32_t taddr = tmem + (uint32_t)(grp * 128) + ((uint32_t)(q4 * 32) << 16);
+      const float hc = 0.5f / den_ring[rd.s * 128 + row];
+      const uint32_t taddr = tmem + (uint32_t)(ab * 128) + ((uint32_t)(q4 * 32) << 16);
       const uint32_t gt = sbase + TcApplySmem::G + gsl * kTileBytes;
       const uint32_t grow = gt + (uint32_t)row * 128u;
       const uint32_t sw = (uint32_t)(row & 7);
@@ -840,18 +892,24 @@ __global__ void __launch_bounds__(kApThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[grp]);
+      if (lane == 0) mbar_arrive(&accempty[ab]);
       fence_proxy_async_smem();
       named_barrier(2 + grp, 128);
       if (storer) {
         tma_store_3d(&tmO, sm + TcApplySmem::G + gsl * kTileBytes, h * 128, n0, b, pol);
         tma_store_3d(&tmO, sm + TcApplySmem::G + gsl * kTileBytes + kBox, h * 128 + 64, n0, b, pol);
         bulk_commit();
-        bulk_wait_read_all();
-        mbar_arrive(&gempty[gsl]);
+        // Release the previous tile's slot once its store has read it; this
+        // tile's store keeps running while the group starts the next tile.
+        bulk_wait_read_1();
+        if (prev_gsl >= 0) mbar_arrive(&gempty[prev_gsl]);
+        prev_gsl = gsl;
       }
     }
-    if (storer) bulk_wait_all();
+    if (storer) {
+      bulk_wait_all();
+      if (prev_gsl >= 0) mbar_arrive(&gempty[prev_gsl]);
+    }
   }
 
   tc_fence_before();
