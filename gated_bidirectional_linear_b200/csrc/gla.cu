@@ -16,6 +16,25 @@
 
 using namespace gla;
 
+namespace gla {
+
+// One CTA waits on an mbarrier that no thread arrives on, through the
+// pipelines' bounded wait with a short limit, then returns (see
+// gla_selftest_wait_timeout).
+__global__ void __launch_bounds__(32) selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  mbar_wait_for(&bar, 0, reinterpret_cast<volatile int*>(&abort_flag), limit_ns);
+}
+
+}  // namespace gla
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -133,6 +152,7 @@ inline cudaError_t mark(const Call& c, int i) {
 // its tile rings; grids whose table does not fit use the CUDA-core path.
 bool tensor_fits(const Geom& g, int sms) {
   if (g.H >= (1 << kPosBits) || g.W >= (1 << kPosBits) || g.T >= (1 << kPosBits)) return false;
+  if (!tc_rope_lanes_ok(g)) return false;
   const int stab = tc_table_entries(g, tc_state_partition(g, sms));
   const int tab = tc_table_entries(g, tc_apply_partition(g, sms));
   return tc_state_smem(stab) <= kMaxSmem && tc_apply_smem(tab) <= kMaxSmem;
@@ -498,6 +518,13 @@ gla_status gla_forward_noalloc(const void* q, const void* k, const void* v, cons
   c.S_dbg = c.z_dbg = c.den_dbg = c.x_dbg = nullptr;
   c.events = nullptr;
   return run_call(c);
+}
+
+gla_status gla_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000u) return GLA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
 }
 
 gla_status gla_get_device_status(void* stream) {

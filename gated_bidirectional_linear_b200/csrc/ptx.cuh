@@ -74,20 +74,31 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Wait for the phase of `bar` with the given parity.  Gives up (returns false,
 // records kErrTimeout in the device error word and raises *abort) after
-// kWaitLimitNs, or as soon as another role of the CTA raised *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort) {
+// limit_ns, or as soon as another role of the CTA raised *abort.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    // The abort flag and the clock are looked at every 16th poll only, so a
+    // waiting warp takes few issue slots from the warps doing the work.
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_device_error, kErrTimeout);
       *abort = 1;
       return false;
     }
   }
+}
+
+// The pipelines' wait: limit kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // ------------------------------------------------ programmatic dependent launch
@@ -126,6 +137,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z),
       "l"(policy)
       : "memory");
+}
+
+// Bring a tile of a tensor map into L2 ahead of its load (no shared memory,
+// no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x,
@@ -268,6 +288,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
         "=r"(u[31])
       : "r"(taddr)
       : "memory");
+}
+
+// As tmem_ld32 with 8 consecutive columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&r)[8]) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(r);
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]),
+                 "=r"(u[6]), "=r"(u[7])
+               : "r"(taddr)
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&r)[32]) {

@@ -32,26 +32,30 @@ constexpr uint32_t kTileBytes = 2 * kBox;    // 128 tokens x 128 channels, 16-bi
 constexpr int kStTile = 96;                  // tokens per state tile (MMA K)
 constexpr uint32_t kStBox = kStTile * 128;   // 96 rows x 128 bytes
 constexpr uint32_t kStTileBytes = 2 * kStBox;
-constexpr int kPosBits = 11;                 // packed (t, h, w) offsets, < 2048 each
+constexpr int kPosBits = 11;                 // (t, h, w) positions, < 2048 each
+constexpr int kRecBytes = 20;                // per-row RoPE record (tile_rowrec)
 
 // --------------------------------------------------------------- state kernel
 
 constexpr int kStStages = 4;
-constexpr int kStTW = 12;                    // transform warps; the first four
-                                             // also drain finished S partials
+constexpr int kStTW = 12;                    // transform warps; they also drain
+                                             // finished S partials, three per
+                                             // TMEM lane quarter
 constexpr int kStTW0 = 2;                    // first transform warp
 constexpr int kStThreads = (kStTW0 + kStTW) * 32;
 static_assert(kStTW <= kMaxZPartsCombined, "combine adds at most this many z partials");
+static_assert(kStTW == 12, "the S drain splits each lane quarter over three warps");
 static_assert((kStTW * 4) % 8 == 0, "rows per pass keep the 8-row swizzle phase");
-static_assert(kStTile % (kStTW * 4) == 0, "whole passes per state tile");
+static_assert(kStTile % (kStTW * 4) == 0, "whole row groups per state tile");
 static_assert(kStTile % 16 == 0 && kStBox % 1024 == 0, "MMA K steps and swizzle atoms");
 constexpr int kStRowsPerPass = kStTW * 4;
+constexpr int kStRows = kStTile / kStRowsPerPass;   // row groups per transform warp
 
 struct TcStateSmem {
   static constexpr uint32_t K = 0;
   static constexpr uint32_t V = kStStages * kStTileBytes;
-  static constexpr uint32_t ROWPOS = 2 * kStStages * kStTileBytes;    // [stage][96] uint2
-  static constexpr uint32_t BETA = ROWPOS + kStStages * kStTile * 8;  // [stage][96] f32
+  static constexpr uint32_t ROWREC = 2 * kStStages * kStTileBytes;   // [stage][96] records
+  static constexpr uint32_t BETA = ROWREC + kStStages * kStTile * kRecBytes;  // [stage][96] f32
   static constexpr uint32_t BAR = BETA + kStStages * kStTile * 4;     // barriers
   static constexpr uint32_t NBAR = 3 * kStStages + 5;
   static constexpr uint32_t MISC = BAR + NBAR * 8;                     // tmem base, abort
@@ -114,13 +118,17 @@ __device__ __forceinline__ bool seg_last(const Partition& p, long long w, long l
   return w == we - 1 || ((w + 1) % p.tiles_per_head) == 0;
 }
 
-// Per-tile row metadata.  For every row r of a tile (token n0 + r) the
-// producer warp stores the byte offsets, inside the RoPE table, of the token's
-// time, height and width rows: (offT | offH << 16, offW).  The table is at
-// most 22.5 KB, so 16 bits hold each offset.
+// Per-tile row records.  For every row r of a tile (token n0 + r) the producer
+// warp stores the byte offsets, inside the RoPE table, of the token's time (T),
+// height (H) and width (W) rows as ten 16-bit words
+//   T T T H H H H W W W
+// so that for axes a <= b with b - a <= 1 (0 = T, 1 = H, 2 = W) the pair of
+// offsets (a, b) is the 32-bit word a + b of the record: TT, TH, HH, HW, WW.
+// The table is at most 22.5 KB, so 16 bits hold each offset.
+
 template <int kRows>
-__device__ __forceinline__ void tile_rowpos(const Geom& g, RopeWindow win, int n0, int lane,
-                                            uint2* rowpos) {
+__device__ __forceinline__ void tile_rowrec(const Geom& g, RopeWindow win, int n0, int lane,
+                                            unsigned char* rec) {
   const uint32_t HW = g.div_HW.d, W = g.div_W.d;
   const RopeLayout L = rope_layout(g, win.Lt);
 #pragma unroll
@@ -137,51 +145,72 @@ __device__ __forceinline__ void tile_rowpos(const Geom& g, RopeWindow win, int n
     const uint32_t offT = 8u * (uint32_t)(L.base[0] + tl * L.stride[0]);
     const uint32_t offH = 8u * (uint32_t)(L.base[1] + (int)hh * L.stride[1]);
     const uint32_t offW = 8u * (uint32_t)(L.base[2] + (int)ww * L.stride[2]);
-    rowpos[r] = make_uint2(offT | (offH << 16), offW);
+    uint32_t* q = reinterpret_cast<uint32_t*>(rec + r * kRecBytes);
+    q[0] = offT | (offT << 16);
+    q[1] = offT | (offH << 16);
+    q[2] = offH | (offH << 16);
+    q[3] = offH | (offW << 16);
+    q[4] = offW | (offW << 16);
   }
 }
 
 // Per-lane view of the RoPE table.  Lane j of a row group handles channels
-// 16j .. 16j+15, i.e. rotation pairs 8j .. 8j+7; for d = 128 every axis has at
-// least 21 pairs, so those 8 pairs lie on at most two axes A and B.  In the
-// table, pair 8j + i of axis X sits at column idx = 8j + i - start + j -
-// (start >> 3) of its row, so slot i of the lane is at byte
-//   offA(row) + inA + 8 i   (pairs on axis A)
-//   offB(row) + inB + 8 i   (pairs on axis B, useB[i] = 1)
-// where offX(row) is the row's metadata for axis X.
+// 16j .. 16j+15, i.e. rotation pairs 8j .. 8j+7 (slots 0..7); for d = 128 the
+// axes hold 22, 21 and 21 pairs, so a lane's slots lie on at most two axes A
+// and B, with slots 0..2 on A, slots 6..7 on B and slots 3..5 all on one of
+// them (tc_rope_lanes_ok checks this on the host).  In the table, pair 8j + i
+// of axis X sits at column idx = 8j + i - start + j - (start >> 3) of its row,
+// so slot i of the lane is at byte offX(row) + inX + 8 i.
 struct LaneRope {
-  int inA, inB;          // byte offset of pair p0 = 8j inside its axis row
-  int wA, shA, wB, shB;  // where offA / offB sit in the row metadata
-  int useB[8];
+  uint32_t cA, cB;       // table base + byte offset of pair 8j inside its A / B row
+  int rec;               // byte offset of the lane's (A, B) word in a row record
+  bool midB;             // slots 3..5 lie on axis B
 };
 
-__device__ __forceinline__ int axis_of(const Geom& g, int p) {
+__host__ __device__ inline int axis_of(const Geom& g, int p) {
   return p < g.pt ? 0 : (p < g.pt + g.ph ? 1 : 2);
 }
 
-__device__ __forceinline__ void lane_rope(const Geom& g, int j, LaneRope& lr) {
+// First slot of lane j on its second axis (8: the lane stays on one axis).
+__host__ __device__ inline int lane_split(const Geom& g, int j) {
+  const int aA = axis_of(g, 8 * j);
+  for (int i = 1; i < 8; ++i)
+    if (axis_of(g, 8 * j + i) != aA) return i;
+  return 8;
+}
+
+// The slot grouping above holds for every lane (d = 128 only).
+inline bool tc_rope_lanes_ok(const Geom& g) {
+  if (g.d != 128) return false;
+  for (int j = 0; j < 8; ++j) {
+    const int kb = lane_split(g, j);
+    if (kb != 3 && kb != 6 && kb != 8) return false;
+    if (axis_of(g, 8 * j + 7) - axis_of(g, 8 * j) > 1) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void lane_rope(const Geom& g, int j, uint32_t tab_s, LaneRope& lr) {
   const int p0 = 8 * j;
   const int start[3] = {0, g.pt, g.pt + g.ph};
   const int aA = axis_of(g, p0), aB = axis_of(g, p0 + 7);
-  lr.inA = 8 * (p0 - start[aA] + j - (start[aA] >> 3));
-  lr.inB = 8 * (p0 - start[aB] + j - (start[aB] >> 3));
-  lr.wA = aA == 2 ? 1 : 0;
-  lr.shA = aA == 1 ? 16 : 0;
-  lr.wB = aB == 2 ? 1 : 0;
-  lr.shB = aB == 1 ? 16 : 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) lr.useB[i] = axis_of(g, p0 + i) != aA ? 1 : 0;
+  lr.cA = tab_s + (uint32_t)(8 * (p0 - start[aA] + j - (start[aA] >> 3)));
+  lr.cB = tab_s + (uint32_t)(8 * (p0 - start[aB] + j - (start[aB] >> 3)));
+  lr.rec = 4 * (aA + aB);
+  lr.midB = lane_split(g, j) == 3;
 }
 
-// Shared-memory address of the lane's pair-0 table entry for a row, and the
-// byte distance from its axis-A run to its axis-B run.
-__device__ __forceinline__ void lane_rope_row(const LaneRope& lr, uint32_t tab_s, uint2 m,
-                                              uint32_t& aA, int& dB) {
-  const uint32_t offA = ((lr.wA ? m.y : m.x) >> lr.shA) & 0xFFFFu;
-  const uint32_t offB = ((lr.wB ? m.y : m.x) >> lr.shB) & 0xFFFFu;
-  const int bA = (int)offA + lr.inA, bB = (int)offB + lr.inB;
-  aA = tab_s + (uint32_t)bA;
-  dB = bB - bA;
+// Shared-memory addresses of the lane's slots 0..2, 3..5 and 6..7 runs for the
+// row whose record starts at rec_row.
+__device__ __forceinline__ void lane_rope_row(const LaneRope& lr, uint32_t rec_row,
+                                              uint32_t& a012, uint32_t& a345, uint32_t& a67) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(rec_row + (uint32_t)lr.rec));
+  const uint32_t aA = (v & 0xFFFFu) + lr.cA;
+  const uint32_t aB = (v >> 16) + lr.cB;
+  a012 = aA;
+  a67 = aB;
+  a345 = lr.midB ? aB : aA;
 }
 
 // Shared-memory addresses of the two 16-byte chunks a lane owns in row r of a
@@ -232,25 +261,29 @@ __device__ __forceinline__ f2_t f2_relu(f2_t x) {
 #define GLA_TAB_LOAD(I, base, out)                                              \
   asm volatile("ld.shared.b64 %0, [%1+%2];" : "=l"(out) : "r"(base), "n"(8 * (I)))
 
-// Rotate the lane's 8 ReLU'd pairs r (still unnormalised), scaled by `scl`:
-// y = scl * RoPE(r), packed to bf16 (kHalf = false) or fp16.
+// The lane's 8 (cos, sin) entries of one row (see LaneRope).
+__device__ __forceinline__ void tab_load8(uint32_t a012, uint32_t a345, uint32_t a67,
+                                          f2_t (&e)[8]) {
+  GLA_TAB_LOAD(0, a012, e[0]);
+  GLA_TAB_LOAD(1, a012, e[1]);
+  GLA_TAB_LOAD(2, a012, e[2]);
+  GLA_TAB_LOAD(3, a345, e[3]);
+  GLA_TAB_LOAD(4, a345, e[4]);
+  GLA_TAB_LOAD(5, a345, e[5]);
+  GLA_TAB_LOAD(6, a67, e[6]);
+  GLA_TAB_LOAD(7, a67, e[7]);
+}
+
+// Rotate the lane's 8 ReLU'd pairs r (still unnormalised) by the entries e,
+// scaled by `scl`: y = scl * RoPE(r), packed to bf16 (kHalf = false) or fp16.
+// Without RoPE the entries are ignored.
 template <bool kHalf>
-__device__ __forceinline__ void rope_scale_pack(const Geom& g, const LaneRope& lr,
-                                                uint32_t aA, int dB,
+__device__ __forceinline__ void rope_scale_pack(bool rope_on, const f2_t (&e)[8],
                                                 const f2_t (&r)[8], float scl, uint4& o0,
                                                 uint4& o1) {
   uint32_t w[8];
   const f2_t scl2 = f2(scl, scl);
-  if (g.rope_on) {
-    f2_t e[8];
-    GLA_TAB_LOAD(0, aA + (uint32_t)(lr.useB[0] * dB), e[0]);
-    GLA_TAB_LOAD(1, aA + (uint32_t)(lr.useB[1] * dB), e[1]);
-    GLA_TAB_LOAD(2, aA + (uint32_t)(lr.useB[2] * dB), e[2]);
-    GLA_TAB_LOAD(3, aA + (uint32_t)(lr.useB[3] * dB), e[3]);
-    GLA_TAB_LOAD(4, aA + (uint32_t)(lr.useB[4] * dB), e[4]);
-    GLA_TAB_LOAD(5, aA + (uint32_t)(lr.useB[5] * dB), e[5]);
-    GLA_TAB_LOAD(6, aA + (uint32_t)(lr.useB[6] * dB), e[6]);
-    GLA_TAB_LOAD(7, aA + (uint32_t)(lr.useB[7] * dB), e[7]);
+  if (rope_on) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float r0 = f2_lo(r[i]), r1 = f2_hi(r[i]);
@@ -304,7 +337,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&accfull[a], 1);
-      mbar_init(&accempty[a], 4);
+      mbar_init(&accempty[a], kStTW);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -314,7 +347,6 @@ __global__ void __launch_bounds__(kStThreads, 1)
     tmem_alloc(tmem_holder, 256);
     tmem_relinquish();
   }
-  if (warp >= kStTW0) rope_build(tab, g, win, threadIdx.x - kStTW0 * 32, kStTW * 32);
   pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
@@ -333,13 +365,26 @@ __global__ void __launch_bounds__(kStThreads, 1)
       int issued = 0;
       ItemWalk iw(wb, we, tph, g.Hh);
       RingPos<kStStages> rp;
+      // beta of the item about to be issued, fetched one item ahead so that
+      // its global-load latency overlaps the wait for a free stage.
+      uint16_t braw[kStTile / 32];
+      auto fetch_beta = [&](const ItemWalk& w) {
+#pragma unroll
+        for (int k2 = 0; k2 < kStTile / 32; ++k2) {
+          const int n = w.ti * kStTile + lane + 32 * k2;
+          braw[k2] = n < g.N ? ld_u16_policy(p.beta + ((size_t)w.b * g.N + n) * g.Hh + w.h, pol_beta)
+                             : (uint16_t)0;
+        }
+      };
+      if (iw.more()) fetch_beta(iw);
       for (; iw.more(); iw.next(), rp.next(), ++it) {
         const int s = rp.s;
         if (!mbar_wait(&empty[s], rp.ph ^ 1u, abort_flag)) break;
         const int b = iw.b, h = iw.h;
         const int n0 = iw.ti * kStTile;
-        // Lane 0 starts the tile copies first; then the warp fetches beta and
-        // the row metadata while they are in flight, and arrives once more.
+        // Lane 0 starts the tile copies first; then the warp stores beta,
+        // prefetches the next item's, computes the row metadata and arrives
+        // once more.
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], 2 * kStTileBytes);
           unsigned char* kt = sm + TcStateSmem::K + s * kStTileBytes;
@@ -351,18 +396,16 @@ __global__ void __launch_bounds__(kStThreads, 1)
         }
         float* bs = reinterpret_cast<float*>(sm + TcStateSmem::BETA + s * kStTile * 4);
 #pragma unroll
-        for (int k2 = 0; k2 < kStTile / 32; ++k2) {
-          const int n = n0 + lane + 32 * k2;
-          float bv = 0.f;
-          if (n < g.N) {
-            const uint16_t raw = ld_u16_policy(p.beta + ((size_t)b * g.N + n) * g.Hh + h, pol_beta);
-            bv = __uint_as_float((uint32_t)raw << 16);
-          }
-          bs[lane + 32 * k2] = bv;
+        for (int k2 = 0; k2 < kStTile / 32; ++k2)
+          bs[lane + 32 * k2] = __uint_as_float((uint32_t)braw[k2] << 16);
+        {
+          ItemWalk nx = iw;
+          nx.next();
+          if (nx.more()) fetch_beta(nx);
         }
         if (g.rope_on)
-          tile_rowpos<kStTile>(g, win, n0, lane,
-                               reinterpret_cast<uint2*>(sm + TcStateSmem::ROWPOS + s * kStTile * 8));
+          tile_rowrec<kStTile>(g, win, n0, lane,
+                               sm + TcStateSmem::ROWREC + s * kStTile * kRecBytes);
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[s]);
         ++issued;
@@ -414,11 +457,13 @@ __global__ void __launch_bounds__(kStThreads, 1)
     }
   } else {
     // ------------------------------------------- transform warps: k -> beta k_til
+    // The RoPE table is built here, while the first tiles are in flight.
+    rope_build(tab, g, win, threadIdx.x - kStTW0 * 32, kStTW * 32);
+    named_barrier(1, kStTW * 32);
     const int tw = warp - kStTW0;
     const int rg = tw_row(lane), j = tw_chunk(lane);
     LaneRope lr;
-    lane_rope(g, j, lr);
-    const uint32_t tab_s = smem_u32(tab);
+    lane_rope(g, j, smem_u32(tab), lr);
     // This lane's two 16-byte chunks in row (tw*4 + rg) of a tile; rows of later
     // passes add whole multiples of 8 rows, which keeps the swizzle phase.
     uint32_t ch0, ch1;
@@ -434,21 +479,38 @@ __global__ void __launch_bounds__(kStThreads, 1)
       const int s = rp.s;
       const uint32_t ph = rp.ph;
       const int bh = iw.bh;
-      constexpr int kPasses = kStTile / kStRowsPerPass;
       if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
       const uint32_t kt = sbase + TcStateSmem::K + s * kStTileBytes;
-#pragma unroll 1
-      for (int ps = 0; ps < kPasses; ++ps) {
-        const int r = ps * kStRowsPerPass + tw * 4 + rg;
-        const float bcur = reinterpret_cast<const float*>(sm + TcStateSmem::BETA + s * kStTile * 4)[r];
-        const uint32_t a0 = kt + ch0 + ps * kStRowsPerPass * 128;
-        const uint32_t a1 = kt + ch1 + ps * kStRowsPerPass * 128;
-        uint32_t aA = 0;
-        int dB = 0;
-        if (g.rope_on)
-          lane_rope_row(lr, tab_s, reinterpret_cast<const uint2*>(sm + TcStateSmem::ROWPOS + s * kStTile * 8)[r], aA, dB);
+      const float* bs = reinterpret_cast<const float*>(sm + TcStateSmem::BETA + s * kStTile * 4);
+      const uint32_t rec_s = sbase + TcStateSmem::ROWREC + s * kStTile * kRecBytes;
+      // The warp's kStRows row groups of the tile (4 rows each, kStRowsPerPass
+      // apart) are processed together: all shared loads first, then each row
+      // group's arithmetic and stores.
+      uint32_t a0[kStRows], a1[kStRows], t012[kStRows], t345[kStRows], t67[kStRows];
+      float bcur[kStRows];
+      uint4 in0[kStRows], in1[kStRows];
+      f2_t e[kStRows][8];
+#pragma unroll
+      for (int u = 0; u < kStRows; ++u) {
+        const int r = u * kStRowsPerPass + tw * 4 + rg;
+        a0[u] = kt + ch0 + u * kStRowsPerPass * 128;
+        a1[u] = kt + ch1 + u * kStRowsPerPass * 128;
+        bcur[u] = bs[r];
+        if (g.rope_on) lane_rope_row(lr, rec_s + r * kRecBytes, t012[u], t345[u], t67[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kStRows; ++u) {
+        in0[u] = lds128(a0[u]);
+        in1[u] = lds128(a1[u]);
+      }
+      if (g.rope_on) {
+#pragma unroll
+        for (int u = 0; u < kStRows; ++u) tab_load8(t012[u], t345[u], t67[u], e[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kStRows; ++u) {
         f2_t x[8];
-        unpack8(lds128(a0), lds128(a1), x);
+        unpack8(in0[u], in1[u], x);
         const float rstd = row_rstd(x);
         const f2_t rstd2 = f2(rstd, rstd);
 #pragma unroll
@@ -457,9 +519,9 @@ __global__ void __launch_bounds__(kStThreads, 1)
           zacc[i] = f2_fma(x[i], rstd2, zacc[i]);   // z += k_pls
         }
         uint4 o0, o1;
-        rope_scale_pack<false>(g, lr, aA, dB, x, rstd * bcur, o0, o1);
-        sts128(a0, o0);
-        sts128(a1, o1);
+        rope_scale_pack<false>(g.rope_on, e[u], x, rstd * bcur[u], o0, o1);
+        sts128(a0[u], o0);
+        sts128(a1[u], o1);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -488,24 +550,24 @@ __global__ void __launch_bounds__(kStThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) zacc[i] = 0ull;
 
-        // Warps tw = 0..3 (one per TMEM lane quarter) drain the finished
-        // accumulator: row a of the partial S is TMEM lane a.
-        if (tw < 4) {
+        // All transform warps drain the finished accumulator: row a of the
+        // partial S is TMEM lane a; the three warps of a lane quarter take
+        // every third group of 8 columns.
+        {
           const int q4 = warp & 3;
+          const int third = tw >> 2;
           const int a = q4 * 32 + lane;
           const int ab = seg & 1;
           if (!mbar_wait(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag)) { ok = false; break; }
           tc_fence_after();
           float* dst = p.part_S + ((size_t)c + bh) * 128 * 128 + (size_t)a * 128;
 #pragma unroll 1
-          for (int cb = 0; cb < 4; ++cb) {
-            float rr[32];
-            tmem_ld32(tmem + (uint32_t)(ab * 128 + cb * 32) + ((uint32_t)(q4 * 32) << 16), rr);
+          for (int cb = third; cb < 16; cb += 3) {
+            float rr[8];
+            tmem_ld8(tmem + (uint32_t)(ab * 128 + cb * 8) + ((uint32_t)(q4 * 32) << 16), rr);
             tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dst + cb * 32 + i) =
-                  make_float4(rr[i], rr[i + 1], rr[i + 2], rr[i + 3]);
+            *reinterpret_cast<float4*>(dst + cb * 8) = make_float4(rr[0], rr[1], rr[2], rr[3]);
+            *reinterpret_cast<float4*>(dst + cb * 8 + 4) = make_float4(rr[4], rr[5], rr[6], rr[7]);
           }
           tc_fence_before();
           __syncwarp();
@@ -530,13 +592,18 @@ constexpr int kApQ = 2;                      // q ring
 constexpr int kApG = 3;                      // g / out ring
 constexpr int kApAcc = 2;                    // TMEM accumulators
 constexpr int kApDen = kApQ + kApAcc;        // den ring
-constexpr int kApTW = 12;
-constexpr int kApTW0 = 3;                    // transform warps 3..14
-constexpr int kApEW0 = kApTW0 + kApTW;       // epilogue warps 15..18
-constexpr int kApEWGroups = 1;               // groups of 4 epilogue warps
-constexpr int kApEW = 4 * kApEWGroups;
-constexpr int kApThreads = (kApEW0 + kApEW) * 32;
-constexpr int kApRowsPerPass = kApTW * 4;
+constexpr int kApTW = 8;
+constexpr int kApIL = 2;                     // row groups a transform warp takes at once
+constexpr int kApTW0 = 3;                    // transform warps 3..10
+constexpr int kApEW0 = kApTW0 + kApTW;       // epilogue warps 11..14
+constexpr int kApEW = 4;                     // one per TMEM lane quarter
+constexpr int kApST = kApEW0 + kApEW;        // store warp 15
+constexpr int kApThreads = (kApST + 1) * 32;
+constexpr int kApPrefetch = 2;               // items ahead whose q, g tiles go to L2 early
+constexpr int kApRowsPerPass = kApTW * 4 * kApIL;
+constexpr int kApPasses = kTcTile / kApRowsPerPass;
+static_assert(kTcTile % kApRowsPerPass == 0, "whole passes per read-out tile");
+static_assert((kApTW * 4) % 8 == 0, "row groups keep the 8-row swizzle phase");
 
 struct TcApplySmem {
   static constexpr uint32_t Q = 0;
@@ -545,9 +612,9 @@ struct TcApplySmem {
   static constexpr uint32_t Z = SIMG + kTileBytes;         // z [128] f32
   static constexpr uint32_t SCL = Z + 512;                  // image scale [4] f32
   static constexpr uint32_t DEN = SCL + 16;                 // [kApDen][128] den*scale per tile
-  static constexpr uint32_t ROWPOS = DEN + kApDen * 512;    // [q slot][128] uint2
-  static constexpr uint32_t BAR = ROWPOS + kApQ * 1024;
-  static constexpr uint32_t NBAR = 3 * kApQ + 2 * kApG + 2 * kApAcc + 3;
+  static constexpr uint32_t ROWREC = DEN + kApDen * 512;    // [q slot][128] records
+  static constexpr uint32_t BAR = ROWREC + kApQ * kTcTile * kRecBytes;
+  static constexpr uint32_t NBAR = 3 * kApQ + 3 * kApG + 2 * kApAcc + 3;
   static constexpr uint32_t MISC = BAR + NBAR * 8;
   static constexpr uint32_t TAB = (MISC + 16 + 15) & ~15u;
 };
@@ -577,7 +644,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
   uint64_t* qempty = qready + kApQ;
   uint64_t* gfull = qempty + kApQ;
   uint64_t* gempty = gfull + kApG;
-  uint64_t* accfull = gempty + kApG;
+  uint64_t* ostaged = gempty + kApG;
+  uint64_t* accfull = ostaged + kApG;
   uint64_t* accempty = accfull + kApAcc;
   uint64_t* sfull = accempty + kApAcc;
   uint64_t* sfree = sfull + 1;
@@ -606,6 +674,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
     for (int s = 0; s < kApG; ++s) {
       mbar_init(&gfull[s], 1);
       mbar_init(&gempty[s], 1);
+      mbar_init(&ostaged[s], kApEW);
     }
     for (int a = 0; a < kApAcc; ++a) {
       mbar_init(&accfull[a], 1);
@@ -621,8 +690,6 @@ __global__ void __launch_bounds__(kApThreads, 1)
     tmem_alloc(tmem_holder, 256);
     tmem_relinquish();
   }
-  if (warp >= kApTW0 && warp < kApEW0)
-    rope_build(tab, g, win, threadIdx.x - kApTW0 * 32, kApTW * 32);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -640,9 +707,18 @@ __global__ void __launch_bounds__(kApThreads, 1)
       long long it = 0;
       int seg = 0, issued = 0;
       ItemWalk iw(wb, we, tph, g.Hh);
+      ItemWalk ahead = iw;      // the item kApPrefetch ahead of iw
+      for (int k = 0; k < kApPrefetch && ahead.more(); ++k) ahead.next();
       RingPos<kApQ> rq;
       for (; iw.more(); iw.next(), rq.next(), ++it) {
         const int bh = iw.bh, b = iw.b, h = iw.h;
+        if (ahead.more()) {
+          if (lane == 0) {
+            tma_prefetch_3d(&tmQ, ahead.h * 128, ahead.ti * kTcTile, ahead.b);
+            tma_prefetch_3d(&tmQ, ahead.h * 128 + 64, ahead.ti * kTcTile, ahead.b);
+          }
+          ahead.next();
+        }
         if (iw.first) {
           // Every lane waits, so the warp leaves the loop together on a timeout.
           if (!mbar_wait(sfree, (uint32_t)((seg & 1) ^ 1), abort_flag)) break;
@@ -658,7 +734,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
         if (!mbar_wait(&qempty[s], rq.ph ^ 1u, abort_flag)) break;
         const int n0 = iw.ti * kTcTile;
         if (g.rope_on)
-          tile_rowpos<kTcTile>(g, win, n0, lane, reinterpret_cast<uint2*>(sm + TcApplySmem::ROWPOS + s * 1024));
+          tile_rowrec<kTcTile>(g, win, n0, lane, sm + TcApplySmem::ROWREC + s * kTcTile * kRecBytes);
         __syncwarp();
         if (lane != 0) { ++issued; continue; }
         mbar_arrive_expect_tx(&qfull[s], kTileBytes);
@@ -685,10 +761,17 @@ __global__ void __launch_bounds__(kApThreads, 1)
       long long it = 0;
       int issued = 0;
       ItemWalk iw(wb, we, tph, g.Hh);
+      ItemWalk ahead = iw;
+      for (int k = 0; k < kApPrefetch && ahead.more(); ++k) ahead.next();
       RingPos<kApG> rg_;
       for (; iw.more(); iw.next(), rg_.next(), ++it) {
         const int b = iw.b, h = iw.h;
         const int s = rg_.s;
+        if (ahead.more()) {
+          tma_prefetch_3d(&tmG, ahead.h * 128, ahead.ti * kTcTile, ahead.b);
+          tma_prefetch_3d(&tmG, ahead.h * 128 + 64, ahead.ti * kTcTile, ahead.b);
+          ahead.next();
+        }
         if (!mbar_wait(&gempty[s], rg_.ph ^ 1u, abort_flag)) break;
         const int n0 = iw.ti * kTcTile;
         mbar_arrive_expect_tx(&gfull[s], kTileBytes);
@@ -744,11 +827,13 @@ __global__ void __launch_bounds__(kApThreads, 1)
     }
   } else if (warp < kApEW0) {
     // ------------------------------------ transform warps: q -> q_til, den
+    // The RoPE table is built here, while the first tiles are in flight.
+    rope_build(tab, g, win, threadIdx.x - kApTW0 * 32, kApTW * 32);
+    named_barrier(1, kApTW * 32);
     const int tw = warp - kApTW0;
     const int rg = tw_row(lane), j = tw_chunk(lane);
     LaneRope lr;
-    lane_rope(g, j, lr);
-    const uint32_t tab_s = smem_u32(tab);
+    lane_rope(g, j, smem_u32(tab), lr);
     uint32_t ch0, ch1;
     lane_chunks(0, kBox, tw * 4 + rg, j, ch0, ch1);
     f2_t zr[8];
@@ -771,59 +856,73 @@ __global__ void __launch_bounds__(kApThreads, 1)
       const int n0 = iw.ti * kTcTile;
       const uint32_t qt = sbase + TcApplySmem::Q + s * kTileBytes;
       float* den = den_ring + rd.s * 128;
+      const uint32_t rec_s = sbase + TcApplySmem::ROWREC + s * kTcTile * kRecBytes;
 #pragma unroll 1
-      for (int ps = 0; ps < (kTcTile + kApRowsPerPass - 1) / kApRowsPerPass; ++ps) {
-        if (ps * kApRowsPerPass + tw * 4 >= kTcTile) break;
-        const int r = ps * kApRowsPerPass + tw * 4 + rg;
-        const int n = n0 + r;
-        const uint32_t a0 = qt + ch0 + ps * kApRowsPerPass * 128;
-        const uint32_t a1 = qt + ch1 + ps * kApRowsPerPass * 128;
-        uint32_t aA = 0;
-        int dB = 0;
-        if (g.rope_on)
-          lane_rope_row(lr, tab_s, reinterpret_cast<const uint2*>(sm + TcApplySmem::ROWPOS + s * 1024)[r], aA, dB);
-        f2_t x[8];
-        unpack8(lds128(a0), lds128(a1), x);
-        const float rstd = row_rstd(x);
-        f2_t dp2 = 0ull;
+      for (int ps = 0; ps < kApPasses; ++ps) {
+        // kApIL row groups (4 rows each, kApTW * 4 rows apart) at once: shared
+        // loads of every row first, then each row group's arithmetic and stores.
+        uint32_t a0[kApIL], a1[kApIL], t012[kApIL], t345[kApIL], t67[kApIL];
+        uint4 in0[kApIL], in1[kApIL];
+        f2_t e[kApIL][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          x[i] = f2_relu(x[i]);
-          dp2 = f2_fma(zr[i], x[i], dp2);
+        for (int u = 0; u < kApIL; ++u) {
+          const int r = ps * kApRowsPerPass + u * kApTW * 4 + tw * 4 + rg;
+          a0[u] = qt + ch0 + (ps * kApRowsPerPass + u * kApTW * 4) * 128;
+          a1[u] = qt + ch1 + (ps * kApRowsPerPass + u * kApTW * 4) * 128;
+          if (g.rope_on) lane_rope_row(lr, rec_s + r * kRecBytes, t012[u], t345[u], t67[u]);
         }
-        uint4 o0, o1;
-        rope_scale_pack<true>(g, lr, aA, dB, x, rstd, o0, o1);
-        sts128(a0, o0);
-        sts128(a1, o1);
-        float dp = f2_lo(dp2) + f2_hi(dp2);
-        dp = row_sum(dp);
-        const float dn = fmaf(dp, rstd, g.eps);      // z . q_pls + eps
+#pragma unroll
+        for (int u = 0; u < kApIL; ++u) {
+          in0[u] = lds128(a0[u]);
+          in1[u] = lds128(a1[u]);
+        }
+        if (g.rope_on) {
+#pragma unroll
+          for (int u = 0; u < kApIL; ++u) tab_load8(t012[u], t345[u], t67[u], e[u]);
+        }
+        float dn[kApIL];
+#pragma unroll
+        for (int u = 0; u < kApIL; ++u) {
+          f2_t x[8];
+          unpack8(in0[u], in1[u], x);
+          const float rstd = row_rstd(x);
+          f2_t dp2 = 0ull;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            x[i] = f2_relu(x[i]);
+            dp2 = f2_fma(zr[i], x[i], dp2);
+          }
+          uint4 o0, o1;
+          rope_scale_pack<true>(g.rope_on, e[u], x, rstd, o0, o1);
+          sts128(a0[u], o0);
+          sts128(a1[u], o1);
+          const float dp = row_sum(f2_lo(dp2) + f2_hi(dp2));
+          dn[u] = fmaf(dp, rstd, g.eps);               // z . q_pls + eps
+        }
         if (j == 0) {
-          // The read-out sees S * scale; fold the scale into the denominator.
-          den[r] = dn * hscale;
-          if (kDebug && p.den_out && n < g.N) p.den_out[((size_t)b * g.N + n) * g.Hh + h] = dn;
+#pragma unroll
+          for (int u = 0; u < kApIL; ++u) {
+            const int r = ps * kApRowsPerPass + u * kApTW * 4 + tw * 4 + rg;
+            // The read-out sees S * scale; fold the scale into the denominator.
+            den[r] = dn[u] * hscale;
+            const int n = n0 + r;
+            if (kDebug && p.den_out && n < g.N) p.den_out[((size_t)b * g.N + n) * g.Hh + h] = dn[u];
+          }
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&qready[s]);
     }
-  } else {
-    // ---------------------- epilogue warps: gate, denominator, RMSNorm, store
-    const int ew = warp - kApEW0;
-    const int grp = ew >> 2;            // this group takes every kApEWGroups-th tile
+  } else if (warp < kApST) {
+    // ------------------------- epilogue warps: gate, denominator, RMSNorm
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
-    const bool storer = (ew & 3) == 0 && lane == 0;
-    const uint64_t pol = policy_evict_first();
-    int prev_gsl = -1;                  // g slot whose store may still be reading
     ItemWalk iw(wb, we, tph, g.Hh);
     RingPos<kApAcc> ra;
     RingPos<kApG> rg_;
     RingPos<kApDen> rd;
-    RingPos<kApEWGroups> rsel;
-    for (; iw.more(); iw.next(), ra.next(), rg_.next(), rd.next(), rsel.next()) {
-      if (rsel.s != grp) continue;
+    for (; iw.more(); iw.next(), ra.next(), rg_.next(), rd.next()) {
       const int b = iw.b, h = iw.h;
       const int n0 = iw.ti * kTcTile;
       const int ab = ra.s;
@@ -891,24 +990,34 @@ __global__ void __launch_bounds__(kApThreads, 1)
         }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[ab]);
       fence_proxy_async_smem();
-      named_barrier(2 + grp, 128);
-      if (storer) {
-        tma_store_3d(&tmO, sm + TcApplySmem::G + gsl * kTileBytes, h * 128, n0, b, pol);
-        tma_store_3d(&tmO, sm + TcApplySmem::G + gsl * kTileBytes + kBox, h * 128 + 64, n0, b, pol);
-        bulk_commit();
-        // Release the previous tile's slot once its store has read it; this
-        // tile's store keeps running while the group starts the next tile.
-        bulk_wait_read_1();
-        if (prev_gsl >= 0) mbar_arrive(&gempty[prev_gsl]);
-        prev_gsl = gsl;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&accempty[ab]);
+        mbar_arrive(&ostaged[gsl]);
       }
     }
-    if (storer) {
+  } else if (warp == kApST) {
+    // ------------------------------------------------------------- store
+    // Once the four epilogue warps have staged a tile's output in its g slot,
+    // store it and hand the slot back to the g producer as soon as the store
+    // has read it.
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      ItemWalk iw(wb, we, tph, g.Hh);
+      RingPos<kApG> rg_;
+      for (; iw.more(); iw.next(), rg_.next()) {
+        const int gsl = rg_.s;
+        if (!mbar_wait(&ostaged[gsl], rg_.ph, abort_flag)) break;
+        const int n0 = iw.ti * kTcTile;
+        unsigned char* gt = sm + TcApplySmem::G + gsl * kTileBytes;
+        tma_store_3d(&tmO, gt, iw.h * 128, n0, iw.b, pol);
+        tma_store_3d(&tmO, gt + kBox, iw.h * 128 + 64, n0, iw.b, pol);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(&gempty[gsl]);
+      }
       bulk_wait_all();
-      if (prev_gsl >= 0) mbar_arrive(&gempty[prev_gsl]);
     }
   }
 
@@ -996,6 +1105,7 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   if (sms <= 0) return GLA_ERR_CUDA;
   if (g.H >= (1 << kPosBits) || g.W >= (1 << kPosBits) || g.T >= (1 << kPosBits))
     return GLA_ERR_UNSUPPORTED;
+  if (!tc_rope_lanes_ok(g)) return GLA_ERR_UNSUPPORTED;
   const Partition spart = tc_state_partition(g, sms);
   const Partition part = tc_apply_partition(g, sms);
   const int stab = tc_table_entries(g, spart), tab = tc_table_entries(g, part);

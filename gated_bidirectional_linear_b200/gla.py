@@ -40,6 +40,7 @@ _SIGS = {
     "gla_forward_host": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
     "gla_forward_noalloc": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp]),
     "gla_get_device_status": (_i, [_vp]),
+    "gla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "gla_plan": (_i, [_i] * 9 + [ctypes.POINTER(_i)] * 3),
 }
 
@@ -235,6 +236,14 @@ def gla_forward_noalloc(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6,
 def gla_get_device_status(stream=None):
     """Synchronise the stream and return (and clear) the device error status."""
     return lib().gla_get_device_status(_stream(stream))
+
+
+def gla_selftest_wait_timeout(limit_us, stream=None):
+    """Launch the failure-detection self-test: a bounded wait that nothing
+    satisfies gives up after `limit_us` microseconds and records a timeout
+    (read it with gla_get_device_status)."""
+    _check(lib().gla_selftest_wait_timeout(int(limit_us), _stream(stream)),
+           "gla_selftest_wait_timeout")
 
 
 def gla_plan(batch, heads, head_dim, T, H, W, dtype, path, num_sms):

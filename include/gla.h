@@ -219,6 +219,17 @@ GLA_API gla_status gla_forward_noalloc(const void* q, const void* k, const void*
  * call, GLA_ERR_CUDA if the synchronisation itself failed, else GLA_OK. */
 GLA_API gla_status gla_get_device_status(void* stream);
 
+/* Self-test of the failure-detection path.  Launches one CTA on `stream` whose
+ * threads wait on an mbarrier that nothing arrives on, through the same
+ * bounded wait every pipeline stage of the library uses, but with a limit of
+ * `limit_us` microseconds (1 .. 1000000) instead of the pipelines' 2 s.  The
+ * wait gives up, records the timeout in the device error word as a stalled
+ * pipeline would, and the kernel returns; nothing faults or hangs.  A later
+ * gla_get_device_status() reports GLA_ERR_TIMEOUT and clears it.  Returns
+ * GLA_ERR_INVALID_ARG for a limit outside that range (nothing launched),
+ * GLA_ERR_CUDA if the launch fails, else GLA_OK. */
+GLA_API gla_status gla_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
 /* Host-only planning query (no GPU needed): the grid of the state-reduction
  * kernel and the tokens per tile for this problem on a GPU with `num_sms`
  * SMs and the given path.  Returns GLA_OK and fills *grid, *tile_tokens,

@@ -116,3 +116,10 @@ def test_plan_paths():
     assert gla.gla_plan(1, 2, 128, 1, 1, 100, 1, 0, 148)[0] == 4
     with pytest.raises(gla.GlaError):
         gla.gla_plan(1, 2, 32, 2, 4, 4, 0, gla.GLA_PATH_TENSOR, 148)
+
+
+def test_selftest_rejects_out_of_range_limits():
+    # Rejected before anything is launched, so no GPU is needed.
+    lib = gla.lib()
+    assert lib.gla_selftest_wait_timeout(0, None) == gla.GLA_ERR_INVALID_ARG
+    assert lib.gla_selftest_wait_timeout(1000001, None) == gla.GLA_ERR_INVALID_ARG
