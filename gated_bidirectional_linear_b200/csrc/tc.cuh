@@ -700,17 +700,24 @@ __global__ void __launch_bounds__(kApThreads, 1)
     // ------------------------------------------------- producer: S image + q
     // All lanes compute the tile's row metadata; lane 0 issues the copies.
     // The S image, z and scale come from the combine kernel, which may still
-    // be running (programmatic dependent launch): wait for it first.
-    pdl_wait();
+    // be running (programmatic dependent launch): the first q tiles are
+    // requested before waiting for it.
     {
       const uint64_t pol = policy_evict_first();
-      long long it = 0;
       int seg = 0, issued = 0;
+      bool combined = false;
       ItemWalk iw(wb, we, tph, g.Hh);
       ItemWalk ahead = iw;      // the item kApPrefetch ahead of iw
-      for (int k = 0; k < kApPrefetch && ahead.more(); ++k) ahead.next();
+      ahead.next();
+      for (int k = 1; k < kApPrefetch && ahead.more(); ++k) {
+        if (lane == 0) {
+          tma_prefetch_3d(&tmQ, ahead.h * 128, ahead.ti * kTcTile, ahead.b);
+          tma_prefetch_3d(&tmQ, ahead.h * 128 + 64, ahead.ti * kTcTile, ahead.b);
+        }
+        ahead.next();
+      }
       RingPos<kApQ> rq;
-      for (; iw.more(); iw.next(), rq.next(), ++it) {
+      for (; iw.more(); iw.next(), rq.next()) {
         const int bh = iw.bh, b = iw.b, h = iw.h;
         if (ahead.more()) {
           if (lane == 0) {
@@ -719,7 +726,24 @@ __global__ void __launch_bounds__(kApThreads, 1)
           }
           ahead.next();
         }
+        const int s = rq.s;
+        if (!mbar_wait(&qempty[s], rq.ph ^ 1u, abort_flag)) break;
+        const int n0 = iw.ti * kTcTile;
+        if (g.rope_on)
+          tile_rowrec<kTcTile>(g, win, n0, lane, sm + TcApplySmem::ROWREC + s * kTcTile * kRecBytes);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&qfull[s], kTileBytes);
+          unsigned char* qt = sm + TcApplySmem::Q + s * kTileBytes;
+          tma_load_3d(qt, &tmQ, &qfull[s], h * 128, n0, b, pol);
+          tma_load_3d(qt + kBox, &tmQ, &qfull[s], h * 128 + 64, n0, b, pol);
+        }
+        ++issued;
         if (iw.first) {
+          if (!combined) {
+            pdl_wait();
+            combined = true;
+          }
           // Every lane waits, so the warp leaves the loop together on a timeout.
           if (!mbar_wait(sfree, (uint32_t)((seg & 1) ^ 1), abort_flag)) break;
           if (lane == 0) {
@@ -730,22 +754,10 @@ __global__ void __launch_bounds__(kApThreads, 1)
           }
           ++seg;
         }
-        const int s = rq.s;
-        if (!mbar_wait(&qempty[s], rq.ph ^ 1u, abort_flag)) break;
-        const int n0 = iw.ti * kTcTile;
-        if (g.rope_on)
-          tile_rowrec<kTcTile>(g, win, n0, lane, sm + TcApplySmem::ROWREC + s * kTcTile * kRecBytes);
-        __syncwarp();
-        if (lane != 0) { ++issued; continue; }
-        mbar_arrive_expect_tx(&qfull[s], kTileBytes);
-        unsigned char* qt = sm + TcApplySmem::Q + s * kTileBytes;
-        tma_load_3d(qt, &tmQ, &qfull[s], h * 128, n0, b, pol);
-        tma_load_3d(qt + kBox, &tmQ, &qfull[s], h * 128 + 64, n0, b, pol);
-        ++issued;
       }
       if (*abort_flag && lane == 0) {
-        long long first = it - (issued < kApQ ? issued : kApQ);
-        for (long long i2 = first; i2 < it; ++i2) {
+        // q loads went out for items 0 .. issued-1: let the last kApQ land.
+        for (int i2 = issued - (issued < kApQ ? issued : kApQ); i2 < issued; ++i2) {
           int dummy = 0;
           mbar_wait(&qfull[i2 % kApQ], (uint32_t)((i2 / kApQ) & 1),
                     reinterpret_cast<volatile int*>(&dummy));
