@@ -1,21 +1,22 @@
 // Tensor-core path (bf16 inputs, head dim 128) for sm_100a.
 //
-//   tc_state_kernel  persistent split-N state reduction.  TMA streams 128-token
-//                    tiles of k and v (128-byte swizzle) into a 3-stage ring;
+//   tc_state_kernel  persistent split-N state reduction.  TMA streams 96-token
+//                    tiles of k and v (128-byte swizzle) into a 4-stage ring;
 //                    transform warps apply RMSNorm, ReLU, 3D RoPE and beta to
 //                    the k tile in place (bf16) while summing z in registers;
 //                    one thread issues tcgen05.mma  S += V^T (beta K_til)  with
-//                    both operands MN-major, accumulating in TMEM; epilogue warps
-//                    drain each finished head segment to its partial slot.
+//                    both operands MN-major, accumulating in TMEM; the
+//                    transform warps drain each finished head segment to its
+//                    partial slot.
 //   combine_kernel   (combine.cuh) fixed-order sum of the partials, plus the
-//                    swizzled bf16 image of S.
+//                    swizzled fp16 image of S.
 //   tc_apply_kernel  persistent read-out.  TMA streams q and g tiles; transform
 //                    warps turn q into q_til (fp16, in place) and the
 //                    denominator z.q_pls + eps; one thread issues
 //                    tcgen05.mma  U = Q_til S^T  into a double-buffered TMEM
 //                    accumulator; epilogue warps (one token row per thread)
-//                    apply sigmoid(g) / den, the output RMSNorm, round to bf16
-//                    into the g tile and TMA-store it.
+//                    apply sigmoid(g) / den and the output RMSNorm, round to
+//                    bf16 into the g tile, and a store warp TMA-stores it.
 //
 // All waits are bounded (mbar_wait): on expiry the kernel records a timeout in
 // the device error word, stops issuing work, drains its copies and frees TMEM.
@@ -110,13 +111,6 @@ struct RingPos {
     if (++s == N) { s = 0; ph ^= 1u; }
   }
 };
-
-__device__ __forceinline__ bool seg_first(const Partition& p, long long w, long long wb) {
-  return w == wb || (w % p.tiles_per_head) == 0;
-}
-__device__ __forceinline__ bool seg_last(const Partition& p, long long w, long long we) {
-  return w == we - 1 || ((w + 1) % p.tiles_per_head) == 0;
-}
 
 // Per-tile row records.  For every row r of a tile (token n0 + r) the producer
 // warp stores the byte offsets, inside the RoPE table, of the token's time (T),
