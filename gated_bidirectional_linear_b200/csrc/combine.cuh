@@ -36,7 +36,8 @@ struct CombineParams {
   const float* part_z;   // [slots][zparts][d]
   const float* S_in;     // optional carried state (may alias S_out)
   const float* z_in;     // optional carried key sum (may alias z_out)
-  float* S_out;          // [BH][d][d]
+  float* S_out;          // optional [BH][d][d] (null: only the image is needed)
+  int chunked;           // partials in the tensor path's chunk-major layout (d = 128)
   float* z_out;          // [BH][d]
   __half* S_img;         // optional [BH][128*128] swizzled fp16 image (d = 128)
   float* S_scale;        // [BH][4]: [0] = scale of the image
@@ -49,6 +50,14 @@ __host__ __device__ inline uint32_t simg_offset(int a, int c) {
   const int byte_in_row = (c & 63) * 2;
   const int chunk = byte_in_row >> 4;
   return (uint32_t)(kb * 16384 + a * 128 + (((chunk ^ (a & 7)) << 4) | (byte_in_row & 15)));
+}
+
+// Row-major offset S[a][c] of partial element e.  The tensor path drains its
+// accumulator chunk-major (8 columns of all 128 rows after another, so that a
+// warp's stores are contiguous): e = (c/8 * 128 + a) * 8 + c%8.
+__device__ __forceinline__ int row_major(const CombineParams& p, int e) {
+  if (!p.chunked) return e;
+  return ((e >> 3) & 127) * 128 + ((e >> 10) << 3) + (e & 7);
 }
 
 __device__ __forceinline__ void add4(float4& s, const float4 t) {
@@ -89,7 +98,8 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
     const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
     live[k] = e < e_base + chunk;
     acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (live[k] && p.S_in) acc[k] = *reinterpret_cast<const float4*>(p.S_in + bh * dd + e);
+    if (live[k] && p.S_in)
+      acc[k] = *reinterpret_cast<const float4*>(p.S_in + bh * dd + row_major(p, e));
   }
   const bool zlive = (int)threadIdx.x < d;
   for (int c0 = c_lo; c0 <= c_hi; c0 += kBatch) {
@@ -126,7 +136,7 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
   for (int k = 0; k < 2; ++k) {
     if (!live[k]) continue;
     const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
-    *reinterpret_cast<float4*>(p.S_out + bh * dd + e) = acc[k];
+    if (p.S_out) *reinterpret_cast<float4*>(p.S_out + bh * dd + row_major(p, e)) = acc[k];
     m = fmaxf(m, fmaxf(fmaxf(fabsf(acc[k].x), fabsf(acc[k].y)),
                        fmaxf(fabsf(acc[k].z), fabsf(acc[k].w))));
   }
@@ -173,7 +183,8 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
   for (int k = 0; k < 2; ++k) {
     const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
     if (e >= e_base + chunk) continue;
-    const int a = e / d, cc = e % d;
+    const int rm = row_major(p, e);
+    const int a = rm / d, cc = rm % d;
     __half2 lo = __floats2half2_rn(acc[k].x * sc, acc[k].y * sc);
     __half2 hi = __floats2half2_rn(acc[k].z * sc, acc[k].w * sc);
     uint2 pk;   // cc .. cc+3 stay inside one 16-byte chunk (cc is a multiple of 4)

@@ -199,6 +199,7 @@ gla_status run_simt(const Call& c) {
   cp.z_in = c.carry ? c.z : nullptr;
   cp.S_out = c.S; cp.z_out = c.z;
   cp.S_img = nullptr; cp.S_scale = nullptr;
+  cp.chunked = 0;
   dim3 cgrid(kCombineCluster, g.B * g.Hh);
   combine_kernel<<<cgrid, kCombineThreads, 0, c.stream>>>(cp);
   if (cudaGetLastError() != cudaSuccess || mark(c, 2) != cudaSuccess) return GLA_ERR_CUDA;
@@ -229,7 +230,8 @@ gla_status run_simt_dtype(const Call& c) {
 gla_status run_call(Call& c) {
   gla_status st;
   if (c.path == GLA_PATH_TENSOR) {
-    st = run_tensor(c.g, c.q, c.k, c.v, c.beta, c.gate, c.out, c.S, c.z, c.carry,
+    const bool write_state = c.carry || c.S_dbg != nullptr;
+    st = run_tensor(c.g, c.q, c.k, c.v, c.beta, c.gate, c.out, c.S, c.z, c.carry, write_state,
                     reinterpret_cast<float*>(c.ws + c.L.part_S),
                     reinterpret_cast<float*>(c.ws + c.L.part_z),
                     reinterpret_cast<__half*>(c.ws + c.L.S_img),

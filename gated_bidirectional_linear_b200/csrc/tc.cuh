@@ -353,6 +353,10 @@ __global__ void __launch_bounds__(kStThreads, 1)
     // All lanes fetch beta and compute the tile's row metadata; lane 0 issues
     // the copies.
     {
+      // Launched as a programmatic dependent of whatever precedes it on the
+      // stream: the prologue above overlapped that kernel's tail, but the
+      // inputs may be its outputs, so wait for it before the first load.
+      pdl_wait();
       const uint64_t pol = policy_evict_first();
       const uint64_t pol_beta = policy_evict_last();
       long long it = 0;
@@ -554,14 +558,16 @@ __global__ void __launch_bounds__(kStThreads, 1)
           const int ab = seg & 1;
           if (!mbar_wait(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag)) { ok = false; break; }
           tc_fence_after();
-          float* dst = p.part_S + ((size_t)c + bh) * 128 * 128 + (size_t)a * 128;
+          // Chunk-major partial: columns 8cb .. 8cb+7 of row a at (cb * 128 + a) * 8,
+          // so the warp's 32 rows of a chunk are 1 KB of contiguous stores.
+          float* dst = p.part_S + ((size_t)c + bh) * 128 * 128 + (size_t)a * 8;
 #pragma unroll 1
           for (int cb = third; cb < 16; cb += 3) {
             float rr[8];
             tmem_ld8(tmem + (uint32_t)(ab * 128 + cb * 8) + ((uint32_t)(q4 * 32) << 16), rr);
             tmem_wait_ld();
-            *reinterpret_cast<float4*>(dst + cb * 8) = make_float4(rr[0], rr[1], rr[2], rr[3]);
-            *reinterpret_cast<float4*>(dst + cb * 8 + 4) = make_float4(rr[4], rr[5], rr[6], rr[7]);
+            *reinterpret_cast<float4*>(dst + cb * 1024) = make_float4(rr[0], rr[1], rr[2], rr[3]);
+            *reinterpret_cast<float4*>(dst + cb * 1024 + 4) = make_float4(rr[4], rr[5], rr[6], rr[7]);
           }
           tc_fence_before();
           __syncwarp();
@@ -684,6 +690,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
     tmem_alloc(tmem_holder, 256);
     tmem_relinquish();
   }
+  // The next kernel on the stream may start its prologue as our CTAs finish.
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1099,11 +1107,14 @@ inline int tc_table_entries(const Geom& g, const Partition& part) {
   return mx;
 }
 
+// The tensor path: state reduction, combine, read-out, each a programmatic
+// dependent of the kernel before it.  S / z: the fp32 state (block-causal: in
+// and out); z is always written, S only when write_state.
 inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const void* v,
                              const void* beta, const void* gate, void* out, float* S,
-                             float* z, bool carry, float* part_S, float* part_z,
-                             __half* S_img, float* S_scale, float* den_dbg, float* x_dbg,
-                             int sms, cudaStream_t stream, void* const* events) {
+                             float* z, bool carry, bool write_state, float* part_S,
+                             float* part_z, __half* S_img, float* S_scale, float* den_dbg,
+                             float* x_dbg, int sms, cudaStream_t stream, void* const* events) {
   auto mark = [&](int i) {
     if (!events || !events[i]) return cudaSuccess;
     return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream);
@@ -1132,18 +1143,27 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
                            (int)smem_st) != cudaSuccess)
     return GLA_ERR_CUDA;
   if (mark(0) != cudaSuccess) return GLA_ERR_CUDA;
-  tc_state_kernel<<<spart.grid, kStThreads, smem_st, stream>>>(mK, mV, sp);
-  if (cudaGetLastError() != cudaSuccess || mark(1) != cudaSuccess) return GLA_ERR_CUDA;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t sc = {};
+  sc.gridDim = dim3(spart.grid);
+  sc.blockDim = dim3(kStThreads);
+  sc.dynamicSmemBytes = smem_st;
+  sc.stream = stream;
+  sc.attrs = pdl;
+  sc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&sc, tc_state_kernel, mK, mV, sp) != cudaSuccess || mark(1) != cudaSuccess)
+    return GLA_ERR_CUDA;
 
   CombineParams cp;
   cp.part = spart; cp.d = 128; cp.zparts = kStTW;
   cp.part_S = part_S; cp.part_z = part_z;
   cp.S_in = carry ? S : nullptr;
   cp.z_in = carry ? z : nullptr;
-  cp.S_out = S; cp.z_out = z; cp.S_img = S_img; cp.S_scale = S_scale;
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cp.S_out = write_state ? S : nullptr;
+  cp.z_out = z; cp.S_img = S_img; cp.S_scale = S_scale;
+  cp.chunked = 1;
   cudaLaunchConfig_t cc = {};
   cc.gridDim = dim3(kCombineCluster, g.B * g.Hh);
   cc.blockDim = dim3(kCombineThreads);
