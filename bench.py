@@ -148,9 +148,14 @@ class ClockMonitor:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def cpu_oracle_rate(wl, seconds):
+def cpu_oracle_rate(wl, seconds, threads=None):
     """The oracle, as it stands, on whole heads of the workload until
-    `seconds` have passed: returns (tokens/s of the full layer, heads, s)."""
+    `seconds` have passed: returns (tokens/s of the full layer, heads, s,
+    threads).  threads=None: the BLAS threads as configured; else that many."""
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=threads, user_api="blas"):
+            return cpu_oracle_rate(wl, seconds)
     import oracle.gla_oracle as O
     from threadpoolctl import threadpool_info
     t_used, th = 0.0, 0
@@ -298,7 +303,8 @@ def main():
     k_state = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     k_comb = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     k_apply = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
-    k_step_events = float(np.mean([e[0].elapsed_time(e[3]) for e in evs]))
+    step_ev = np.array([e[0].elapsed_time(e[3]) for e in evs])
+    k_step_events = float(np.mean(step_ev))
 
     # ---- end to end: host buffers through gla_forward_host, copies timed.
     pinned = {k: v.pin_memory() for k, v in inp.items()}
@@ -346,10 +352,13 @@ def main():
         cpu = None
         if not args.no_cpu_baseline and world == 1:
             rate, heads, secs, cores = cpu_oracle_rate(wl, args.cpu_sample_seconds)
+            rate1, heads1, secs1, _ = cpu_oracle_rate(wl, args.cpu_sample_seconds / 3, threads=1)
             cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                    "sample": (f"oracle.forward on {heads} whole heads ({wl.tokens} tokens each) "
                               f"of the {wl.name} workload, {secs:.1f} s; tokens/s of the full "
-                              f"layer = token-heads/s / {wl.heads}; cores = BLAS threads")}
+                              f"layer = token-heads/s / {wl.heads}; cores = BLAS threads"),
+                   "single_core": {"value": rate1, "unit": "tokens/s", "cores": 1,
+                                   "sample": f"{heads1} whole heads, {secs1:.1f} s, one BLAS thread"}}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -366,7 +375,12 @@ def main():
                            "tc_apply_kernel": k_apply, "step_with_events": k_step_events,
                            "how": "second timed pass of the same K steps, events around each kernel"},
             "kernels_gbs": {"tc_state_kernel": state_gbs, "tc_apply_kernel": apply_gbs},
+            "step_ms_events": {"p10": float(np.percentile(step_ev, 10)),
+                               "p50": float(np.percentile(step_ev, 50)),
+                               "p90": float(np.percentile(step_ev, 90)),
+                               "how": "per step of the events pass (events between kernels)"},
             "step_frac_of_peak": step_gbs / peak,
+            "step_frac_of_nominal_8tbs": step_gbs / 8000.0,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": th * hd * esz * 4 + th * esz,
                     "d2h_bytes_per_step": th * hd * esz, "steps": e2e_steps},
