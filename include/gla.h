@@ -42,15 +42,22 @@
  * head_dim 128 runs on the tcgen05 tensor-core path (TMA-fed state reduction
  * and read-out); every other case, or path GLA_PATH_SIMT, runs on CUDA cores
  * with fp32 arithmetic.  Accumulation is always fp32.  On the tensor path the
- * MMA operands beta*k_til, q_til and S are rounded to bf16; outputs are
- * rounded to nearest even.
+ * state MMA's operand beta*k_til is rounded to bf16 (v arrives in bf16), and
+ * the read-out MMA's operands q_til and S to fp16 (q_til is bounded by
+ * sqrt(d) after the RMSNorm; S carries one power-of-two scale per head that
+ * puts its largest entry in [2^13, 2^14)); outputs are rounded to nearest
+ * even.
  *
  * Errors: every entry point validates its arguments first and returns an
  * error code with nothing launched.  A CUDA launch failure returns
  * GLA_ERR_CUDA.  Calls are asynchronous on `stream` (a cudaStream_t passed as
- * void*; NULL = legacy default stream).  Device-side wait timeouts (the
- * tensor path's bounded mbarrier waits) are recorded in a library-owned
- * device word and reported by gla_get_device_status().
+ * void*; NULL = legacy default stream) and stream-ordered.  On the tensor
+ * path the kernels of a call chain by programmatic dependent launch: the
+ * first may start its set-up while the preceding kernel on the stream is
+ * finishing, but reads no input before that kernel has completed.
+ * Device-side wait timeouts (the tensor path's bounded mbarrier waits) are
+ * recorded in a library-owned device word and reported by
+ * gla_get_device_status().
  *
  * Determinism: the state is reduced in a fixed split order, so the same
  * inputs on the same GPU model give bitwise-identical results.
