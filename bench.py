@@ -230,6 +230,9 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+    if wl.n_blocks > 1:
+        run_block_causal(args, wl, gla, dev, dist, world, rank, local)
+        return
 
     inp = workloads.make_inputs(wl, seed=wl.seed + rank)
     d = {k: v.to(dev) for k, v in inp.items()}
@@ -385,6 +388,130 @@ def main():
                     "h2d_bytes_per_step": th * hd * esz * 4 + th * esz,
                     "d2h_bytes_per_step": th * hd * esz, "steps": e2e_steps},
             "gpu_launches": 3 * args.steps,
+            "clocks": mon.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
+    """One step = a whole sequence of wl.n_blocks blocks through
+    gla_block_causal_step, from a zero state (a new sequence).  Not the
+    headline metric: the block-causal row's own measurement."""
+    inp = workloads.make_inputs(wl, seed=wl.seed + rank)
+    L = wl.tokens
+    blocks = [{k: v[:, i * L:(i + 1) * L].contiguous().to(dev) for k, v in inp.items()}
+              for i in range(wl.n_blocks)]
+    B, _, Hh, hd = blocks[0]["q"].shape
+    code = gla.GLA_DTYPE_BF16
+    S = torch.zeros(B, Hh, hd, hd, dtype=torch.float32, device=dev)
+    z = torch.zeros(B, Hh, hd, dtype=torch.float32, device=dev)
+    outs = [torch.empty_like(b["q"]) for b in blocks]
+    ws = gla.alloc_workspace(gla.gla_block_causal_workspace_size(B, Hh, hd, wl.T, wl.H, wl.W, code), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def sequence():
+        S.zero_()
+        z.zero_()
+        for i, b in enumerate(blocks):
+            gla.gla_block_causal_step(S, z, b["q"], b["k"], b["v"], b["beta"], b["g"], wl.T, wl.H,
+                                      wl.W, i * wl.T, wl.rope_theta, wl.eps, out=outs[i],
+                                      workspace=ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        sequence()
+    torch.cuda.synchronize(dev)
+    assert gla.gla_get_device_status(stream) == gla.GLA_OK
+    steps = max(1, args.steps // wl.n_blocks)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockMonitor(local) as mon:
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for _ in range(steps):
+            sequence()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist:
+            dist.barrier()
+    if gla.gla_get_device_status(stream) != gla.GLA_OK:
+        raise RuntimeError("device status after the timed region")
+    ms = t0.elapsed_time(t1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # End to end: the sequence's inputs from pinned host memory, the steps,
+    # and the outputs back, every step.
+    pinned = [{k: v.cpu().pin_memory() for k, v in b.items()} for b in blocks]
+    outs_h = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+
+    def sequence_host():
+        for b, bp in zip(blocks, pinned):
+            for k in b:
+                b[k].copy_(bp[k], non_blocking=True)
+        sequence()
+        for o, oh in zip(outs, outs_h):
+            oh.copy_(o, non_blocking=True)
+
+    e2e_steps = max(3, min(steps, 50))
+    sequence_host()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        sequence_host()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    tokens = B * wl.total_tokens
+    th = tokens * Hh
+    alg = wl.alg_bytes_per_call() * wl.n_blocks
+    state_io = 2 * (B * Hh * hd * hd * 4 + B * Hh * hd * 4) * wl.n_blocks
+    ms_step = ms / steps
+    peak, peak_kind = measured_peaks()
+    gbs = alg / (ms_step * 1e-3) / 1e9
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            import oracle.gla_oracle as O
+            x = workloads.as_f64(workloads.draw(1, wl.total_tokens, 1, hd, wl.dtype, 2000))
+            c0 = time.perf_counter()
+            O.block_causal_forward(x["q"], x["k"], x["v"], x["beta"], x["g"], wl.n_blocks,
+                                   wl.T, wl.H, wl.W, wl.rope_theta, wl.eps)
+            secs = time.perf_counter() - c0
+            cpu = {"value": wl.total_tokens / secs / wl.heads, "unit": "tokens/s", "cores": 1,
+                   "kind": "oracle",
+                   "sample": (f"oracle.block_causal_forward on one head of the {wl.name} "
+                              f"sequence ({wl.n_blocks} blocks), {secs:.1f} s; tokens/s of the "
+                              f"full layer = token-heads/s / {wl.heads}")}
+        line = {
+            "metric": "gla_block_causal_step tokens/s (20x128 heads, 20 blocks of 3x23x40)",
+            "value": world * tokens * steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(workload_config(wl), blocks=wl.n_blocks,
+                           step=f"{wl.n_blocks} gla_block_causal_step calls from a zero state",
+                           parallelism=f"replicas x{world}"),
+            "roofline": {"bound": "hbm", "kernel": "whole step", "achieved": gbs, "peak": peak,
+                         "unit": "GB/s", "frac": gbs / peak, "peak_kind": peak_kind,
+                         "traffic": None, "alg_bytes_per_step": alg,
+                         "state_bytes_per_step": state_io},
+            "e2e": {"value": world * tokens * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": th * hd * 2 * 4 + th * 2,
+                    "d2h_bytes_per_step": th * hd * 2, "steps": e2e_steps},
+            "gpu_launches": 3 * wl.n_blocks * steps,
             "clocks": mon.summary(),
             "cpu_baseline": cpu,
         }
