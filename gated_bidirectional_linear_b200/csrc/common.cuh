@@ -48,6 +48,7 @@ struct Geom {
   float theta;           // RoPE base
   float eps;             // denominator epsilon
   FastDiv div_HW, div_W; // n -> frame, n % HW -> row
+  double freq[64];       // theta^(-i/np) of global rotation pair i .. (pair i of its axis)
 };
 
 __host__ __device__ inline void rope_split(int d, int* pt, int* ph, int* pw) {
@@ -179,24 +180,31 @@ __host__ __device__ inline int rope_table_entries(const Geom& g, int Lt) {
   return rope_layout(g, Lt).entries;
 }
 
+// (cos, sin) of position x at frequency freq: the angle is formed and reduced
+// to [-pi, pi] in double, then evaluated in fp32.
+__device__ __forceinline__ float2 rope_entry(double x, double freq) {
+  const double two_pi = 6.283185307179586476925286766559;
+  double ang = x * freq;
+  ang -= two_pi * rint(ang * (1.0 / two_pi));
+  float sn, cs;
+  sincosf((float)ang, &sn, &cs);
+  return make_float2(cs, sn);
+}
+
 __device__ inline void rope_build(float2* tab, const Geom& g, RopeWindow win, int tid,
                                   int nthr) {
   if (!g.rope_on) return;
   // Thread tid handles rotation pair (tid mod P) of its axis at every
-  // (nthr / P)-th position: one exp per thread, then per entry the angle
-  // pos * freq in double, reduced to [-pi, pi] in double, and fp32 sincosf.
+  // (nthr / P)-th position: one rope_entry per row.
   const RopeLayout L = rope_layout(g, win.Lt);
   const int P = g.pt + g.ph + g.pw;
   const int pr = tid % P;
   const int lane0 = tid / P, step = nthr / P;
   if (lane0 >= step) return;
   const int axis = pr < g.pt ? 0 : (pr < g.pt + g.ph ? 1 : 2);
-  const int np = axis == 0 ? g.pt : (axis == 1 ? g.ph : g.pw);
-  const int i = pr - L.start[axis];
   const int rows = axis == 0 ? win.Lt : (axis == 1 ? g.H : g.W);
   const int col = rope_idx(L, axis, pr);
-  const double freq = exp(-((double)i / (double)np) * log((double)g.theta));
-  const double two_pi = 6.283185307179586476925286766559;
+  const double freq = g.freq[pr];
   for (int pos = lane0; pos < rows; pos += step) {
     double x;
     if (axis == 0) {
@@ -206,12 +214,62 @@ __device__ inline void rope_build(float2* tab, const Geom& g, RopeWindow win, in
     } else {
       x = (double)pos;
     }
-    double ang = x * freq;
-    ang -= two_pi * rint(ang * (1.0 / two_pi));
-    float sn, cs;
-    sincosf((float)ang, &sn, &cs);
-    tab[L.base[axis] + pos * L.stride[axis] + col] = make_float2(cs, sn);
+    tab[L.base[axis] + pos * L.stride[axis] + col] = rope_entry(x, freq);
   }
+}
+
+// The whole call's table (all T frames: rope_layout(g, g.T), frame f at time
+// row f) written to global memory, one table row (an axis position) per
+// (row, pair) task; CTA `cta` of `ncta` takes rows cta, cta + ncta, ...
+// Entries are the same rope_entry values rope_build produces.
+__device__ inline void rope_build_global(float2* gtab, const Geom& g, int cta, int ncta,
+                                         int tid, int nthr) {
+  if (!g.rope_on) return;
+  const RopeLayout L = rope_layout(g, g.T);
+  const int rows_total = g.T + g.H + g.W;
+  const int np_max = g.pt > g.ph ? (g.pt > g.pw ? g.pt : g.pw) : (g.ph > g.pw ? g.ph : g.pw);
+  const int per = nthr / np_max;   // rows a CTA fills at once
+  if (per == 0) return;
+  const int i = tid % np_max, sub = tid / np_max;
+  if (sub >= per) return;
+  for (int r = cta + ncta * sub; r < rows_total; r += ncta * per) {
+    const int axis = r < g.T ? 0 : (r < g.T + g.H ? 1 : 2);
+    const int pos = axis == 0 ? r : (axis == 1 ? r - g.T : r - g.T - g.H);
+    const int np = axis == 0 ? g.pt : (axis == 1 ? g.ph : g.pw);
+    if (i >= np) continue;
+    const double x = axis == 0 ? (double)(g.t0 + pos) : (double)pos;
+    const int pr = L.start[axis] + i;
+    gtab[L.base[axis] + pos * L.stride[axis] + rope_idx(L, axis, pr)] = rope_entry(x, g.freq[pr]);
+  }
+}
+
+// The copies that turn the whole-call table (rope_layout(g, g.T) in global
+// memory) into a CTA's windowed table (rope_layout(g, win.Lt) in shared
+// memory): time rows t_lo .. T-1 and, for a window that wraps, 0 .. the rest;
+// then the height and width blocks whole.  Offsets and sizes in entries; every
+// one is a multiple of 8 entries (64 bytes), as bulk copies require.
+struct RopeCopy {
+  int n;
+  int src[4], dst[4], len[4];
+};
+
+__host__ __device__ inline RopeCopy rope_copy_plan(const Geom& g, RopeWindow win) {
+  const RopeLayout G = rope_layout(g, g.T), W = rope_layout(g, win.Lt);
+  RopeCopy c;
+  c.n = 0;
+  int rows1 = g.T - win.t_lo;
+  if (rows1 > win.Lt) rows1 = win.Lt;
+  c.src[c.n] = G.base[0] + win.t_lo * G.stride[0];
+  c.dst[c.n] = W.base[0];
+  c.len[c.n++] = rows1 * G.stride[0];
+  if (win.Lt > rows1) {
+    c.src[c.n] = G.base[0];
+    c.dst[c.n] = W.base[0] + rows1 * W.stride[0];
+    c.len[c.n++] = (win.Lt - rows1) * G.stride[0];
+  }
+  c.src[c.n] = G.base[1]; c.dst[c.n] = W.base[1]; c.len[c.n++] = g.H * G.stride[1];
+  c.src[c.n] = G.base[2]; c.dst[c.n] = W.base[2]; c.len[c.n++] = g.W * G.stride[2];
+  return c;
 }
 
 // Index of the (cos, sin) entry of rotation pair `pr` (0 .. d/2-1) for a token

@@ -45,12 +45,22 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 struct WsLayout {
-  size_t part_S, part_z, S, z, S_img, S_scale, total;
+  size_t part_S, part_z, S, z, S_img, S_scale, rope_tab, total;
   int slots;
 };
 
+// Bytes of the whole-call RoPE table the tensor path's combine writes for the
+// read-out (every frame of the call; at least one 16-byte unit).
+size_t rope_tab_bytes(int d, int T, int H, int W) {
+  Geom g = {};
+  g.d = d; g.T = T; g.H = H; g.W = W;
+  rope_split(d, &g.pt, &g.ph, &g.pw);
+  const size_t e = (size_t)rope_layout(g, T).entries;
+  return (e > 2 ? e : 2) * sizeof(float2);
+}
+
 // Workspace carve-up; independent of the GPU (uses the maximum grid).
-WsLayout ws_layout(int BH, int d, bool own_state) {
+WsLayout ws_layout(int BH, int d, bool own_state, int T, int H, int W) {
   WsLayout L;
   L.slots = kMaxStateCtas + BH;
   size_t off = 0;
@@ -66,6 +76,8 @@ WsLayout ws_layout(int BH, int d, bool own_state) {
   if (d == 128) off = align_up(off + (size_t)BH * d * d * 2, kAlign);
   L.S_scale = off;
   if (d == 128) off = align_up(off + (size_t)BH * 4 * 4, kAlign);
+  L.rope_tab = off;
+  if (d == 128) off = align_up(off + rope_tab_bytes(d, T, H, W), kAlign);
   L.total = off;
   return L;
 }
@@ -103,6 +115,16 @@ Geom make_geom(int batch, int heads, int head_dim, int T, int H, int W, int t0,
   g.eps = eps;
   g.div_HW = make_fastdiv((uint32_t)(H * W));
   g.div_W = make_fastdiv((uint32_t)W);
+  // Rotation frequencies, once per call in double: pair i of an axis with np
+  // pairs turns at theta^(-i/np) radians per position.
+  const int np[3] = {g.pt, g.ph, g.pw};
+  for (int pr = 0, a = 0, i = 0; pr < 64; ++pr) {
+    g.freq[pr] = 0.0;
+    if (pr >= g.pt + g.ph + g.pw || !g.rope_on) continue;
+    while (i >= np[a]) { i -= np[a]; ++a; }
+    g.freq[pr] = exp(-((double)i / (double)np[a]) * log((double)rope_theta));
+    ++i;
+  }
   return g;
 }
 
@@ -192,7 +214,7 @@ gla_status run_simt(const Call& c) {
   simt_state_kernel<D, Tin><<<part.grid, kSimtThreads, smem_state, c.stream>>>(sp);
   if (cudaGetLastError() != cudaSuccess || mark(c, 1) != cudaSuccess) return GLA_ERR_CUDA;
 
-  CombineParams cp;
+  CombineParams cp = {};
   cp.part = part; cp.d = D; cp.zparts = 1;
   cp.part_S = sp.part_S; cp.part_z = sp.part_z;
   cp.S_in = c.carry ? c.S : nullptr;
@@ -235,7 +257,8 @@ gla_status run_call(Call& c) {
                     reinterpret_cast<float*>(c.ws + c.L.part_S),
                     reinterpret_cast<float*>(c.ws + c.L.part_z),
                     reinterpret_cast<__half*>(c.ws + c.L.S_img),
-                    reinterpret_cast<float*>(c.ws + c.L.S_scale), c.den_dbg, c.x_dbg,
+                    reinterpret_cast<float*>(c.ws + c.L.S_scale),
+                    reinterpret_cast<float2*>(c.ws + c.L.rope_tab), c.den_dbg, c.x_dbg,
                     device_sm_count(), c.stream, c.events);
   } else {
     st = c.dtype == GLA_DTYPE_F32 ? run_simt_dtype<float>(c)
@@ -264,7 +287,7 @@ gla_status forward_common(const void* q, const void* k, const void* v, const voi
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
   if (resolve_path(path, dtype, head_dim) < 0) return GLA_ERR_UNSUPPORTED;
-  const WsLayout L = ws_layout(batch * heads, head_dim, true);
+  const WsLayout L = ws_layout(batch * heads, head_dim, true, T, H, W);
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < L.total)
     return GLA_ERR_WORKSPACE;
   Call c;
@@ -306,14 +329,14 @@ size_t gla_forward_workspace_size(int batch, int heads, int head_dim, int T, int
                                   int dtype) {
   if (!dims_ok(batch, heads, head_dim, T, H, W)) return 0;
   if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return 0;
-  return ws_layout(batch * heads, head_dim, true).total;
+  return ws_layout(batch * heads, head_dim, true, T, H, W).total;
 }
 
 size_t gla_block_causal_workspace_size(int batch, int heads, int head_dim, int T_blk, int H,
                                        int W, int dtype) {
   if (!dims_ok(batch, heads, head_dim, T_blk, H, W)) return 0;
   if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return 0;
-  return ws_layout(batch * heads, head_dim, false).total;
+  return ws_layout(batch * heads, head_dim, false, T_blk, H, W).total;
 }
 
 gla_status gla_forward(const void* q, const void* k, const void* v, const void* beta,
@@ -367,7 +390,7 @@ gla_status gla_block_causal_step_ex(float* state, float* z, const void* q, const
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
   if (resolve_path(path, dtype, head_dim) < 0) return GLA_ERR_UNSUPPORTED;
-  const WsLayout L = ws_layout(batch * heads, head_dim, false);
+  const WsLayout L = ws_layout(batch * heads, head_dim, false, T_blk, H, W);
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < L.total)
     return GLA_ERR_WORKSPACE;
   Call c;
@@ -467,7 +490,7 @@ unsigned char* noalloc_scratch() {
 
 // Scratch layout sized for the grid this GPU actually runs (at most `grid`
 // state CTAs, `zparts` z partials per slot) rather than the worst case.
-WsLayout noalloc_layout(int BH, int d, int grid, int zparts) {
+WsLayout noalloc_layout(int BH, int d, int grid, int zparts, int T, int H, int W) {
   WsLayout L;
   L.slots = grid + BH;
   size_t off = 0;
@@ -479,6 +502,8 @@ WsLayout noalloc_layout(int BH, int d, int grid, int zparts) {
   if (d == 128) off = align_up(off + (size_t)BH * d * d * 2, kAlign);
   L.S_scale = off;
   if (d == 128) off = align_up(off + (size_t)BH * 4 * 4, kAlign);
+  L.rope_tab = off;
+  if (d == 128) off = align_up(off + rope_tab_bytes(d, T, H, W), kAlign);
   L.total = off;
   return L;
 }
@@ -506,7 +531,7 @@ gla_status gla_forward_noalloc(const void* q, const void* k, const void* v, cons
   const bool tensor = c.path == GLA_PATH_TENSOR;
   const Partition part = tensor ? tc_state_partition(c.g, sms)
                                 : make_partition(batch * heads, c.g.N, kSimtTile, 2 * sms);
-  const WsLayout L = noalloc_layout(batch * heads, head_dim, part.grid, tensor ? kStTW : 1);
+  const WsLayout L = noalloc_layout(batch * heads, head_dim, part.grid, tensor ? kStTW : 1, T, H, W);
   if (L.total > GLA_NOALLOC_SCRATCH_BYTES) return GLA_ERR_WORKSPACE;
   unsigned char* scratch = noalloc_scratch();
   if (!scratch) return GLA_ERR_CUDA;

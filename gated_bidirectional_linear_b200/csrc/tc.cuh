@@ -69,6 +69,7 @@ struct TcStateParams {
   const __nv_bfloat16* beta;
   float* part_S;
   float* part_z;
+  float2* rope_tab;   // optional: the call's whole RoPE table for the read-out
   int tab_entries;
 };
 
@@ -407,6 +408,11 @@ __global__ void __launch_bounds__(kStThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[s]);
         ++issued;
+        // While the first tiles land: this CTA's rows of the whole-call RoPE
+        // table the read-out copies.  Written after the wait above, so the
+        // previous call's read-out, which read the same buffer, has finished.
+        if (it == 0 && p.rope_tab != nullptr)
+          rope_build_global(p.rope_tab, g, blockIdx.x, gridDim.x, lane, 32);
       }
       if (*abort_flag && lane == 0) {
         // Let every load in flight land before shared memory is released.
@@ -614,7 +620,7 @@ struct TcApplySmem {
   static constexpr uint32_t DEN = SCL + 16;                 // [kApDen][128] den*scale per tile
   static constexpr uint32_t ROWREC = DEN + kApDen * 512;    // [q slot][128] records
   static constexpr uint32_t BAR = ROWREC + kApQ * kTcTile * kRecBytes;
-  static constexpr uint32_t NBAR = 3 * kApQ + 3 * kApG + 2 * kApAcc + 3;
+  static constexpr uint32_t NBAR = 3 * kApQ + 3 * kApG + 2 * kApAcc + 5;
   static constexpr uint32_t MISC = BAR + NBAR * 8;
   static constexpr uint32_t TAB = (MISC + 16 + 15) & ~15u;
 };
@@ -625,6 +631,7 @@ struct TcApplyParams {
   const __half* S_img;         // [BH][128*128] swizzled fp16 image of S * scale
   const float* S_scale;        // [BH][4]: [0] = scale of the image
   const float* z;              // [BH][128]
+  const float2* rope_tab;      // the call's whole RoPE table (rope_layout(g, g.T))
   float* den_out;              // optional
   float* x_out;                // optional
   int tab_entries;
@@ -650,6 +657,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
   uint64_t* sfull = accempty + kApAcc;
   uint64_t* sfree = sfull + 1;
   uint64_t* drain = sfree + 1;
+  uint64_t* zfull = drain + 1;    // z and the image scale of a segment's head
+  uint64_t* tfull = zfull + 1;    // the RoPE table (once)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + TcApplySmem::MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + TcApplySmem::MISC + 4);
   float* zs = reinterpret_cast<float*>(sm + TcApplySmem::Z);
@@ -683,6 +692,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
     mbar_init(sfull, 1);
     mbar_init(sfree, 1);
     mbar_init(drain, 1);
+    mbar_init(zfull, 1);
+    mbar_init(tfull, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -749,10 +760,29 @@ __global__ void __launch_bounds__(kApThreads, 1)
           // Every lane waits, so the warp leaves the loop together on a timeout.
           if (!mbar_wait(sfree, (uint32_t)((seg & 1) ^ 1), abort_flag)) break;
           if (lane == 0) {
-            mbar_arrive_expect_tx(sfull, kTileBytes + 512 + 16);
+            // Smallest first: z and the scale (the transform warps' only
+            // dependence on the combine), the RoPE table, then the S image.
+            mbar_arrive_expect_tx(zfull, 512 + 16);
+            bulk_load(sm + TcApplySmem::Z, p.z + (size_t)bh * 128, 512, zfull);
+            bulk_load(sm + TcApplySmem::SCL, p.S_scale + (size_t)bh * 4, 16, zfull);
+            if (seg == 0) {
+              if (g.rope_on) {
+                const RopeCopy rc = rope_copy_plan(g, win);
+                uint32_t bytes = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  if (i < rc.n) bytes += (uint32_t)rc.len[i] * 8u;
+                mbar_arrive_expect_tx(tfull, bytes);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  if (i < rc.n)
+                    bulk_load(tab + rc.dst[i], p.rope_tab + rc.src[i], (uint32_t)rc.len[i] * 8u, tfull);
+              } else {
+                mbar_arrive(tfull);
+              }
+            }
+            mbar_arrive_expect_tx(sfull, kTileBytes);
             bulk_load(sm + TcApplySmem::SIMG, p.S_img + (size_t)bh * 128 * 128, kTileBytes, sfull);
-            bulk_load(sm + TcApplySmem::Z, p.z + (size_t)bh * 128, 512, sfull);
-            bulk_load(sm + TcApplySmem::SCL, p.S_scale + (size_t)bh * 4, 16, sfull);
           }
           ++seg;
         }
@@ -765,7 +795,12 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     reinterpret_cast<volatile int*>(&dummy));
         }
         int dummy = 0;
-        if (seg > 0) mbar_wait(sfull, (uint32_t)((seg - 1) & 1), reinterpret_cast<volatile int*>(&dummy));
+        if (seg > 0) {
+          volatile int* nd = reinterpret_cast<volatile int*>(&dummy);
+          mbar_wait(sfull, (uint32_t)((seg - 1) & 1), nd);
+          mbar_wait(zfull, (uint32_t)((seg - 1) & 1), nd);
+          mbar_wait(tfull, 0u, nd);
+        }
       }
     }
   } else if (warp == 2) {
@@ -778,7 +813,11 @@ __global__ void __launch_bounds__(kApThreads, 1)
       ItemWalk ahead = iw;
       for (int k = 0; k < kApPrefetch && ahead.more(); ++k) ahead.next();
       RingPos<kApG> rg_;
-      for (; iw.more(); iw.next(), rg_.next(), ++it) {
+      // The first g tiles are needed only after the first read-out MMA: let
+      // the q tiles, z, the table and the S image go first.  tfull completes
+      // once, after the q producer has issued all of them.
+      const bool go = !iw.more() || mbar_wait(tfull, 0u, abort_flag);
+      for (; go && iw.more(); iw.next(), rg_.next(), ++it) {
         const int b = iw.b, h = iw.h;
         const int s = rg_.s;
         if (ahead.more()) {
@@ -841,9 +880,9 @@ __global__ void __launch_bounds__(kApThreads, 1)
     }
   } else if (warp < kApEW0) {
     // ------------------------------------ transform warps: q -> q_til, den
-    // The RoPE table is built here, while the first tiles are in flight.
-    rope_build(tab, g, win, threadIdx.x - kApTW0 * 32, kApTW * 32);
-    named_barrier(1, kApTW * 32);
+    // The RoPE table comes by bulk copy from the whole-call table the combine
+    // kernel writes.
+    const bool tab_ok = wb >= we || mbar_wait(tfull, 0u, abort_flag);
     const int tw = warp - kApTW0;
     const int rg = tw_row(lane), j = tw_chunk(lane);
     LaneRope lr;
@@ -856,10 +895,10 @@ __global__ void __launch_bounds__(kApThreads, 1)
     ItemWalk iw(wb, we, tph, g.Hh);
     RingPos<kApQ> rq;
     RingPos<kApDen> rd;
-    for (; iw.more(); iw.next(), rq.next(), rd.next()) {
+    for (; tab_ok && iw.more(); iw.next(), rq.next(), rd.next()) {
       const int b = iw.b, h = iw.h;
       if (iw.first) {
-        if (!mbar_wait(sfull, (uint32_t)(seg & 1), abort_flag)) break;
+        if (!mbar_wait(zfull, (uint32_t)(seg & 1), abort_flag)) break;
 #pragma unroll
         for (int i = 0; i < 8; ++i) zr[i] = f2(zs[16 * j + 2 * i], zs[16 * j + 2 * i + 1]);
         hscale = scl_s[0];
@@ -1113,8 +1152,9 @@ inline int tc_table_entries(const Geom& g, const Partition& part) {
 inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const void* v,
                              const void* beta, const void* gate, void* out, float* S,
                              float* z, bool carry, bool write_state, float* part_S,
-                             float* part_z, __half* S_img, float* S_scale, float* den_dbg,
-                             float* x_dbg, int sms, cudaStream_t stream, void* const* events) {
+                             float* part_z, __half* S_img, float* S_scale, float2* rope_tab,
+                             float* den_dbg, float* x_dbg, int sms, cudaStream_t stream,
+                             void* const* events) {
   auto mark = [&](int i) {
     if (!events || !events[i]) return cudaSuccess;
     return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream);
@@ -1135,10 +1175,11 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
       !make_act_map(&mO, out, g, kTcTile))
     return GLA_ERR_CUDA;
 
-  TcStateParams sp;
+  TcStateParams sp = {};
   sp.g = g; sp.part = spart;
   sp.beta = static_cast<const __nv_bfloat16*>(beta);
   sp.part_S = part_S; sp.part_z = part_z; sp.tab_entries = stab;
+  sp.rope_tab = g.rope_on ? rope_tab : nullptr;
   if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem_st) != cudaSuccess)
     return GLA_ERR_CUDA;
@@ -1156,7 +1197,7 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   if (cudaLaunchKernelEx(&sc, tc_state_kernel, mK, mV, sp) != cudaSuccess || mark(1) != cudaSuccess)
     return GLA_ERR_CUDA;
 
-  CombineParams cp;
+  CombineParams cp = {};
   cp.part = spart; cp.d = 128; cp.zparts = kStTW;
   cp.part_S = part_S; cp.part_z = part_z;
   cp.S_in = carry ? S : nullptr;
@@ -1174,8 +1215,9 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   if (cudaLaunchKernelEx(&cc, combine_kernel, cp) != cudaSuccess || mark(2) != cudaSuccess)
     return GLA_ERR_CUDA;
 
-  TcApplyParams ap;
+  TcApplyParams ap = {};
   ap.g = g; ap.part = part; ap.S_img = S_img; ap.S_scale = S_scale; ap.z = z;
+  ap.rope_tab = rope_tab;
   ap.den_out = den_dbg; ap.x_out = x_dbg; ap.tab_entries = tab;
   const bool dbg = den_dbg != nullptr || x_dbg != nullptr;
   cudaLaunchConfig_t ac = {};
