@@ -7,10 +7,12 @@
 //                    one thread issues tcgen05.mma  S += V^T (beta K_til)  with
 //                    both operands MN-major, accumulating in TMEM; the
 //                    transform warps drain each finished head segment to its
-//                    partial slot.
+//                    partial slot.  The producer warps also write the call's
+//                    whole RoPE table for the read-out.
 //   combine_kernel   (combine.cuh) fixed-order sum of the partials, plus the
 //                    swizzled fp16 image of S.
-//   tc_apply_kernel  persistent read-out.  TMA streams q and g tiles; transform
+//   tc_apply_kernel  persistent read-out.  TMA streams q and g tiles, bulk
+//                    copies bring S, z and its RoPE window; transform
 //                    warps turn q into q_til (fp16, in place) and the
 //                    denominator z.q_pls + eps; one thread issues
 //                    tcgen05.mma  U = Q_til S^T  into a double-buffered TMEM
@@ -880,8 +882,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
     }
   } else if (warp < kApEW0) {
     // ------------------------------------ transform warps: q -> q_til, den
-    // The RoPE table comes by bulk copy from the whole-call table the combine
-    // kernel writes.
+    // The RoPE table comes by bulk copy from the whole-call table that the
+    // state kernel's producer warps write.
     const bool tab_ok = wb >= we || mbar_wait(tfull, 0u, abort_flag);
     const int tw = warp - kApTW0;
     const int rg = tw_row(lane), j = tw_chunk(lane);
