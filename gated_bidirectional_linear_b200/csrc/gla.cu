@@ -115,16 +115,24 @@ Geom make_geom(int batch, int heads, int head_dim, int T, int H, int W, int t0,
   g.eps = eps;
   g.div_HW = make_fastdiv((uint32_t)(H * W));
   g.div_W = make_fastdiv((uint32_t)W);
-  // Rotation frequencies, once per call in double: pair i of an axis with np
-  // pairs turns at theta^(-i/np) radians per position.
-  const int np[3] = {g.pt, g.ph, g.pw};
-  for (int pr = 0, a = 0, i = 0; pr < 64; ++pr) {
-    g.freq[pr] = 0.0;
-    if (pr >= g.pt + g.ph + g.pw || !g.rope_on) continue;
-    while (i >= np[a]) { i -= np[a]; ++a; }
-    g.freq[pr] = exp(-((double)i / (double)np[a]) * log((double)rope_theta));
-    ++i;
+  // Rotation frequencies in double: pair i of an axis with np pairs turns at
+  // theta^(-i/np) radians per position.  Kept per thread for the last
+  // (theta, d), since consecutive calls nearly always repeat them.
+  struct FreqCache { float theta; int d; double freq[64]; };
+  static thread_local FreqCache cache = {0.f, 0, {}};
+  if (!(cache.theta == rope_theta && cache.d == head_dim)) {
+    const int np[3] = {g.pt, g.ph, g.pw};
+    for (int pr = 0, a = 0, i = 0; pr < 64; ++pr) {
+      cache.freq[pr] = 0.0;
+      if (pr >= g.pt + g.ph + g.pw || !g.rope_on) continue;
+      while (i >= np[a]) { i -= np[a]; ++a; }
+      cache.freq[pr] = exp(-((double)i / (double)np[a]) * log((double)rope_theta));
+      ++i;
+    }
+    cache.theta = rope_theta;
+    cache.d = head_dim;
   }
+  memcpy(g.freq, cache.freq, sizeof(g.freq));
   return g;
 }
 

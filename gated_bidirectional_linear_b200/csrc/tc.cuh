@@ -24,6 +24,8 @@
 // the device error word, stops issuing work, drains its copies and frees TMEM.
 #pragma once
 
+#include <atomic>
+
 #include "combine.cuh"
 #include "ptx.cuh"
 
@@ -1127,6 +1129,22 @@ inline size_t tc_apply_smem(int tab_entries) {
 }
 constexpr size_t kMaxSmem = 232448;
 
+// Raises a kernel's dynamic shared-memory limit to kMaxSmem once per device
+// (slot: which kernel), instead of on every call: the attribute only bounds
+// what a launch may ask for.
+template <typename K>
+inline bool ensure_max_smem(K kernel, int slot) {
+  static std::atomic<unsigned char> done[3][64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev >= 0 && dev < 64 && done[slot][dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem) !=
+      cudaSuccess)
+    return false;
+  if (dev >= 0 && dev < 64) done[slot][dev].store(1, std::memory_order_release);
+  return true;
+}
+
 // The state reduction and the read-out split the same items differently
 // (96- and 128-token tiles); each CTA count is at most the SM count.
 inline Partition tc_state_partition(const Geom& g, int sms) {
@@ -1182,9 +1200,7 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   sp.beta = static_cast<const __nv_bfloat16*>(beta);
   sp.part_S = part_S; sp.part_z = part_z; sp.tab_entries = stab;
   sp.rope_tab = g.rope_on ? rope_tab : nullptr;
-  if (cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem_st) != cudaSuccess)
-    return GLA_ERR_CUDA;
+  if (!ensure_max_smem(tc_state_kernel, 0)) return GLA_ERR_CUDA;
   if (mark(0) != cudaSuccess) return GLA_ERR_CUDA;
   cudaLaunchAttribute pdl[1];
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1231,14 +1247,10 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   ac.numAttrs = 1;
   cudaError_t e;
   if (dbg) {
-    if (cudaFuncSetAttribute(tc_apply_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_ap) != cudaSuccess)
-      return GLA_ERR_CUDA;
+    if (!ensure_max_smem(tc_apply_kernel<true>, 1)) return GLA_ERR_CUDA;
     e = cudaLaunchKernelEx(&ac, tc_apply_kernel<true>, mQ, mG, mO, ap);
   } else {
-    if (cudaFuncSetAttribute(tc_apply_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_ap) != cudaSuccess)
-      return GLA_ERR_CUDA;
+    if (!ensure_max_smem(tc_apply_kernel<false>, 2)) return GLA_ERR_CUDA;
     e = cudaLaunchKernelEx(&ac, tc_apply_kernel<false>, mQ, mG, mO, ap);
   }
   if (e != cudaSuccess || mark(3) != cudaSuccess) return GLA_ERR_CUDA;

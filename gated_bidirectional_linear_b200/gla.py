@@ -97,10 +97,43 @@ def _stream(stream):
 
 
 def _dims(q, T, H, W):
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, N, heads, head_dim], got {tuple(q.shape)}")
     B, N, Hh, d = q.shape
     if N != T * H * W:
         raise ValueError(f"q has {N} tokens, grid {T}x{H}x{W} has {T * H * W}")
     return B, Hh, d
+
+
+def _validate(q, k, v, beta, g, out, cuda=True, **extra):
+    """The library sees raw pointers only: check here what it cannot, i.e.
+    that every tensor has the layout and dtype the C ABI documents, is
+    contiguous and lives on one device (a GPU for the device entry points,
+    the host for gla_forward_host).  extra: name -> (tensor, shape, dtype)."""
+    dev = q.device
+    if cuda != (dev.type == "cuda"):
+        raise ValueError(f"q is on {dev}; this entry point takes "
+                         f"{'GPU' if cuda else 'host'} tensors")
+    checks = {"q": (q, q.shape, q.dtype), "k": (k, q.shape, q.dtype), "v": (v, q.shape, q.dtype),
+              "g": (g, q.shape, q.dtype), "beta": (beta, q.shape[:3], q.dtype),
+              "out": (out, q.shape, q.dtype)}
+    checks.update(extra)
+    for name, (t, shape, dtype) in checks.items():
+        if t is None:
+            raise ValueError(f"{name} is missing")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if dtype is not None and t.dtype != dtype:
+            raise ValueError(f"{name} is {t.dtype}, expected {dtype}")
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, q on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def _check_workspace(ws, dev):
+    if ws.device != dev or ws.dtype != torch.uint8 or not ws.is_contiguous():
+        raise ValueError(f"workspace must be a contiguous uint8 tensor on {dev}")
 
 
 def gla_forward_workspace_size(batch, heads, head_dim, T, H, W, dtype):
@@ -129,8 +162,10 @@ def gla_forward(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, out=Non
     code = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out)
     if workspace is None:
         workspace = alloc_workspace(gla_forward_workspace_size(B, Hh, d, T, H, W, code), q.device)
+    _check_workspace(workspace, q.device)
     st = lib().gla_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T, H,
                               W, rope_theta, eps, code, _ptr(out), _ptr(workspace),
                               workspace.numel(), _stream(stream), path)
@@ -147,8 +182,10 @@ def gla_forward_timed(q, k, v, beta, g, T, H, W, events, rope_theta=10000.0, eps
     code = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out)
     if workspace is None:
         workspace = alloc_workspace(gla_forward_workspace_size(B, Hh, d, T, H, W, code), q.device)
+    _check_workspace(workspace, q.device)
     ev = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) if e is not None else None
                                  for e in events])
     st = lib().gla_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
@@ -166,6 +203,7 @@ def gla_forward_debug(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6,
     code = _dtype_code(q)
     dev = q.device
     out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out)
     S = torch.empty(B, Hh, d, d, dtype=torch.float32, device=dev)
     z = torch.empty(B, Hh, d, dtype=torch.float32, device=dev)
     den = torch.empty(B, N, Hh, dtype=torch.float32, device=dev)
@@ -188,9 +226,12 @@ def gla_block_causal_step(state, z, q, k, v, beta, g, T_blk, H, W, t0, rope_thet
     code = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out, state=(state, (B, Hh, d, d), torch.float32),
+              z=(z, (B, Hh, d), torch.float32))
     if workspace is None:
         workspace = alloc_workspace(
             gla_block_causal_workspace_size(B, Hh, d, T_blk, H, W, code), q.device)
+    _check_workspace(workspace, q.device)
     st = lib().gla_block_causal_step_ex(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v),
                                         _ptr(beta), _ptr(g), B, Hh, d, T_blk, H, W, t0,
                                         rope_theta, eps, code, _ptr(out), _ptr(workspace),
@@ -208,8 +249,11 @@ def gla_forward_host(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, ou
     code = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out, cuda=False)
     if arena is None:
         arena = alloc_workspace(gla_forward_host_arena_size(B, Hh, d, T, H, W, code))
+    if arena.device.type != "cuda" or arena.dtype != torch.uint8 or not arena.is_contiguous():
+        raise ValueError("arena must be a contiguous uint8 tensor on the GPU")
     st = lib().gla_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
                                 H, W, rope_theta, eps, code, _ptr(out), _ptr(arena),
                                 arena.numel(), _stream(stream))
@@ -227,6 +271,7 @@ def gla_forward_noalloc(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6,
     code = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out)
     st = lib().gla_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
                                    H, W, rope_theta, eps, code, _ptr(out), _stream(stream))
     _check(st, "gla_forward_noalloc")
