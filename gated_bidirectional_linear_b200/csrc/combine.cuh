@@ -73,7 +73,6 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cg::cluster_group cluster = cg::this_cluster();
   __shared__ float red[kCombineThreads / 32];
-  __shared__ float cta_max;
 
   const int bh = blockIdx.y;
   const int rank = (int)cluster.block_rank();
@@ -141,29 +140,32 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
                        fmaxf(fabsf(acc[k].z), fabsf(acc[k].w))));
   }
 
-  // z: rank 0 adds the ranks' sums in rank order; the head maximum of |S|
-  // travels in the same exchange.
-  __shared__ float zsum[128];
-  if (zlive) zsum[threadIdx.x] = zacc;
+  // One exchange through distributed shared memory and one cluster barrier:
+  // every rank stores its z sums into rank 0's zsum_all[rank] and its |S|
+  // maximum into every rank's max_all[rank]; then rank 0 adds the z sums in
+  // rank order and each rank takes the head maximum from its own copy.  No
+  // rank touches another's shared memory after the barrier, so any may exit.
+  __shared__ float zsum_all[kCombineCluster][128];
+  __shared__ float max_all[kCombineCluster];
+  if (zlive) *cluster.map_shared_rank(&zsum_all[rank][threadIdx.x], 0) = zacc;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < kCombineCluster) {
     float mm = red[0];
     for (int w = 1; w < kCombineThreads / 32; ++w) mm = fmaxf(mm, red[w]);
-    cta_max = mm;
+    *cluster.map_shared_rank(&max_all[rank], (int)threadIdx.x) = mm;
   }
   cluster.sync();
   if (rank == 0 && zlive) {
     float zs = p.z_in ? p.z_in[(size_t)bh * d + threadIdx.x] : 0.f;
-    for (int r = 0; r < kCombineCluster; ++r) zs += *cluster.map_shared_rank(&zsum[threadIdx.x], r);
+    for (int r = 0; r < kCombineCluster; ++r) zs += zsum_all[r][threadIdx.x];
     p.z_out[(size_t)bh * d + threadIdx.x] = zs;
   }
   float hm = 0.f;
   if (p.S_img != nullptr)
-    for (int r = 0; r < kCombineCluster; ++r) hm = fmaxf(hm, *cluster.map_shared_rank(&cta_max, r));
-  cluster.sync();   // every rank's zsum / cta_max stays valid until all have read
+    for (int r = 0; r < kCombineCluster; ++r) hm = fmaxf(hm, max_all[r]);
 
   if (p.S_img == nullptr) return;     // uniform over the whole grid
 
