@@ -30,7 +30,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from gated_bidirectional_linear_b200 import workloads  # noqa: E402
+from gated_bidirectional_linear_b200 import replicas, workloads  # noqa: E402
 
 METRIC = "gla_forward tokens/s (20x128 heads, 14720 tok) and HBM GB/s vs B200 peak"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -234,7 +234,7 @@ def main():
         run_block_causal(args, wl, gla, dev, dist, world, rank, local)
         return
 
-    inp = workloads.make_inputs(wl, seed=wl.seed + rank)
+    inp = workloads.make_inputs(wl, seed=replicas.replica_seed(wl.seed, rank))
     d = {k: v.to(dev) for k, v in inp.items()}
     B, N, Hh, hd = d["q"].shape
     code = gla.GLA_DTYPE_BF16 if d["q"].dtype == torch.bfloat16 else gla.GLA_DTYPE_F32
@@ -268,28 +268,14 @@ def main():
                         wl.rope_theta, wl.eps, out=out, workspace=ws, stream=stream)
 
     # Timed region: K plain steps (the kernels chain by programmatic dependent
-    # launch, so nothing is recorded between them).
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    # launch, so nothing is recorded between them); max over ranks.
+    sync = lambda: torch.cuda.synchronize(dev)
     with ClockMonitor(local) as mon:
-        if dist:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        t_start.record(stream)
-        for i in range(args.steps):
-            plain_step()
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
-        if dist:
-            dist.barrier()
+        elapsed_ms = replicas.timed(lambda: [plain_step() for _ in range(args.steps)],
+                                    replicas.CudaTimer(stream), dist, sync, dev)
     status = gla.gla_get_device_status(stream)
     if status != gla.GLA_OK:
         raise RuntimeError(f"device status after the timed region: {gla.status_string(status)}")
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if dist:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
 
     # Per-kernel durations for the roofline: a second timed pass of K steps
     # with CUDA events recorded on the launching stream around each kernel
@@ -318,31 +304,21 @@ def main():
         gla.gla_forward_host(pinned["q"], pinned["k"], pinned["v"], pinned["beta"], pinned["g"],
                              wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, out=out_h, arena=arena,
                              stream=stream)
-    torch.cuda.synchronize(dev)
-    if dist:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        gla.gla_forward_host(pinned["q"], pinned["k"], pinned["v"], pinned["beta"], pinned["g"],
-                             wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, out=out_h, arena=arena,
-                             stream=stream)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-        dist.barrier()
+
+    def host_steps():
+        for _ in range(e2e_steps):
+            gla.gla_forward_host(pinned["q"], pinned["k"], pinned["v"], pinned["beta"],
+                                 pinned["g"], wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, out=out_h,
+                                 arena=arena, stream=stream)
+
+    e2e_ms = replicas.timed(host_steps, replicas.CudaTimer(stream), dist, sync, dev)
 
     th = B * N * Hh
     esz = 2 if code == gla.GLA_DTYPE_BF16 else 4
     tokens_per_step = B * N
     ms_per_step = elapsed_ms / args.steps
-    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
-    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+    value = replicas.aggregate_rate(world, tokens_per_step, args.steps, elapsed_ms)
+    e2e_value = replicas.aggregate_rate(world, tokens_per_step, e2e_steps, e2e_ms)
     peak, peak_kind = measured_peaks()
     apply_bytes = th * hd * esz * 3                # q, g read + out written
     state_bytes = th * hd * esz * 2 + th * esz     # k, v, beta read
@@ -401,7 +377,7 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
     """One step = a whole sequence of wl.n_blocks blocks through
     gla_block_causal_step, from a zero state (a new sequence).  Not the
     headline metric: the block-causal row's own measurement."""
-    inp = workloads.make_inputs(wl, seed=wl.seed + rank)
+    inp = workloads.make_inputs(wl, seed=replicas.replica_seed(wl.seed, rank))
     L = wl.tokens
     blocks = [{k: v[:, i * L:(i + 1) * L].contiguous().to(dev) for k, v in inp.items()}
               for i in range(wl.n_blocks)]
@@ -426,25 +402,12 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
     torch.cuda.synchronize(dev)
     assert gla.gla_get_device_status(stream) == gla.GLA_OK
     steps = max(1, args.steps // wl.n_blocks)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync = lambda: torch.cuda.synchronize(dev)
     with ClockMonitor(local) as mon:
-        if dist:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        t0.record(stream)
-        for _ in range(steps):
-            sequence()
-        t1.record(stream)
-        torch.cuda.synchronize(dev)
-        if dist:
-            dist.barrier()
+        ms = replicas.timed(lambda: [sequence() for _ in range(steps)],
+                            replicas.CudaTimer(stream), dist, sync, dev)
     if gla.gla_get_device_status(stream) != gla.GLA_OK:
         raise RuntimeError("device status after the timed region")
-    ms = t0.elapsed_time(t1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
 
     # End to end: the sequence's inputs from pinned host memory, the steps,
     # and the outputs back, every step.
@@ -461,18 +424,8 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
 
     e2e_steps = max(3, min(steps, 50))
     sequence_host()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        sequence_host()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = replicas.timed(lambda: [sequence_host() for _ in range(e2e_steps)],
+                            replicas.CudaTimer(stream), dist, sync, dev)
 
     tokens = B * wl.total_tokens
     th = tokens * Hh
@@ -507,7 +460,8 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
                               f"cores = BLAS threads")}
         line = {
             "metric": "gla_block_causal_step tokens/s (20x128 heads, 20 blocks of 3x23x40)",
-            "value": world * tokens * steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "value": replicas.aggregate_rate(world, tokens, steps, ms), "unit": "tokens/s",
+            "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
@@ -518,7 +472,8 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
                          "unit": "GB/s", "frac": gbs / peak, "peak_kind": peak_kind,
                          "traffic": None, "alg_bytes_per_step": alg,
                          "state_bytes_per_step": state_io},
-            "e2e": {"value": world * tokens * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": replicas.aggregate_rate(world, tokens, e2e_steps, e2e_ms),
+                    "unit": "tokens/s",
                     "h2d_bytes_per_step": th * hd * 2 * 4 + th * 2,
                     "d2h_bytes_per_step": th * hd * 2, "steps": e2e_steps},
             "gpu_launches": 3 * wl.n_blocks * steps,
