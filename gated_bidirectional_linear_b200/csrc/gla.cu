@@ -4,6 +4,8 @@
 // Host code validates arguments, plans the split-N partition, carves the
 // caller's workspace and launches the kernels on the caller's stream.
 #include <math.h>
+
+#include <mutex>
 #include <stdint.h>
 #include <string.h>
 
@@ -80,6 +82,34 @@ WsLayout ws_layout(int BH, int d, bool own_state, int T, int H, int W) {
   if (d == 128) off = align_up(off + rope_tab_bytes(d, T, H, W), kAlign);
   L.total = off;
   return L;
+}
+
+// The helper stream (one per device, created on first use and kept for the
+// process) that carries gla_forward_host's output copies, and the events that
+// fork it from and join it to the caller's stream.  The mutex keeps one
+// call's fork and join together when several host threads use the device.
+constexpr int kHostChunks = 8;
+struct HostPipe {
+  std::mutex mu;
+  cudaStream_t s = nullptr;
+  cudaEvent_t ev[kHostChunks + 1] = {};
+};
+
+HostPipe* host_pipe() {
+  static std::mutex init_mu;
+  static HostPipe pipes[64];
+  static bool ready[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(init_mu);
+  if (!ready[dev]) {
+    HostPipe& p = pipes[dev];
+    if (cudaStreamCreateWithFlags(&p.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    for (auto& e : p.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    ready[dev] = true;
+  }
+  return &pipes[dev];
 }
 
 bool dims_ok(int batch, int heads, int head_dim, int T, int H, int W) {
@@ -432,7 +462,9 @@ size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, int T, in
   if (!ws) return 0;
   const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
   const size_t th = (size_t)batch * T * H * W * heads;
-  return 5 * align_up(th * head_dim * esz, kAlign) + align_up(th * esz, kAlign) + ws;
+  // beta: room for each batch group's slice to start on a 16-byte boundary.
+  return 5 * align_up(th * head_dim * esz, kAlign) +
+         align_up(th * esz + 16 * (kHostChunks + 1), kAlign) + ws;
 }
 
 gla_status gla_forward_host(const void* q_h, const void* k_h, const void* v_h,
@@ -456,21 +488,67 @@ gla_status gla_forward_host(const void* q_h, const void* k_h, const void* v_h,
   unsigned char* dg = dv + align_up(big, kAlign);
   unsigned char* dout = dg + align_up(big, kAlign);
   unsigned char* dbeta = dout + align_up(big, kAlign);
-  unsigned char* dws = dbeta + align_up(small, kAlign);
+  unsigned char* dws = dbeta + align_up(small + 16 * (kHostChunks + 1), kAlign);
+  const size_t ws_bytes = arena_bytes - (size_t)(dws - a);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(dq, q_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dg, g_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dbeta, beta_h, small, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return GLA_ERR_CUDA;
-  const gla_status st = gla_forward(dq, dk, dv, dbeta, dg, batch, heads, head_dim, T, H, W,
-                                    rope_theta, eps, dtype, dout, dws,
-                                    arena_bytes - (size_t)(dws - a), stream);
-  if (st != GLA_OK) return st;
-  if (cudaMemcpyAsync(out_h, dout, big, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return GLA_ERR_CUDA;
-  return GLA_OK;
+  const unsigned char* hq = static_cast<const unsigned char*>(q_h);
+  const unsigned char* hk = static_cast<const unsigned char*>(k_h);
+  const unsigned char* hv = static_cast<const unsigned char*>(v_h);
+  const unsigned char* hg = static_cast<const unsigned char*>(g_h);
+  const unsigned char* hb = static_cast<const unsigned char*>(beta_h);
+  unsigned char* ho = static_cast<unsigned char*>(out_h);
+
+  // Batch elements are independent and contiguous: with two or more, the
+  // call runs per group of them, and each group's output copy goes out on a
+  // helper stream while the next group's inputs come in (PCIe carries both
+  // directions at once).  The helper is joined back into `stream` before
+  // the call returns, so `stream` orders everything as before.
+  HostPipe* pipe = batch >= 2 ? host_pipe() : nullptr;
+  const int chunks = pipe ? (batch < kHostChunks ? batch : kHostChunks) : 1;
+  std::unique_lock<std::mutex> lock;
+  if (pipe) lock = std::unique_lock<std::mutex>(pipe->mu);
+  bool forked = false;
+  gla_status st = GLA_OK;
+  for (int c = 0; c < chunks && st == GLA_OK; ++c) {
+    const int b0 = (int)((long long)batch * c / chunks), b1 = (int)((long long)batch * (c + 1) / chunks);
+    const size_t ob = big / batch * b0, nb = big / batch * (b1 - b0);
+    const size_t os = small / batch * b0, ns = small / batch * (b1 - b0);
+    // The group's beta slice starts on a 16-byte boundary in the arena (the
+    // operator's pointers must be 16-byte aligned); slices stay disjoint.
+    const size_t od = align_up(os, 16) + 16 * (size_t)c;
+    if (cudaMemcpyAsync(dq + ob, hq + ob, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dk + ob, hk + ob, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv + ob, hv + ob, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dg + ob, hg + ob, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dbeta + od, hb + os, ns, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+      st = GLA_ERR_CUDA;
+      break;
+    }
+    st = gla_forward(dq + ob, dk + ob, dv + ob, dbeta + od, dg + ob, b1 - b0, heads, head_dim,
+                     T, H, W, rope_theta, eps, dtype, dout + ob, dws, ws_bytes, stream);
+    if (st != GLA_OK) break;
+    if (!pipe) {
+      if (cudaMemcpyAsync(ho + ob, dout + ob, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        st = GLA_ERR_CUDA;
+      break;
+    }
+    if (cudaEventRecord(pipe->ev[c], s) != cudaSuccess ||
+        cudaStreamWaitEvent(pipe->s, pipe->ev[c], 0) != cudaSuccess) {
+      st = GLA_ERR_CUDA;
+      break;
+    }
+    forked = true;
+    if (cudaMemcpyAsync(ho + ob, dout + ob, nb, cudaMemcpyDeviceToHost, pipe->s) != cudaSuccess)
+      st = GLA_ERR_CUDA;
+  }
+  if (forked) {
+    // Join, also after an error, so that no copy of this call outlives it
+    // unordered with `stream`.
+    if (cudaEventRecord(pipe->ev[kHostChunks], pipe->s) != cudaSuccess ||
+        cudaStreamWaitEvent(s, pipe->ev[kHostChunks], 0) != cudaSuccess)
+      st = GLA_ERR_CUDA;
+  }
+  return st;
 }
 
 // ---------------------------------------------------------------------------

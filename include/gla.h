@@ -183,11 +183,20 @@ GLA_API size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, i
                                    int dtype);
 
 /* gla_forward on HOST buffers (q_h .. out_h; pinned memory gives asynchronous
- * copies).  Enqueues on `stream`: one host-to-device copy per input into the
- * caller's device `arena`, the operator, and one device-to-host copy of the
- * output.  Returns after enqueueing; synchronise `stream` before reading
- * out_h.  The arena is caller-owned device memory of at least
- * gla_forward_host_arena_size() bytes, 256-byte aligned. */
+ * copies).  Enqueues on `stream`: host-to-device copies of the inputs into the
+ * caller's device `arena`, the operator, and device-to-host copies of the
+ * output.  With batch >= 2 the call runs per group of batch elements (at most
+ * 8 groups; batch elements are independent): each group's output copy is
+ * issued on a helper stream the library owns (one per device, created on the
+ * first such call) so that it overlaps the next group's input copies, and the
+ * helper is joined back into `stream` before the call's work ends.  Each
+ * group is one gla_forward call over its batch elements, so the output equals
+ * that of gla_forward on the same groups bit for bit, and a whole-batch
+ * gla_forward call within rounding (the split-N partition differs).  Returns
+ * after enqueueing; synchronise `stream` before reading out_h.  The arena is
+ * caller-owned device memory of at least gla_forward_host_arena_size() bytes,
+ * 256-byte aligned.  Not for use inside a CUDA graph capture when batch >= 2
+ * (the helper stream is not part of the capture). */
 GLA_API gla_status gla_forward_host(const void* q_h, const void* k_h, const void* v_h,
                             const void* beta_h, const void* g_h, int batch, int heads,
                             int head_dim, int T, int H, int W, float rope_theta, float eps,

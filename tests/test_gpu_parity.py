@@ -222,6 +222,28 @@ def test_host_entry_matches_device_entry():
     assert torch.equal(out_h, dev.cpu())
 
 
+def test_host_entry_overlapped_batches():
+    """batch >= 2: the host entry runs per batch element, output copies on a
+    helper stream; the result equals gla_forward on each element, bit for
+    bit, and the oracle within the bf16 tolerance."""
+    T, H, W, B, HH = 3, 5, 7, 3, 4
+    inp = workloads.draw(B, T * H * W, HH, 128, "bf16", seed=23)
+    pinned = {k: v.pin_memory() for k, v in inp.items()}
+    out_h = torch.empty_like(pinned["q"]).pin_memory()
+    gla.gla_forward_host(pinned["q"], pinned["k"], pinned["v"], pinned["beta"], pinned["g"],
+                         T, H, W, out=out_h)
+    torch.cuda.synchronize()
+    d = to_device(inp)
+    for b in range(B):
+        one = {k: v[b:b + 1].contiguous() for k, v in d.items()}
+        dev = gla.gla_forward(one["q"], one["k"], one["v"], one["beta"], one["g"], T, H, W)
+        torch.cuda.synchronize()
+        assert torch.equal(out_h[b:b + 1], dev.cpu())
+    x = workloads.as_f64(inp)
+    ref = O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T, H, W, 10000.0, 1e-6)
+    assert O.max_err_over_rms(out_h.to(torch.float64).numpy(), ref["out"]) <= 2e-2
+
+
 def test_time_offset_invariance_single_block():
     """One block from zero state with t0 = 0 and t0 = 7 (fp32): rotated dot
     products depend on position differences only."""
