@@ -235,7 +235,7 @@ def test_host_entry_overlapped_batches():
     torch.cuda.synchronize()
     d = to_device(inp)
     for b in range(B):
-        one = {k: v[b:b + 1].contiguous() for k, v in d.items()}
+        one = {k: v[b:b + 1].clone() for k, v in d.items()}   # fresh, 16-byte aligned
         dev = gla.gla_forward(one["q"], one["k"], one["v"], one["beta"], one["g"], T, H, W)
         torch.cuda.synchronize()
         assert torch.equal(out_h[b:b + 1], dev.cpu())
