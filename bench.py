@@ -269,10 +269,15 @@ def main():
 
     # Timed region: K plain steps (the kernels chain by programmatic dependent
     # launch, so nothing is recorded between them); max over ranks.
-    sync = lambda: torch.cuda.synchronize(dev)
+    def sync():
+        torch.cuda.synchronize(dev)
+
+    def timed_steps():
+        for _ in range(args.steps):
+            plain_step()
+
     with ClockMonitor(local) as mon:
-        elapsed_ms = replicas.timed(lambda: [plain_step() for _ in range(args.steps)],
-                                    replicas.CudaTimer(stream), dist, sync, dev)
+        elapsed_ms = replicas.timed(timed_steps, replicas.CudaTimer(stream), dist, sync, dev)
     status = gla.gla_get_device_status(stream)
     if status != gla.GLA_OK:
         raise RuntimeError(f"device status after the timed region: {gla.status_string(status)}")
@@ -402,10 +407,15 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
     torch.cuda.synchronize(dev)
     assert gla.gla_get_device_status(stream) == gla.GLA_OK
     steps = max(1, args.steps // wl.n_blocks)
-    sync = lambda: torch.cuda.synchronize(dev)
+    def sync():
+        torch.cuda.synchronize(dev)
+
+    def timed_sequences():
+        for _ in range(steps):
+            sequence()
+
     with ClockMonitor(local) as mon:
-        ms = replicas.timed(lambda: [sequence() for _ in range(steps)],
-                            replicas.CudaTimer(stream), dist, sync, dev)
+        ms = replicas.timed(timed_sequences, replicas.CudaTimer(stream), dist, sync, dev)
     if gla.gla_get_device_status(stream) != gla.GLA_OK:
         raise RuntimeError("device status after the timed region")
 
@@ -424,8 +434,11 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
 
     e2e_steps = max(3, min(steps, 50))
     sequence_host()
-    e2e_ms = replicas.timed(lambda: [sequence_host() for _ in range(e2e_steps)],
-                            replicas.CudaTimer(stream), dist, sync, dev)
+    def host_sequences():
+        for _ in range(e2e_steps):
+            sequence_host()
+
+    e2e_ms = replicas.timed(host_sequences, replicas.CudaTimer(stream), dist, sync, dev)
 
     tokens = B * wl.total_tokens
     th = tokens * Hh

@@ -211,7 +211,8 @@ GLA_API gla_status gla_forward_host(const void* q_h, const void* k_h, const void
  * runtime that owns every allocation, in a plugin that must not grow the
  * process footprint at call time, or on a path that may not synchronise the
  * device, which cudaMalloc can do).  The operator's scratch space (split-N
- * partial states, the combined state and its fp16 image) comes from one
+ * partial states, the combined state, its fp16 image and the RoPE table)
+ * comes from one
  * array of GLA_NOALLOC_SCRATCH_BYTES compiled into this library; every GPU
  * that loads the library holds that array until the process exits.  The
  * caller still passes the inputs and `out`.  No counterpart on the pages: it
