@@ -673,4 +673,48 @@ gla_status gla_plan(int batch, int heads, int head_dim, int T, int H, int W, int
   return GLA_OK;
 }
 
+gla_status gla_check_rope_copy(int batch, int heads, int head_dim, int T, int H, int W,
+                               int num_sms) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W) || num_sms <= 0) return GLA_ERR_INVALID_ARG;
+  const Geom g = make_geom(batch, heads, head_dim, T, H, W, 0, 10000.f, 1e-6f);
+  if (!tc_rope_lanes_ok(g)) return GLA_ERR_UNSUPPORTED;
+  const Partition p = tc_apply_partition(g, num_sms);
+  const RopeLayout G = rope_layout(g, g.T);
+  const int smem_entries = tc_table_entries(g, p);
+  const int P = g.pt + g.ph + g.pw;
+  for (int c = 0; c < p.grid; ++c) {
+    const RopeWindow win = rope_window(g, p, part_begin(p, c), part_begin(p, c + 1) - 1);
+    const RopeLayout L = rope_layout(g, win.Lt);
+    const RopeCopy rc = rope_copy_plan(g, win);
+    if (rc.n < 3 || rc.n > 4 || L.entries > smem_entries) return GLA_ERR_INVALID_ARG;
+    for (int i = 0; i < rc.n; ++i) {
+      // Bulk copies: 16-byte aligned addresses and sizes (entries are 8 bytes;
+      // the plan promises multiples of 8 entries).
+      if (rc.src[i] % 8 || rc.dst[i] % 8 || rc.len[i] % 8 || rc.len[i] <= 0) return GLA_ERR_INVALID_ARG;
+      if (rc.src[i] + rc.len[i] > G.entries || rc.dst[i] + rc.len[i] > L.entries)
+        return GLA_ERR_INVALID_ARG;
+    }
+    // Every entry the read-out looks up comes from the whole-call entry of
+    // the same pair at the same absolute position.
+    for (int pr = 0; pr < P; ++pr) {
+      const int a = pr < g.pt ? 0 : (pr < g.pt + g.ph ? 1 : 2);
+      const int rows = a == 0 ? win.Lt : (a == 1 ? g.H : g.W);
+      for (int pos = 0; pos < rows; ++pos) {
+        const int e = L.base[a] + pos * L.stride[a] + rope_idx(L, a, pr);
+        int gp = pos;
+        if (a == 0) {
+          gp = win.t_lo + pos;
+          if (gp >= g.T) gp -= g.T;
+        }
+        const int ge = G.base[a] + gp * G.stride[a] + rope_idx(G, a, pr);
+        int src = -1;
+        for (int i = 0; i < rc.n; ++i)
+          if (e >= rc.dst[i] && e < rc.dst[i] + rc.len[i]) src = rc.src[i] + (e - rc.dst[i]);
+        if (src != ge) return GLA_ERR_INVALID_ARG;
+      }
+    }
+  }
+  return GLA_OK;
+}
+
 }  // extern "C"

@@ -42,6 +42,7 @@ _SIGS = {
     "gla_get_device_status": (_i, [_vp]),
     "gla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "gla_plan": (_i, [_i] * 9 + [ctypes.POINTER(_i)] * 3),
+    "gla_check_rope_copy": (_i, [_i] * 7),
 }
 
 _lib = None
@@ -297,3 +298,8 @@ def gla_plan(batch, heads, head_dim, T, H, W, dtype, path, num_sms):
                         ctypes.byref(grid), ctypes.byref(tile), ctypes.byref(used))
     _check(st, "gla_plan")
     return grid.value, tile.value, used.value
+
+
+def gla_check_rope_copy(batch, heads, head_dim, T, H, W, num_sms):
+    """Host-only check of the read-out's RoPE table copy plan (status code)."""
+    return lib().gla_check_rope_copy(batch, heads, head_dim, T, H, W, num_sms)

@@ -247,6 +247,17 @@ GLA_API gla_status gla_get_device_status(void* stream);
  * GLA_ERR_CUDA if the launch fails, else GLA_OK. */
 GLA_API gla_status gla_selftest_wait_timeout(unsigned int limit_us, void* stream);
 
+/* Host-only self-check of the tensor read-out's RoPE table copies (tests; no
+ * GPU needed): for every read-out CTA of this problem on num_sms SMs, the bulk
+ * copies that bring its table window from the whole-call table are 16-byte
+ * aligned, stay inside both tables and the CTA's shared-memory table, and
+ * bring every entry the CTA looks up from the whole-call entry of the same
+ * rotation pair and absolute position.  GLA_OK, GLA_ERR_UNSUPPORTED (no
+ * tensor path for this head dim) or GLA_ERR_INVALID_ARG (bad sizes, or a
+ * violated check). */
+GLA_API gla_status gla_check_rope_copy(int batch, int heads, int head_dim, int T, int H, int W,
+                                       int num_sms);
+
 /* Host-only planning query (no GPU needed): the grid of the state-reduction
  * kernel and the tokens per tile for this problem on a GPU with `num_sms`
  * SMs and the given path.  Returns GLA_OK and fills *grid, *tile_tokens,
