@@ -52,7 +52,8 @@ Readings taken where the pages are silent (all listed in the design notes):
     position is offset by t0 in the block-causal variant.  rope_theta <= 0
     turns RoPE off.
   * Block-causal: a token of block b sees every token of blocks 0..b
-    (inclusive of its own block).
+    (inclusive of its own block).  Token-level causal: token j sees tokens
+    0..j (inclusive of itself).
 
 Tensors are numpy float64 arrays: q, k, v, g are [B, N, Hh, d] and beta is
 [B, N, Hh]; N = T*H*W.
@@ -261,6 +262,45 @@ def block_causal_bruteforce(q, k, v, beta, g, n_blocks, T_blk, H, W, rope_theta,
     L = T_blk * H * W
     return forward_bruteforce(q, k, v, beta, g, n_blocks * T_blk, H, W, rope_theta,
                               eps, visible=lambda j, n: n // L <= j // L)
+
+
+# -------------------------------------------------------- token-level causal
+
+def causal_forward(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
+    """Token-level causal variant: token j is read out against the running
+    sums, over tokens 0..j, of the per-token states v_n (beta_n k_til_n)^T and
+    of the key features k_pls_n ([BLK]: causal linear attention needs only
+    these two running sums; a token sees itself, as a block does).
+
+        S_j = sum_{n<=j} v_n (beta_n k_til_n)^T      z_j = sum_{n<=j} k_pls_n
+        den_j = z_j . q_pls_j + eps                  pre_j = S_j q_til_j / den_j
+
+    Positions and the rest of the read-out as in forward().  The running sums
+    are np.cumsum over the per-token terms, so memory grows as N*d*d: small
+    inputs only."""
+    d = q.shape[-1]
+    assert q.shape[1] == T * H * W
+    angles = _angles_or_none(d, T, H, W, rope_theta, t0)
+    q_pls, q_til = feature_maps(q, angles)
+    k_pls, k_til = feature_maps(k, angles)
+    B, N, Hh, _ = q.shape
+    den = np.empty((B, N, Hh))
+    pre = np.empty_like(q)
+    for b in range(B):
+        for h in range(Hh):
+            per_token = v[b, :, h, :, None] * (beta[b, :, h, None, None] * k_til[b, :, h, None, :])
+            S_run = np.cumsum(per_token, axis=0)                  # [N, d, d]
+            z_run = np.cumsum(k_pls[b, :, h, :], axis=0)          # [N, d]
+            den[b, :, h] = np.einsum("nc,nc->n", z_run, q_pls[b, :, h, :]) + eps
+            pre[b, :, h, :] = np.einsum("nac,nc->na", S_run, q_til[b, :, h, :]) / den[b, :, h, None]
+    x = sigmoid(g) * pre
+    return dict(den=den, pre=pre, x=x, out=rms_normalize(x))
+
+
+def causal_bruteforce(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
+    """Prefix-masked pair sum: token j sees token n iff n <= j."""
+    return forward_bruteforce(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=t0,
+                              visible=lambda j, n: n <= j)
 
 
 # ------------------------------------------------------------- parity metric

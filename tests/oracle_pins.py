@@ -307,4 +307,58 @@ def check_block_causal_final_state():
     _close(c["out"][:, -L:], f["out"][:, -L:], 1e-11, "last block = bidirectional")
 
 
+def _causal_inputs(H=3, W=2, T=4, d=8, seed=31):
+    rng = np.random.default_rng(seed)
+    N = T * H * W
+    q, k, v, g = (rng.standard_normal((2, N, 2, d)) for _ in range(4))
+    beta = rng.uniform(0.0, 1.0, (2, N, 2))
+    return (q, k, v, beta, g), (T, H, W)
+
+
+def check_causal_bruteforce():
+    """Token-level causal ([BLK] running sums): equals the pair sum where
+    token j sees token n iff n <= j."""
+    (q, k, v, beta, g), (T, H, W) = _causal_inputs()
+    c = O.causal_forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5)
+    bf = O.causal_bruteforce(q, k, v, beta, g, T, H, W, 10000.0, 1e-5)
+    _close(c["out"], bf["out"], 1e-11, "causal vs prefix-masked brute force")
+    _close(c["x"], bf["x"], 1e-11, "causal gated read-out vs brute force")
+
+
+def check_causal_last_token_sees_everything():
+    """The last token's prefix is the whole sequence: its output is the
+    bidirectional output."""
+    (q, k, v, beta, g), (T, H, W) = _causal_inputs()
+    c = O.causal_forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5)
+    f = O.forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5)
+    _close(c["out"][:, -1], f["out"][:, -1], 1e-11, "causal last token = bidirectional")
+
+
+def check_causal_first_token_alone():
+    """The first token sees only itself: its output is the one-token
+    operator on that token, whatever follows."""
+    (q, k, v, beta, g), (T, H, W) = _causal_inputs()
+    c = O.causal_forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5)
+    one = O.forward(q[:, :1], k[:, :1], v[:, :1], beta[:, :1], g[:, :1], 1, 1, 1, 10000.0, 1e-5)
+    _close(c["out"][:, 0], one["out"][:, 0], 1e-12, "causal first token = single token")
+
+
+def check_causal_is_one_token_blocks():
+    """With one token per frame (H = W = 1), token-level causal equals the
+    block-causal carry with one-frame blocks."""
+    (q, k, v, beta, g), (T, H, W) = _causal_inputs(H=1, W=1, T=9)
+    c = O.causal_forward(q, k, v, beta, g, T, 1, 1, 10000.0, 1e-5)
+    b = O.block_causal_forward(q, k, v, beta, g, T, 1, 1, 1, 10000.0, 1e-5)
+    _close(c["out"], b["out"], 1e-11, "causal = one-token blocks")
+
+
+def check_causal_time_shift_invariance():
+    """ReLU before RoPE: numerators depend on position differences only, so a
+    global time shift leaves the causal output unchanged ([V1])."""
+    (q, k, v, beta, g), (T, H, W) = _causal_inputs()
+    a = O.causal_forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5, t0=0)
+    b = O.causal_forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5, t0=7)
+    _close(a["out"], b["out"], 1e-10, "causal time shift")
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

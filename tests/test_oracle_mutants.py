@@ -85,6 +85,34 @@ def _neg_sigmoid(x):
     return 1.0 / (1.0 + np.exp(x))
 
 
+def _causal_exclusive(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
+    """Token j reads the running sums over tokens 0..j-1 only (the printed
+    sum_{j<i} taken literally)."""
+    d = q.shape[-1]
+    angles = None if rope_theta <= 0 else O.rope_angles(d, T, H, W, rope_theta, t0)
+    q_pls, q_til = O.feature_maps(q, angles)
+    k_pls, k_til = O.feature_maps(k, angles)
+    B, N, Hh, _ = q.shape
+    pre = np.empty_like(q)
+    for b in range(B):
+        for h in range(Hh):
+            per = v[b, :, h, :, None] * (beta[b, :, h, None, None] * k_til[b, :, h, None, :])
+            S_run = np.cumsum(per, axis=0) - per
+            z_run = np.cumsum(k_pls[b, :, h, :], axis=0) - k_pls[b, :, h, :]
+            den = np.einsum("nc,nc->n", z_run, q_pls[b, :, h, :]) + eps
+            pre[b, :, h, :] = np.einsum("nac,nc->na", S_run, q_til[b, :, h, :]) / den[:, None]
+    x = O.sigmoid(g) * pre
+    return dict(pre=pre, x=x, out=O.rms_normalize(x))
+
+
+def _causal_suffix(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
+    """Running sums taken from the end of the sequence instead of the start."""
+    flip = lambda a: a[:, ::-1]
+    r = _orig["causal_forward"](flip(q), flip(k), flip(v), flip(beta), flip(g), T, H, W,
+                                rope_theta, eps, t0)
+    return {key: flip(val) for key, val in r.items()}
+
+
 MUTANTS = {
     "rope_backwards": ("rope_rotate", _rotate_backwards),
     "rope_before_relu": ("feature_maps", _rope_before_relu),
@@ -101,6 +129,8 @@ MUTANTS = {
     "rope_no_time_offset": ("token_positions", _no_time_offset),
     "block_exclusive": ("block_causal_step", _exclusive_block),
     "sigmoid_sign": ("sigmoid", _neg_sigmoid),
+    "causal_exclusive": ("causal_forward", _causal_exclusive),
+    "causal_suffix": ("causal_forward", _causal_suffix),
 }
 
 
