@@ -21,6 +21,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace gla {
 
@@ -64,72 +65,19 @@ __device__ __forceinline__ void add4(float4& s, const float4 t) {
   s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
 }
 
-__global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombineThreads)
-    combine_kernel(CombineParams p) {
-  namespace cg = cooperative_groups;
-  // Launched as a programmatic dependent of the state reduction: wait for its
-  // partials, and let the read-out kernel start its own prologue meanwhile.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  cg::cluster_group cluster = cg::this_cluster();
+// The part both combine kernels share, from the summed slice on: S_out, the
+// head maximum and z through one exchange in distributed shared memory, the
+// image scale and the fp16 image of this rank's slice.
+__device__ __forceinline__ void combine_finish(const CombineParams& p,
+                                               cooperative_groups::cluster_group& cluster,
+                                               int bh, int rank, const float4 (&acc)[2],
+                                               const bool (&live)[2], float zacc) {
   __shared__ float red[kCombineThreads / 32];
-
-  const int bh = blockIdx.y;
-  const int rank = (int)cluster.block_rank();
   const int d = p.d;
-  const long long tph = p.part.tiles_per_head;
-  const int c_lo = part_cta_of(p.part, (long long)bh * tph);
-  const int c_hi = part_cta_of(p.part, (long long)(bh + 1) * tph - 1);
   const size_t dd = (size_t)d * d;
-  const int chunk = (int)(dd / kCombineCluster);        // 2048 for d = 128
+  const int chunk = (int)(dd / kCombineCluster);
   const int e_base = rank * chunk;
-
-  // Each thread owns up to two float4 groups of S (e = e_base + 4*tid + 1024*k)
-  // and, for d <= 128, one element e = tid of the z partials this rank adds
-  // (partials rank, rank + 8, ... of each slot).  All loads of a batch of
-  // slots are issued before any is added, then added in slot order.
-  constexpr int kBatch = 4;
-  float4 acc[2];
-  float zacc = 0.f;
-  bool live[2];
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
-    live[k] = e < e_base + chunk;
-    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (live[k] && p.S_in)
-      acc[k] = *reinterpret_cast<const float4*>(p.S_in + bh * dd + row_major(p, e));
-  }
   const bool zlive = (int)threadIdx.x < d;
-  for (int c0 = c_lo; c0 <= c_hi; c0 += kBatch) {
-    float4 t[kBatch][2];
-    float zt[kBatch][4];
-#pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int c = c0 + b;
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
-        t[b][k] = (c <= c_hi && live[k])
-                      ? *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + bh) * dd + e)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int zp = rank + kCombineCluster * q;
-        zt[b][q] = (c <= c_hi && zlive && zp < p.zparts)
-                       ? p.part_z[(((size_t)c + bh) * p.zparts + zp) * d + threadIdx.x]
-                       : 0.f;
-      }
-    }
-#pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      if (c0 + b > c_hi) break;
-      add4(acc[0], t[b][0]);
-      add4(acc[1], t[b][1]);
-      zacc += zt[b][0]; zacc += zt[b][1]; zacc += zt[b][2]; zacc += zt[b][3];
-    }
-  }
   float m = 0.f;
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
@@ -194,6 +142,161 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
     pk.y = *reinterpret_cast<uint32_t*>(&hi);
     *reinterpret_cast<uint2*>(img + simg_offset(a, cc)) = pk;
   }
+}
+
+__global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombineThreads)
+    combine_kernel(CombineParams p) {
+  namespace cg = cooperative_groups;
+  // Launched as a programmatic dependent of the state reduction: wait for its
+  // partials, and let the read-out kernel start its own prologue meanwhile.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  cg::cluster_group cluster = cg::this_cluster();
+
+  const int bh = blockIdx.y;
+  const int rank = (int)cluster.block_rank();
+  const int d = p.d;
+  const long long tph = p.part.tiles_per_head;
+  const int c_lo = part_cta_of(p.part, (long long)bh * tph);
+  const int c_hi = part_cta_of(p.part, (long long)(bh + 1) * tph - 1);
+  const size_t dd = (size_t)d * d;
+  const int chunk = (int)(dd / kCombineCluster);        // 2048 for d = 128
+  const int e_base = rank * chunk;
+
+  // Each thread owns up to two float4 groups of S (e = e_base + 4*tid + 1024*k)
+  // and, for d <= 128, one element e = tid of the z partials this rank adds
+  // (partials rank, rank + 8, ... of each slot).  All loads of a batch of
+  // slots are issued before any is added, then added in slot order.
+  constexpr int kBatch = 4;
+  float4 acc[2];
+  float zacc = 0.f;
+  bool live[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
+    live[k] = e < e_base + chunk;
+    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (live[k] && p.S_in)
+      acc[k] = *reinterpret_cast<const float4*>(p.S_in + bh * dd + row_major(p, e));
+  }
+  const bool zlive = (int)threadIdx.x < d;
+  for (int c0 = c_lo; c0 <= c_hi; c0 += kBatch) {
+    float4 t[kBatch][2];
+    float zt[kBatch][4];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int c = c0 + b;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
+        t[b][k] = (c <= c_hi && live[k])
+                      ? *reinterpret_cast<const float4*>(p.part_S + ((size_t)c + bh) * dd + e)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int zp = rank + kCombineCluster * q;
+        zt[b][q] = (c <= c_hi && zlive && zp < p.zparts)
+                       ? p.part_z[(((size_t)c + bh) * p.zparts + zp) * d + threadIdx.x]
+                       : 0.f;
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      if (c0 + b > c_hi) break;
+      add4(acc[0], t[b][0]);
+      add4(acc[1], t[b][1]);
+      zacc += zt[b][0]; zacc += zt[b][1]; zacc += zt[b][2]; zacc += zt[b][3];
+    }
+  }
+  combine_finish(p, cluster, bh, rank, acc, live, zacc);
+}
+
+// The same combine with every partial of the head brought in at once: one
+// warp issues bulk copies of each slot's slice of S (8 KB) and of the z
+// partials this rank adds into shared memory, all completing on one mbarrier,
+// so the loads take one round trip however many slots the head has.  The
+// sums then run from shared memory in the same order as combine_kernel's, so
+// the two kernels give the same bits.  For the tensor path's chunk-major
+// partials (d = 128) and heads of at most kCombineBulkSlots slots.
+constexpr int kCombineBulkSlots = 20;
+constexpr uint32_t kCombineSliceBytes = 128 * 128 / kCombineCluster * 4;   // 8 KB
+constexpr uint32_t kCombineZBytes = 128 * 4;                                // one z partial
+
+inline size_t combine_bulk_smem(int slots) {
+  return (size_t)slots * (kCombineSliceBytes + 4 * kCombineZBytes);
+}
+
+__global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombineThreads)
+    combine_bulk_kernel(CombineParams p) {
+  namespace cg = cooperative_groups;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(128) unsigned char cb_smem[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+
+  const int bh = blockIdx.y;
+  const int rank = (int)cluster.block_rank();
+  const long long tph = p.part.tiles_per_head;
+  const int c_lo = part_cta_of(p.part, (long long)bh * tph);
+  const int c_hi = part_cta_of(p.part, (long long)(bh + 1) * tph - 1);
+  const int nslots = c_hi - c_lo + 1;
+  const size_t dd = 128 * 128;
+  const int e_base = rank * (int)(dd / kCombineCluster);
+  float* sl = reinterpret_cast<float*>(cb_smem);                       // [slot][2048]
+  float* zs = sl + (size_t)nslots * (kCombineSliceBytes / 4);          // [slot][4][128]
+  int nq = 0;   // z partials this rank adds per slot: rank, rank + 8, ...
+  for (int q = 0; q < 4; ++q)
+    if (rank + kCombineCluster * q < p.zparts) nq = q + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    if (threadIdx.x == 0)
+      mbar_arrive_expect_tx(&bar, (uint32_t)nslots * (kCombineSliceBytes + nq * kCombineZBytes));
+    __syncwarp();
+    for (int i = threadIdx.x; i < nslots; i += 32) {
+      const size_t slot = (size_t)c_lo + i + bh;
+      bulk_load(sl + (size_t)i * (kCombineSliceBytes / 4), p.part_S + slot * dd + e_base,
+                kCombineSliceBytes, &bar);
+      for (int q = 0; q < nq; ++q)
+        bulk_load(zs + ((size_t)i * 4 + q) * 128,
+                  p.part_z + (slot * p.zparts + rank + kCombineCluster * q) * 128,
+                  kCombineZBytes, &bar);
+    }
+  }
+
+  float4 acc[2];
+  const bool live[2] = {true, true};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = e_base + 4 * threadIdx.x + 4 * kCombineThreads * k;
+    acc[k] = p.S_in ? *reinterpret_cast<const float4*>(p.S_in + bh * dd + row_major(p, e))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float zacc = 0.f;
+  if (mbar_wait(&bar, 0u, &abort_flag)) {
+    for (int i = 0; i < nslots; ++i) {
+      const float* si = sl + (size_t)i * (kCombineSliceBytes / 4);
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        add4(acc[k], *reinterpret_cast<const float4*>(si + 4 * threadIdx.x + 4 * kCombineThreads * k));
+      if (threadIdx.x < 128)
+        for (int q = 0; q < nq; ++q) zacc += zs[((size_t)i * 4 + q) * 128 + threadIdx.x];
+    }
+  } else {
+    // Timed out (recorded in the device error word): let the copies land
+    // before this CTA's shared memory is released; the result is void.
+    int dummy = 0;
+    mbar_wait(&bar, 0u, reinterpret_cast<volatile int*>(&dummy));
+  }
+  combine_finish(p, cluster, bh, rank, acc, live, zacc);
 }
 
 }  // namespace gla

@@ -1129,17 +1129,20 @@ inline size_t tc_apply_smem(int tab_entries) {
 }
 constexpr size_t kMaxSmem = 232448;
 
-// Raises a kernel's dynamic shared-memory limit to kMaxSmem once per device
-// (slot: which kernel), instead of on every call: the attribute only bounds
-// what a launch may ask for.
+// Raises a kernel's dynamic shared-memory limit to all that its static shared
+// memory leaves of kMaxSmem, once per device (slot: which kernel), instead of
+// on every call: the attribute only bounds what a launch may ask for.
 template <typename K>
 inline bool ensure_max_smem(K kernel, int slot) {
-  static std::atomic<unsigned char> done[3][64];
+  static std::atomic<unsigned char> done[4][64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (dev >= 0 && dev < 64 && done[slot][dev].load(std::memory_order_acquire)) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem) !=
-      cudaSuccess)
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.sharedSizeBytes > kMaxSmem)
+    return false;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)(kMaxSmem - fa.sharedSizeBytes)) != cudaSuccess)
     return false;
   if (dev >= 0 && dev < 64) done[slot][dev].store(1, std::memory_order_release);
   return true;
@@ -1223,15 +1226,30 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   cp.S_out = write_state ? S : nullptr;
   cp.z_out = z; cp.S_img = S_img; cp.S_scale = S_scale;
   cp.chunked = 1;
+  // Slots of the head with the most: the bulk-copy combine takes every slot
+  // of a head in one round while they fit its shared memory.
+  int max_slots = 0;
+  for (int bh = 0; bh < g.B * g.Hh; ++bh) {
+    const int lo = part_cta_of(spart, (long long)bh * spart.tiles_per_head);
+    const int hi = part_cta_of(spart, (long long)(bh + 1) * spart.tiles_per_head - 1);
+    if (hi - lo + 1 > max_slots) max_slots = hi - lo + 1;
+  }
+  const bool bulk = max_slots <= kCombineBulkSlots;
   cudaLaunchConfig_t cc = {};
   cc.gridDim = dim3(kCombineCluster, g.B * g.Hh);
   cc.blockDim = dim3(kCombineThreads);
-  cc.dynamicSmemBytes = 0;
+  cc.dynamicSmemBytes = bulk ? combine_bulk_smem(max_slots) : 0;
   cc.stream = stream;
   cc.attrs = pdl;
   cc.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cc, combine_kernel, cp) != cudaSuccess || mark(2) != cudaSuccess)
-    return GLA_ERR_CUDA;
+  cudaError_t ce;
+  if (bulk) {
+    if (!ensure_max_smem(combine_bulk_kernel, 3)) return GLA_ERR_CUDA;
+    ce = cudaLaunchKernelEx(&cc, combine_bulk_kernel, cp);
+  } else {
+    ce = cudaLaunchKernelEx(&cc, combine_kernel, cp);
+  }
+  if (ce != cudaSuccess || mark(2) != cudaSuccess) return GLA_ERR_CUDA;
 
   TcApplyParams ap = {};
   ap.g = g; ap.part = part; ap.S_img = S_img; ap.S_scale = S_scale; ap.z = z;
