@@ -7,8 +7,11 @@
 // for a block-causal step), so the result does not depend on scheduling.
 //
 // One cluster of kCombineCluster CTAs handles one head; each CTA sums a slice
-// of S.  For the tensor read-out the kernel also writes the fp16 image of S
-// that the read-out copies into shared memory as its B operand: two K-blocks
+// of S.  combine_bulk_kernel brings all of its slices in at once by bulk
+// copies (tensor path, heads of up to kCombineBulkSlots slots);
+// combine_kernel loads them into registers a few slots per round.  Both add
+// in the order above.  For the tensor read-out they also write the fp16 image
+// of S that the read-out copies into shared memory as its B operand: two K-blocks
 // of [128 rows][64 columns], rows of 128 bytes, 16-byte chunks XOR-swizzled by
 // (row & 7) -- the canonical K-major 128-byte-swizzle layout of tcgen05.  The
 // image is S * 2^e with one power of two per head, chosen from the head's
