@@ -64,7 +64,10 @@
  *
  * Memory: the library allocates no device memory.  Scratch space is the
  * caller's `workspace` of at least *_workspace_size() bytes, 256-byte
- * aligned; its contents need no initialisation and are overwritten.
+ * aligned; its contents need no initialisation and are overwritten.  The
+ * only resources it creates itself are, per device and on first use by
+ * gla_forward_host with batch >= 2, one non-blocking stream and nine events,
+ * kept until the process exits.
  */
 #ifndef GLA_H
 #define GLA_H
