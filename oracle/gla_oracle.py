@@ -303,6 +303,54 @@ def causal_bruteforce(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
                               visible=lambda j, n: n <= j)
 
 
+# ------------------------------------------------- MXFP8 operator inputs
+
+# The MX block formats (OCP Microscaling): elements in FP8 E4M3, one shared
+# E8M0 power-of-two scale per MX_BLOCK consecutive elements along the
+# innermost axis (the head dim here).  Reading for the FP8-input row: q, k, v
+# and g arrive in this format, beta stays in its own dtype, and the operator
+# is the one above applied to the decoded values.
+
+MX_BLOCK = 32
+
+
+def e4m3_decode(codes):
+    """FP8 E4M3 without infinities: sign bit, 4 exponent bits (bias 7), 3
+    mantissa bits; exponent field 0 holds the subnormals m/8 * 2^-6, and
+    S.1111.111 is NaN (the largest finite value is 1.75 * 2^8 = 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    out = sign * mag
+    out[(e == 15) & (c & 0x7 == 7)] = np.nan
+    return out
+
+
+def e8m0_decode(codes):
+    """E8M0 scale: 2^(code - 127); code 255 is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.float64)
+    out = np.exp2(c - 127.0)
+    out[c == 255] = np.nan
+    return out
+
+
+def mx_dequantize(codes, scales):
+    """Element i of a row is e4m3(codes[..., i]) * e8m0(scales[..., i // MX_BLOCK])."""
+    x = e4m3_decode(codes)
+    sc = e8m0_decode(scales)
+    assert sc.shape[-1] * MX_BLOCK == x.shape[-1]
+    return x * np.repeat(sc, MX_BLOCK, axis=-1)
+
+
+def forward_mx(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
+    """The bidirectional operator on MX inputs: q, k, v and g are (codes,
+    scales) pairs, beta a float array."""
+    dq = lambda pair: mx_dequantize(*pair)
+    return forward(dq(q), dq(k), dq(v), beta, dq(g), T, H, W, rope_theta, eps, t0)
+
+
 # ------------------------------------------------------------- parity metric
 
 def max_err_over_rms(got, ref):

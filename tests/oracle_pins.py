@@ -361,4 +361,69 @@ def check_causal_time_shift_invariance():
     _close(a["out"], b["out"], 1e-10, "causal time shift")
 
 
+# ---------------------------------------------------- MXFP8 input decoding
+
+def check_e4m3_format_values():
+    """Values the OCP FP8 E4M3 definition fixes: 1.0, -2.0, the largest
+    finite 448, the smallest normal 2^-6, the largest subnormal 7/8 * 2^-6,
+    the smallest subnormal 2^-9, signed zeros and the NaN codes."""
+    want = {0x38: 1.0, 0xC0: -2.0, 0x7E: 448.0, 0xFE: -448.0, 0x08: 2.0 ** -6,
+            0x07: 0.875 * 2.0 ** -6, 0x01: 2.0 ** -9, 0x00: 0.0, 0x3C: 1.5, 0x44: 3.0}
+    got = O.e4m3_decode(np.array(list(want), dtype=np.uint8))
+    _close(got, list(want.values()), 0.0, "e4m3 values")
+    assert np.signbit(O.e4m3_decode(np.array([0x80], dtype=np.uint8)))[0], "0x80 is -0"
+    assert np.isnan(O.e4m3_decode(np.array([0x7F, 0xFF], dtype=np.uint8))).all(), "NaN codes"
+
+
+def check_e4m3_matches_library():
+    """All 256 codes against torch's float8_e4m3fn conversion."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(lib)), "e4m3 NaN codes differ"
+    ok = ~np.isnan(lib)
+    assert np.array_equal(got[ok], lib[ok]), "e4m3 decode differs from torch"
+
+
+def check_e8m0_matches_library():
+    """All 256 scale codes against torch's float8_e8m0fnu conversion."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(codes).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    got = O.e8m0_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(lib)), "e8m0 NaN codes differ"
+    ok = ~np.isnan(lib)
+    assert np.array_equal(got[ok], lib[ok]), "e8m0 decode differs from torch"
+
+
+def check_mx_block_layout():
+    """A 64-element row with scales 2^1 and 2^-3: elements 0..31 take the
+    first, 32..63 the second."""
+    codes = np.full((1, 64), 0x38, dtype=np.uint8)          # every element 1.0
+    scales = np.array([[128, 124]], dtype=np.uint8)         # 2^1, 2^-3
+    got = O.mx_dequantize(codes, scales)
+    _close(got[0, :32], [2.0] * 32, 0.0, "first block")
+    _close(got[0, 32:], [0.125] * 32, 0.0, "second block")
+
+
+def check_mx_forward_row_scale_invariance():
+    """Scaling every block scale of a q (or k) row by the same power of two
+    leaves the output unchanged up to the RMSNorm epsilon: the operator sees
+    q and k only through their RMS-normalised values."""
+    rng = np.random.default_rng(57)
+    T, H, W, d = 2, 2, 3, 64
+    N = T * H * W
+    codes = {n: rng.integers(0, 0x77, (1, N, 2, d)).astype(np.uint8) |
+             (rng.integers(0, 2, (1, N, 2, d)).astype(np.uint8) << 7) for n in "qkvg"}
+    scales = {n: rng.integers(120, 130, (1, N, 2, d // O.MX_BLOCK)).astype(np.uint8) for n in "qkv"}
+    scales["g"] = rng.integers(118, 122, (1, N, 2, d // O.MX_BLOCK)).astype(np.uint8)   # |g| < 15
+    beta = rng.uniform(0.0, 1.0, (1, N, 2))
+    args = lambda sc: [(codes[n], sc[n]) for n in "qkv"]
+    a = O.forward_mx(*args(scales), beta, (codes["g"], scales["g"]), T, H, W, 1e4, 1e-5)
+    shifted = dict(scales, q=scales["q"] + 3, k=scales["k"] - 2)
+    b = O.forward_mx(*args(shifted), beta, (codes["g"], scales["g"]), T, H, W, 1e4, 1e-5)
+    _close(b["out"], a["out"], 1e-5, "row scale invariance")
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

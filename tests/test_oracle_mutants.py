@@ -113,6 +113,29 @@ def _causal_suffix(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
     return {key: flip(val) for key, val in r.items()}
 
 
+def _e4m3_bias8(codes):
+    return _orig["e4m3_decode"](codes) / 2.0
+
+
+def _e4m3_no_subnormals(codes):
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    out = _orig["e4m3_decode"](codes)
+    sub = ((c >> 3) & 0xF) == 0
+    m = (c & 0x7).astype(np.float64)
+    out[sub] = np.where(c[sub] & 0x80, -1.0, 1.0) * (1.0 + m[sub] / 8.0) * 2.0 ** -7
+    return out
+
+
+def _e8m0_bias128(codes):
+    return _orig["e8m0_decode"](codes) / 2.0
+
+
+def _mx_scales_tiled(codes, scales):
+    x = O.e4m3_decode(codes)
+    sc = O.e8m0_decode(scales)
+    return x * np.tile(sc, (1,) * (sc.ndim - 1) + (O.MX_BLOCK,))
+
+
 MUTANTS = {
     "rope_backwards": ("rope_rotate", _rotate_backwards),
     "rope_before_relu": ("feature_maps", _rope_before_relu),
@@ -131,6 +154,10 @@ MUTANTS = {
     "sigmoid_sign": ("sigmoid", _neg_sigmoid),
     "causal_exclusive": ("causal_forward", _causal_exclusive),
     "causal_suffix": ("causal_forward", _causal_suffix),
+    "e4m3_bias8": ("e4m3_decode", _e4m3_bias8),
+    "e4m3_no_subnormals": ("e4m3_decode", _e4m3_no_subnormals),
+    "e8m0_bias128": ("e8m0_decode", _e8m0_bias128),
+    "mx_scales_tiled": ("mx_dequantize", _mx_scales_tiled),
 }
 
 
