@@ -426,4 +426,66 @@ def check_mx_forward_row_scale_invariance():
     _close(b["out"], a["out"], 1e-5, "row scale invariance")
 
 
+# ------------------------------------------------------ tolerance metrics
+#
+# Every GPU pass/fail goes through these four functions, so each is pinned to
+# values worked out by hand (and the bf16 spacing to torch's bf16 rounding):
+# a slip in one of them (the RMS of the wrong array, a lost abs, a wrong
+# exponent) would otherwise loosen every parity test without anything failing.
+
+def _metrics():
+    import gpu_common
+    return gpu_common
+
+
+_REF4 = np.array([3.0, -4.0, 0.0, 0.0])        # rms = sqrt((9 + 16) / 4) = 2.5
+
+
+def check_metric_max_err_over_rms():
+    """max|got - ref| / rms(ref): errors (0.1, 0, 0, -0.3) give 0.3 / 2.5."""
+    got = _REF4 + np.array([0.1, 0.0, 0.0, -0.3])
+    _close(O.max_err_over_rms(got, _REF4), 0.12, 1e-12, "max_err_over_rms")
+    _close(O.max_err_over_rms(_REF4 + np.array([0.0, 0.5, 0.0, 0.0]), _REF4), 0.2, 1e-12,
+           "max_err_over_rms, one error")
+    assert O.max_err_over_rms(_REF4, _REF4) == 0.0
+
+
+def check_metric_rel_rms_floor():
+    """max |got - ref| / max(|ref|, rms(ref)) with rms(ref) = 2.5:
+    errors (0.6, -1.0, 0.3, -0.8) give 0.6/3, 1.0/4, 0.3/2.5, 0.8/2.5, max 0.32;
+    a single error -2 on the 4 gives 2/4 (relative above the RMS)."""
+    got = _REF4 + np.array([0.6, -1.0, 0.3, -0.8])
+    _close(O.max_rel_err_rms_floor(got, _REF4), 0.32, 1e-12, "rel err with RMS floor")
+    got = _REF4 + np.array([0.0, -2.0, 0.0, 0.0])
+    _close(O.max_rel_err_rms_floor(got, _REF4), 0.5, 1e-12, "rel err above the RMS")
+
+
+def check_metric_bf16_half_ulp():
+    """Half the bf16 spacing (8 significant bits) at hand-picked values, then
+    against torch's round-to-nearest-even bf16 conversion: a value halfway
+    between two bf16 neighbours is exactly half a spacing from its rounding."""
+    import torch
+    gc = _metrics()
+    vals = np.array([1.0, 1.99, 4.0, 7.99, 0.75, -3.0, 2.0 ** 20])
+    want = np.array([2.0 ** -8, 2.0 ** -8, 2.0 ** -6, 2.0 ** -6, 2.0 ** -9, 2.0 ** -7, 2.0 ** 12])
+    _close(gc.bf16_half_ulp(vals), want, 0.0, "bf16 half ulp")
+    rng = np.random.default_rng(5)
+    e = rng.integers(-60, 60, 400)
+    m = rng.integers(0, 128, 400)
+    x = np.ldexp(1.0 + (2 * m + 1) / 256.0, e) * np.where(rng.random(400) < 0.5, -1.0, 1.0)
+    rounded = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    _close(np.abs(rounded - x), gc.bf16_half_ulp(x), 0.0, "midpoints vs torch bf16")
+
+
+def check_metric_rel_rms_bf16out():
+    """Error beyond half a bf16 spacing, over rms(ref) = 2.5.  Half spacings:
+    2^-7 at 3, 2^-6 at 4.  Errors (2^-7, -0.025, 0, 0) exceed them by
+    (0, 0.025 - 2^-6, 0, 0): 0.009375 / 2.5 = 0.00375."""
+    gc = _metrics()
+    got = _REF4 + np.array([2.0 ** -7, -0.025, 0.0, 0.0])
+    _close(gc.rel_rms_bf16out(got, _REF4), 0.00375, 1e-9, "bf16 output metric")
+    got = _REF4 + np.array([2.0 ** -7, -2.0 ** -6, 0.0, 0.0])
+    assert gc.rel_rms_bf16out(got, _REF4) == 0.0, "a correct rounding scores 0"
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

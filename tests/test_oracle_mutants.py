@@ -3,6 +3,7 @@ pins catch every one of them: each mutant must fail at least one check."""
 import numpy as np
 import pytest
 
+import gpu_common
 import oracle.gla_oracle as O
 import oracle_pins
 
@@ -172,3 +173,100 @@ def test_mutant_is_caught(name, monkeypatch):
         except (AssertionError, FloatingPointError, ValueError):
             failed.append(check.__name__)
     assert failed, f"mutant {name} passed every pin"
+
+
+# Mistakes in the tolerance metrics (the oracle's and the GPU tests' helpers).
+
+def _rms_of_got(got, ref):
+    return _orig["max_err_over_rms"](ref, got)
+
+
+def _err_no_abs(got, ref):
+    ref = np.asarray(ref, dtype=np.float64)
+    got = np.asarray(got, dtype=np.float64)
+    return float(np.max(got - ref) / np.sqrt(np.mean(ref * ref)))
+
+
+def _err_mean_abs(got, ref):
+    ref = np.asarray(ref, dtype=np.float64)
+    got = np.asarray(got, dtype=np.float64)
+    return float(np.max(np.abs(got - ref)) / np.mean(np.abs(ref)))
+
+
+def _floor_no_abs(got, ref):
+    ref = np.asarray(ref, dtype=np.float64)
+    got = np.asarray(got, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref * ref))
+    return float(np.max((got - ref) / np.maximum(np.abs(ref), rms)))
+
+
+def _floor_rms_of_got(got, ref):
+    ref = np.asarray(ref, dtype=np.float64)
+    got = np.asarray(got, dtype=np.float64)
+    rms = np.sqrt(np.mean(got * got))
+    return float(np.max(np.abs(got - ref) / np.maximum(np.abs(ref), rms)))
+
+
+def _floor_rms_only(got, ref):
+    ref = np.asarray(ref, dtype=np.float64)
+    got = np.asarray(got, dtype=np.float64)
+    return float(np.max(np.abs(got - ref)) / np.sqrt(np.mean(ref * ref)))
+
+
+_orig_gc = {name: getattr(gpu_common, name) for name in ("bf16_half_ulp", "rel_rms_bf16out")}
+
+
+def _half_ulp_exp7(ref):
+    a = np.maximum(np.abs(np.asarray(ref, dtype=np.float64)), 2.0 ** -126)
+    return np.ldexp(1.0, (np.floor(np.log2(a)) - 7).astype(int))
+
+
+def _half_ulp_ceil(ref):
+    a = np.maximum(np.abs(np.asarray(ref, dtype=np.float64)), 2.0 ** -126)
+    return np.ldexp(1.0, (np.ceil(np.log2(a)) - 8).astype(int))
+
+
+def _bf16out_no_rounding_allowance(got, ref):
+    return _orig["max_err_over_rms"](got, ref)
+
+
+def _bf16out_rms_of_got(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    excess = np.maximum(np.abs(got - ref) - _orig_gc["bf16_half_ulp"](ref), 0.0)
+    return float(np.max(excess) / np.sqrt(np.mean(got * got)))
+
+
+def _bf16out_full_ulp(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    excess = np.maximum(np.abs(got - ref) - 2.0 * _orig_gc["bf16_half_ulp"](ref), 0.0)
+    return float(np.max(excess) / np.sqrt(np.mean(ref * ref)))
+
+
+METRIC_MUTANTS = {
+    "err_rms_of_got": (O, "max_err_over_rms", _rms_of_got),
+    "err_no_abs": (O, "max_err_over_rms", _err_no_abs),
+    "err_mean_abs": (O, "max_err_over_rms", _err_mean_abs),
+    "floor_no_abs": (O, "max_rel_err_rms_floor", _floor_no_abs),
+    "floor_rms_of_got": (O, "max_rel_err_rms_floor", _floor_rms_of_got),
+    "floor_missing": (O, "max_rel_err_rms_floor", _floor_rms_only),
+    "half_ulp_exp7": (gpu_common, "bf16_half_ulp", _half_ulp_exp7),
+    "half_ulp_ceil": (gpu_common, "bf16_half_ulp", _half_ulp_ceil),
+    "bf16out_no_allowance": (gpu_common, "rel_rms_bf16out", _bf16out_no_rounding_allowance),
+    "bf16out_rms_of_got": (gpu_common, "rel_rms_bf16out", _bf16out_rms_of_got),
+    "bf16out_full_ulp": (gpu_common, "rel_rms_bf16out", _bf16out_full_ulp),
+}
+
+
+@pytest.mark.parametrize("name", sorted(METRIC_MUTANTS))
+def test_metric_mutant_is_caught(name, monkeypatch):
+    mod, attr, fn = METRIC_MUTANTS[name]
+    monkeypatch.setattr(mod, attr, fn)
+    failed = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check()
+        except (AssertionError, FloatingPointError, ValueError):
+            failed.append(check.__name__)
+    assert failed, f"metric mutant {name} passed every pin"
