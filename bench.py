@@ -34,7 +34,7 @@ from gated_bidirectional_linear_b200 import replicas, workloads  # noqa: E402
 
 METRIC = "gla_forward tokens/s (20x128 heads, 14720 tok) and HBM GB/s vs B200 peak"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["common.cuh", "ptx.cuh", "tc.cuh", "combine.cuh"]
+CSRC = os.path.join(ROOT, "gated_bidirectional_linear_b200", "csrc")
 
 
 def parse():
@@ -48,6 +48,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="only run warmup + steps of gla_forward (for ncu captures)")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="timed regions of --steps steps each; the median is reported")
+    ap.add_argument("--ingest-ncu", metavar="CSV",
+                    help="write profiles/traffic.json entries for --workload from an "
+                         "`ncu -i <report> --page raw --csv` export, then exit")
     return ap.parse_args()
 
 
@@ -64,6 +69,34 @@ def workload_config(wl):
     }
 
 
+def host_info():
+    """The host the CPU baseline ran on: logical CPUs, those this process may
+    use, and the CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count()
+    return {"nproc": os.cpu_count(), "usable_cpus": usable, "cpu_model": model}
+
+
+def timed_repeats(run, stream, dist, sync, dev, repeats):
+    """`repeats` timed regions of the same K steps (each bracketed by a
+    barrier and a device synchronisation, max over ranks); returns the median
+    region time and all of them, in ms."""
+    reps = [replicas.timed(run, replicas.CudaTimer(stream), dist, sync, dev)
+            for _ in range(max(1, repeats))]
+    return float(np.median(reps)), reps
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -74,11 +107,61 @@ def measured_peaks():
 
 
 def source_sha():
+    """Hash of every kernel source file: a traffic record is valid only for
+    the code it was captured on."""
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "gated_bidirectional_linear_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
+
+
+_BYTE_UNITS = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}
+_TIME_UNITS = {"ns": 1e-3, "us": 1.0, "usecond": 1.0, "msecond": 1e3, "ms": 1e3, "nsecond": 1e-3}
+
+
+def ingest_ncu(csv_path, workload):
+    """Per kernel of an ncu raw-page CSV export: the mean over its captured
+    launches of dram__bytes_read.sum + dram__bytes_write.sum (bytes per
+    launch) and of gpu__time_duration.sum, written to profiles/traffic.json
+    under (kernel, workload) with the hash of the current kernel sources."""
+    import csv
+    with open(csv_path, newline="") as f:
+        rows = [r for r in csv.reader(f)]
+    head = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    cols, units, data = rows[head], rows[head + 1], rows[head + 2:]
+    ix = {name: cols.index(name) for name in
+          ("Kernel Name", "dram__bytes_read.sum", "dram__bytes_write.sum",
+           "gpu__time_duration.sum")}
+    per = {}
+    for r in data:
+        if len(r) != len(cols):
+            continue
+        name = r[ix["Kernel Name"]].split("(")[0].split()[-1].split("<")[0]
+        byt = sum(float(r[ix[m]]) * _BYTE_UNITS[units[ix[m]]]
+                  for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"))
+        dur = float(r[ix["gpu__time_duration.sum"]]) * _TIME_UNITS[units[ix["gpu__time_duration.sum"]]]
+        per.setdefault(name, []).append((byt, dur))
+    try:
+        with open(TRAFFIC_FILE) as f:
+            doc = json.load(f)
+    except (OSError, ValueError):
+        doc = {}
+    doc["_note"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, mean over the "
+                    "captured launches, written by `python bench.py --ingest-ncu <csv> "
+                    "--workload <w>` from an `ncu -i <report> --page raw --csv` export; valid "
+                    "only while the kernel sources hash to source_sha")
+    sha = source_sha()
+    for name, v in sorted(per.items()):
+        doc.setdefault(name, {})[workload] = {
+            "bytes_per_launch": int(round(float(np.mean([b for b, _ in v])))),
+            "duration_us_under_ncu": round(float(np.mean([t for _, t in v])), 2),
+            "launches": len(v), "source_sha": sha, "capture": os.path.basename(csv_path)}
+        print(f"{name} [{workload}]: {doc[name][workload]}")
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(doc, f, indent=1, sort_keys=True)
+        f.write("\n")
 
 
 def traffic_for(kernel, workload):
@@ -202,7 +285,7 @@ def run_reference(args, wl, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(wl),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host": host_info()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -212,6 +295,9 @@ def run_reference(args, wl, rank):
 def main():
     args = parse()
     wl = workloads.WORKLOADS[args.workload]
+    if args.ingest_ncu:
+        ingest_ncu(args.ingest_ncu, wl.name)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -277,7 +363,7 @@ def main():
             plain_step()
 
     with ClockMonitor(local) as mon:
-        elapsed_ms = replicas.timed(timed_steps, replicas.CudaTimer(stream), dist, sync, dev)
+        elapsed_ms, reps = timed_repeats(timed_steps, stream, dist, sync, dev, args.repeats)
     status = gla.gla_get_device_status(stream)
     if status != gla.GLA_OK:
         raise RuntimeError(f"device status after the timed region: {gla.status_string(status)}")
@@ -341,11 +427,14 @@ def main():
                    "sample": (f"oracle.forward on {heads} whole heads ({wl.tokens} tokens each) "
                               f"of the {wl.name} workload, {secs:.1f} s; tokens/s of the full "
                               f"layer = token-heads/s / {wl.heads}; cores = BLAS threads"),
+                   "host": host_info(),
                    "single_core": {"value": rate1, "unit": "tokens/s", "cores": 1,
                                    "sample": f"{heads1} whole heads, {secs1:.1f} s, one BLAS thread"}}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "repeats": len(reps),
+            "repeat_ms_per_step": [round(r / args.steps, 5) for r in reps],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": dict(workload_config(wl), parallelism=f"replicas x{world}"),
@@ -415,22 +504,25 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
             sequence()
 
     with ClockMonitor(local) as mon:
-        ms = replicas.timed(timed_sequences, replicas.CudaTimer(stream), dist, sync, dev)
+        ms, reps = timed_repeats(timed_sequences, stream, dist, sync, dev, args.repeats)
     if gla.gla_get_device_status(stream) != gla.GLA_OK:
         raise RuntimeError("device status after the timed region")
 
-    # End to end: the sequence's inputs from pinned host memory, the steps,
-    # and the outputs back, every step.
+    # End to end through the library's host entry: every block's inputs from
+    # pinned host memory into the device arena, the step on the device-resident
+    # state, and the block's output back to pinned host memory.
     pinned = [{k: v.cpu().pin_memory() for k, v in b.items()} for b in blocks]
     outs_h = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    arena = gla.alloc_workspace(
+        gla.gla_block_causal_host_arena_size(B, Hh, hd, wl.T, wl.H, wl.W, code), dev)
 
     def sequence_host():
-        for b, bp in zip(blocks, pinned):
-            for k in b:
-                b[k].copy_(bp[k], non_blocking=True)
-        sequence()
-        for o, oh in zip(outs, outs_h):
-            oh.copy_(o, non_blocking=True)
+        S.zero_()
+        z.zero_()
+        for i, bp in enumerate(pinned):
+            gla.gla_block_causal_step_host(S, z, bp["q"], bp["k"], bp["v"], bp["beta"], bp["g"],
+                                           wl.T, wl.H, wl.W, i * wl.T, wl.rope_theta, wl.eps,
+                                           out=outs_h[i], arena=arena, stream=stream)
 
     e2e_steps = max(3, min(steps, 50))
     sequence_host()
@@ -470,12 +562,14 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
                    "sample": (f"oracle.block_causal_forward on {heads} of the {B * Hh} heads of "
                               f"the {wl.name} sequence ({wl.n_blocks} blocks each), {secs:.1f} s; "
                               f"tokens/s of the full layer = token-heads/s / {wl.heads}; "
-                              f"cores = BLAS threads")}
+                              f"cores = BLAS threads"),
+                   "host": host_info()}
         line = {
             "metric": "gla_block_causal_step tokens/s (20x128 heads, 20 blocks of 3x23x40)",
             "value": replicas.aggregate_rate(world, tokens, steps, ms), "unit": "tokens/s",
             "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "repeats": len(reps), "repeat_ms_per_step": [round(r / steps, 5) for r in reps],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": dict(workload_config(wl), blocks=wl.n_blocks,

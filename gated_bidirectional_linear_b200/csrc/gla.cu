@@ -551,6 +551,55 @@ gla_status gla_forward_host(const void* q_h, const void* k_h, const void* v_h,
   return st;
 }
 
+size_t gla_block_causal_host_arena_size(int batch, int heads, int head_dim, int T_blk, int H,
+                                        int W, int dtype) {
+  const size_t ws = gla_block_causal_workspace_size(batch, heads, head_dim, T_blk, H, W, dtype);
+  if (!ws) return 0;
+  const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
+  const size_t th = (size_t)batch * T_blk * H * W * heads;
+  return 5 * align_up(th * head_dim * esz, kAlign) + align_up(th * esz, kAlign) + ws;
+}
+
+gla_status gla_block_causal_step_host(float* state, float* z, const void* q_h, const void* k_h,
+                                      const void* v_h, const void* beta_h, const void* g_h,
+                                      int batch, int heads, int head_dim, int T_blk, int H,
+                                      int W, int t0, float rope_theta, float eps, int dtype,
+                                      void* out_h, void* arena, size_t arena_bytes,
+                                      void* stream) {
+  const size_t need =
+      gla_block_causal_host_arena_size(batch, heads, head_dim, T_blk, H, W, dtype);
+  if (!need) return GLA_ERR_INVALID_ARG;
+  const void* hp[6] = {q_h, k_h, v_h, beta_h, g_h, out_h};
+  for (const void* p : hp)
+    if (!p) return GLA_ERR_INVALID_ARG;
+  if (!arena || ((uintptr_t)arena % kAlign) != 0 || arena_bytes < need) return GLA_ERR_WORKSPACE;
+  const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
+  const size_t th = (size_t)batch * T_blk * H * W * heads;
+  const size_t big = th * head_dim * esz, small = th * esz;
+  unsigned char* a = static_cast<unsigned char*>(arena);
+  unsigned char* dq = a;
+  unsigned char* dk = dq + align_up(big, kAlign);
+  unsigned char* dv = dk + align_up(big, kAlign);
+  unsigned char* dg = dv + align_up(big, kAlign);
+  unsigned char* dout = dg + align_up(big, kAlign);
+  unsigned char* dbeta = dout + align_up(big, kAlign);
+  unsigned char* dws = dbeta + align_up(small, kAlign);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(dq, q_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dg, g_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dbeta, beta_h, small, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  const gla_status st = gla_block_causal_step(
+      state, z, dq, dk, dv, dbeta, dg, batch, heads, head_dim, T_blk, H, W, t0, rope_theta, eps,
+      dtype, dout, dws, arena_bytes - (size_t)(dws - a), stream);
+  if (st != GLA_OK) return st;
+  if (cudaMemcpyAsync(out_h, dout, big, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  return GLA_OK;
+}
+
 // ---------------------------------------------------------------------------
 // Allocation-free entry point.  The scratch lives in a file-scope device array;
 // host code only ever uses its device address, looked up once per device.
@@ -562,10 +611,14 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GLA_NOALLOC_SCRATCH_BYTES];
 
 // Device address of g_noalloc_scratch on the current device (0 on failure).
+// The per-device cache is filled under a mutex: host threads that make their
+// first call at the same time look the address up once.
 unsigned char* noalloc_scratch() {
+  static std::mutex mu;
   static unsigned char* addr[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
   if (!addr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
@@ -575,8 +628,10 @@ unsigned char* noalloc_scratch() {
 }
 
 // Scratch layout sized for the grid this GPU actually runs (at most `grid`
-// state CTAs, `zparts` z partials per slot) rather than the worst case.
-WsLayout noalloc_layout(int BH, int d, int grid, int zparts, int T, int H, int W) {
+// state CTAs, `zparts` z partials per slot) rather than the worst case.  The
+// fp16 image of S, its scale and the whole-call RoPE table are read by the
+// tensor read-out only, so the CUDA-core path reserves no room for them.
+WsLayout noalloc_layout(int BH, int d, int grid, int zparts, int T, int H, int W, bool tensor) {
   WsLayout L;
   L.slots = grid + BH;
   size_t off = 0;
@@ -585,11 +640,11 @@ WsLayout noalloc_layout(int BH, int d, int grid, int zparts, int T, int H, int W
   L.S = off; off = align_up(off + (size_t)BH * d * d * 4, kAlign);
   L.z = off; off = align_up(off + (size_t)BH * d * 4, kAlign);
   L.S_img = off;
-  if (d == 128) off = align_up(off + (size_t)BH * d * d * 2, kAlign);
+  if (tensor) off = align_up(off + (size_t)BH * d * d * 2, kAlign);
   L.S_scale = off;
-  if (d == 128) off = align_up(off + (size_t)BH * 4 * 4, kAlign);
+  if (tensor) off = align_up(off + (size_t)BH * 4 * 4, kAlign);
   L.rope_tab = off;
-  if (d == 128) off = align_up(off + rope_tab_bytes(d, T, H, W), kAlign);
+  if (tensor) off = align_up(off + rope_tab_bytes(d, T, H, W), kAlign);
   L.total = off;
   return L;
 }
@@ -617,7 +672,8 @@ gla_status gla_forward_noalloc(const void* q, const void* k, const void* v, cons
   const bool tensor = c.path == GLA_PATH_TENSOR;
   const Partition part = tensor ? tc_state_partition(c.g, sms)
                                 : make_partition(batch * heads, c.g.N, kSimtTile, 2 * sms);
-  const WsLayout L = noalloc_layout(batch * heads, head_dim, part.grid, tensor ? kStTW : 1, T, H, W);
+  const WsLayout L =
+      noalloc_layout(batch * heads, head_dim, part.grid, tensor ? kStTW : 1, T, H, W, tensor);
   if (L.total > GLA_NOALLOC_SCRATCH_BYTES) return GLA_ERR_WORKSPACE;
   unsigned char* scratch = noalloc_scratch();
   if (!scratch) return GLA_ERR_CUDA;

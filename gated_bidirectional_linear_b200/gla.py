@@ -38,6 +38,8 @@ _SIGS = {
     "gla_block_causal_step_ex": (_i, [_vp] * 7 + [_i] * 7
                                  + [_f, _f, _i, _vp, _vp, _sz, _vp, _i]),
     "gla_forward_host": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
+    "gla_block_causal_host_arena_size": (_sz, [_i] * 7),
+    "gla_block_causal_step_host": (_i, [_vp] * 7 + [_i] * 7 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
     "gla_forward_noalloc": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp]),
     "gla_get_device_status": (_i, [_vp]),
     "gla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
@@ -91,10 +93,22 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _stream(stream, dev=None):
+    """The cudaStream_t of `stream` (default: the current stream of `dev`).
+    The library launches on the current device, so a stream of another
+    device than the tensors' is refused here."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
+    elif dev is not None and stream.device != dev:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {dev}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on(dev):
+    """Make `dev` the current device for one library call: the C side looks
+    up the SM count, the built-in scratch and its helper stream on the
+    current device, and launches there."""
+    return torch.cuda.device(dev)
 
 
 def _dims(q, T, H, W):
@@ -167,9 +181,10 @@ def gla_forward(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, out=Non
     if workspace is None:
         workspace = alloc_workspace(gla_forward_workspace_size(B, Hh, d, T, H, W, code), q.device)
     _check_workspace(workspace, q.device)
-    st = lib().gla_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T, H,
-                              W, rope_theta, eps, code, _ptr(out), _ptr(workspace),
-                              workspace.numel(), _stream(stream), path)
+    with _on(q.device):
+        st = lib().gla_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
+                                  H, W, rope_theta, eps, code, _ptr(out), _ptr(workspace),
+                                  workspace.numel(), _stream(stream, q.device), path)
     _check(st, "gla_forward")
     return out
 
@@ -189,9 +204,11 @@ def gla_forward_timed(q, k, v, beta, g, T, H, W, events, rope_theta=10000.0, eps
     _check_workspace(workspace, q.device)
     ev = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) if e is not None else None
                                  for e in events])
-    st = lib().gla_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
-                                 H, W, rope_theta, eps, code, _ptr(out), _ptr(workspace),
-                                 workspace.numel(), _stream(stream), path, ev)
+    with _on(q.device):
+        st = lib().gla_forward_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d,
+                                     T, H, W, rope_theta, eps, code, _ptr(out),
+                                     _ptr(workspace), workspace.numel(),
+                                     _stream(stream, q.device), path, ev)
     _check(st, "gla_forward_timed")
     return out
 
@@ -210,9 +227,11 @@ def gla_forward_debug(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6,
     den = torch.empty(B, N, Hh, dtype=torch.float32, device=dev)
     x = torch.empty(B, N, Hh, d, dtype=torch.float32, device=dev)
     ws = alloc_workspace(gla_forward_workspace_size(B, Hh, d, T, H, W, code), dev)
-    st = lib().gla_forward_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
-                                 H, W, rope_theta, eps, code, _ptr(out), _ptr(ws), ws.numel(),
-                                 _stream(stream), path, _ptr(S), _ptr(z), _ptr(den), _ptr(x))
+    with _on(dev):
+        st = lib().gla_forward_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d,
+                                     T, H, W, rope_theta, eps, code, _ptr(out), _ptr(ws),
+                                     ws.numel(), _stream(stream, dev), path, _ptr(S), _ptr(z),
+                                     _ptr(den), _ptr(x))
     _check(st, "gla_forward_debug")
     return dict(out=out, S=S, z=z, den=den, x=x)
 
@@ -233,10 +252,11 @@ def gla_block_causal_step(state, z, q, k, v, beta, g, T_blk, H, W, t0, rope_thet
         workspace = alloc_workspace(
             gla_block_causal_workspace_size(B, Hh, d, T_blk, H, W, code), q.device)
     _check_workspace(workspace, q.device)
-    st = lib().gla_block_causal_step_ex(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v),
-                                        _ptr(beta), _ptr(g), B, Hh, d, T_blk, H, W, t0,
-                                        rope_theta, eps, code, _ptr(out), _ptr(workspace),
-                                        workspace.numel(), _stream(stream), path)
+    with _on(q.device):
+        st = lib().gla_block_causal_step_ex(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(beta), _ptr(g), B, Hh, d, T_blk, H, W, t0,
+                                            rope_theta, eps, code, _ptr(out), _ptr(workspace),
+                                            workspace.numel(), _stream(stream, q.device), path)
     _check(st, "gla_block_causal_step")
     return out
 
@@ -255,10 +275,46 @@ def gla_forward_host(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, ou
         arena = alloc_workspace(gla_forward_host_arena_size(B, Hh, d, T, H, W, code))
     if arena.device.type != "cuda" or arena.dtype != torch.uint8 or not arena.is_contiguous():
         raise ValueError("arena must be a contiguous uint8 tensor on the GPU")
-    st = lib().gla_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
-                                H, W, rope_theta, eps, code, _ptr(out), _ptr(arena),
-                                arena.numel(), _stream(stream))
+    with _on(arena.device):
+        st = lib().gla_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d,
+                                    T, H, W, rope_theta, eps, code, _ptr(out), _ptr(arena),
+                                    arena.numel(), _stream(stream, arena.device))
     _check(st, "gla_forward_host")
+    return out
+
+
+def gla_block_causal_host_arena_size(batch, heads, head_dim, T_blk, H, W, dtype):
+    return lib().gla_block_causal_host_arena_size(batch, heads, head_dim, T_blk, H, W, dtype)
+
+
+def gla_block_causal_step_host(state, z, q, k, v, beta, g, T_blk, H, W, t0, rope_theta=10000.0,
+                               eps=1e-6, out=None, arena=None, stream=None):
+    """One block-causal step on host tensors (pin them for asynchronous
+    copies): the block's inputs go to the device `arena`, the step updates the
+    device-resident state and z in place, and the block's output comes back
+    into `out`.  Asynchronous on `stream`; synchronise before reading `out`."""
+    B, Hh, d = _dims(q, T_blk, H, W)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out, cuda=False)
+    dev = state.device
+    if dev.type != "cuda" or z.device != dev:
+        raise ValueError("state and z must be on the GPU, on one device")
+    for name, t, shape in (("state", state, (B, Hh, d, d)), ("z", z, (B, Hh, d))):
+        if tuple(t.shape) != shape or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 tensor of shape {shape}")
+    if arena is None:
+        arena = alloc_workspace(gla_block_causal_host_arena_size(B, Hh, d, T_blk, H, W, code),
+                                dev)
+    if arena.device != dev or arena.dtype != torch.uint8 or not arena.is_contiguous():
+        raise ValueError(f"arena must be a contiguous uint8 tensor on {dev}")
+    with _on(dev):
+        st = lib().gla_block_causal_step_host(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v),
+                                              _ptr(beta), _ptr(g), B, Hh, d, T_blk, H, W, t0,
+                                              rope_theta, eps, code, _ptr(out), _ptr(arena),
+                                              arena.numel(), _stream(stream, dev))
+    _check(st, "gla_block_causal_step_host")
     return out
 
 
@@ -273,23 +329,29 @@ def gla_forward_noalloc(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6,
     if out is None:
         out = torch.empty_like(q)
     _validate(q, k, v, beta, g, out)
-    st = lib().gla_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d, T,
-                                   H, W, rope_theta, eps, code, _ptr(out), _stream(stream))
+    with _on(q.device):
+        st = lib().gla_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), B, Hh, d,
+                                       T, H, W, rope_theta, eps, code, _ptr(out),
+                                       _stream(stream, q.device))
     _check(st, "gla_forward_noalloc")
     return out
 
 
 def gla_get_device_status(stream=None):
     """Synchronise the stream and return (and clear) the device error status."""
-    return lib().gla_get_device_status(_stream(stream))
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with _on(dev):
+        return lib().gla_get_device_status(_stream(stream, dev))
 
 
 def gla_selftest_wait_timeout(limit_us, stream=None):
     """Launch the failure-detection self-test: a bounded wait that nothing
     satisfies gives up after `limit_us` microseconds and records a timeout
     (read it with gla_get_device_status)."""
-    _check(lib().gla_selftest_wait_timeout(int(limit_us), _stream(stream)),
-           "gla_selftest_wait_timeout")
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with _on(dev):
+        st = lib().gla_selftest_wait_timeout(int(limit_us), _stream(stream, dev))
+    _check(st, "gla_selftest_wait_timeout")
 
 
 def gla_plan(batch, heads, head_dim, T, H, W, dtype, path, num_sms):

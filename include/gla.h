@@ -206,6 +206,29 @@ GLA_API gla_status gla_forward_host(const void* q_h, const void* k_h, const void
                             int dtype, void* out_h, void* arena, size_t arena_bytes,
                             void* stream);
 
+/* Bytes of the device arena gla_block_causal_step_host needs: room for one
+ * block's five inputs, its output and the step's workspace. */
+GLA_API size_t gla_block_causal_host_arena_size(int batch, int heads, int head_dim, int T_blk,
+                                                int H, int W, int dtype);
+
+/* gla_block_causal_step on HOST buffers for one block (key design 2 of the
+ * SANA-Video notes: each block adds its own terms to the running sums that
+ * stay resident on the GPU).  q_h .. g_h and out_h are host memory (pinned
+ * memory gives asynchronous copies); state and z are the caller's DEVICE
+ * memory, carried between calls as in gla_block_causal_step.  Enqueues on
+ * `stream`: host-to-device copies of the block's inputs into the caller's
+ * device `arena` (at least gla_block_causal_host_arena_size() bytes, 256-byte
+ * aligned), the step, and the device-to-host copy of the block's output.
+ * Returns after enqueueing; synchronise `stream` before reading out_h.  The
+ * output equals gla_block_causal_step's on the same inputs bit for bit. */
+GLA_API gla_status gla_block_causal_step_host(float* state, float* z, const void* q_h,
+                                              const void* k_h, const void* v_h,
+                                              const void* beta_h, const void* g_h, int batch,
+                                              int heads, int head_dim, int T_blk, int H, int W,
+                                              int t0, float rope_theta, float eps, int dtype,
+                                              void* out_h, void* arena, size_t arena_bytes,
+                                              void* stream);
+
 /* Size of the scratch array built into the library for gla_forward_noalloc. */
 #define GLA_NOALLOC_SCRATCH_BYTES (24u << 20)
 

@@ -368,3 +368,21 @@ def max_rel_err_rms_floor(got, ref):
     got = np.asarray(got, dtype=np.float64)
     rms = np.sqrt(np.mean(ref * ref))
     return float(np.max(np.abs(got - ref) / np.maximum(np.abs(ref), rms)))
+
+
+def bf16_half_ulp(ref):
+    """Half the spacing of bf16 numbers (8 significant bits) at |ref|: the
+    largest error of a correctly rounded bf16 result."""
+    a = np.maximum(np.abs(np.asarray(ref, dtype=np.float64)), 2.0 ** -126)
+    return np.ldexp(1.0, (np.floor(np.log2(a)) - 8).astype(int))
+
+
+def bf16_out_err_over_rms(got, ref):
+    """Error of a bf16 output beyond its own rounding, over rms(ref):
+    max_i max(0, |got_i - ref_i| - bf16_half_ulp(ref_i)) / rms(ref).  A
+    correctly rounded result of the exact value scores 0; the rounding alone
+    reaches 1.56e-2 x rms for outputs in [4, 8) and is not arithmetic error."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    excess = np.maximum(np.abs(got - ref) - bf16_half_ulp(ref), 0.0)
+    return float(np.max(excess) / np.sqrt(np.mean(ref * ref)))

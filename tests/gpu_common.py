@@ -47,20 +47,14 @@ def rel_floor(got, ref):
 
 
 def bf16_half_ulp(ref):
-    """Half the spacing of bf16 numbers at |ref| (8 significant bits)."""
-    a = np.maximum(np.abs(np.asarray(ref, dtype=np.float64)), 2.0 ** -126)
-    return np.ldexp(1.0, (np.floor(np.log2(a)) - 8).astype(int))
+    """Half the spacing of bf16 numbers at |ref| (the oracle's metric helper)."""
+    return O.bf16_half_ulp(ref)
 
 
 def rel_rms_bf16out(got, ref):
-    """Error of a bf16 output beyond its own rounding, over rms(ref):
-    max_i max(0, |got_i - ref_i| - ulp_bf16(ref_i)/2) / rms(ref).  A correctly
-    rounded result of the exact value scores 0; the bf16 rounding itself is up
-    to 1.56e-2 x rms for outputs in [4, 8) and is not arithmetic error."""
-    got = np.asarray(got, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    excess = np.maximum(np.abs(got - ref) - bf16_half_ulp(ref), 0.0)
-    return float(np.max(excess) / np.sqrt(np.mean(ref * ref)))
+    """Error of a bf16 output beyond its own rounding, over rms(ref) (the
+    oracle's bf16_out_err_over_rms)."""
+    return O.bf16_out_err_over_rms(got, ref)
 
 
 def rel_elem(got, ref):

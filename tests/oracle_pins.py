@@ -433,11 +433,6 @@ def check_mx_forward_row_scale_invariance():
 # a slip in one of them (the RMS of the wrong array, a lost abs, a wrong
 # exponent) would otherwise loosen every parity test without anything failing.
 
-def _metrics():
-    import gpu_common
-    return gpu_common
-
-
 _REF4 = np.array([3.0, -4.0, 0.0, 0.0])        # rms = sqrt((9 + 16) / 4) = 2.5
 
 
@@ -465,27 +460,25 @@ def check_metric_bf16_half_ulp():
     against torch's round-to-nearest-even bf16 conversion: a value halfway
     between two bf16 neighbours is exactly half a spacing from its rounding."""
     import torch
-    gc = _metrics()
     vals = np.array([1.0, 1.99, 4.0, 7.99, 0.75, -3.0, 2.0 ** 20])
     want = np.array([2.0 ** -8, 2.0 ** -8, 2.0 ** -6, 2.0 ** -6, 2.0 ** -9, 2.0 ** -7, 2.0 ** 12])
-    _close(gc.bf16_half_ulp(vals), want, 0.0, "bf16 half ulp")
+    _close(O.bf16_half_ulp(vals), want, 0.0, "bf16 half ulp")
     rng = np.random.default_rng(5)
     e = rng.integers(-60, 60, 400)
     m = rng.integers(0, 128, 400)
     x = np.ldexp(1.0 + (2 * m + 1) / 256.0, e) * np.where(rng.random(400) < 0.5, -1.0, 1.0)
     rounded = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
-    _close(np.abs(rounded - x), gc.bf16_half_ulp(x), 0.0, "midpoints vs torch bf16")
+    _close(np.abs(rounded - x), O.bf16_half_ulp(x), 0.0, "midpoints vs torch bf16")
 
 
 def check_metric_rel_rms_bf16out():
     """Error beyond half a bf16 spacing, over rms(ref) = 2.5.  Half spacings:
     2^-7 at 3, 2^-6 at 4.  Errors (2^-7, -0.025, 0, 0) exceed them by
     (0, 0.025 - 2^-6, 0, 0): 0.009375 / 2.5 = 0.00375."""
-    gc = _metrics()
     got = _REF4 + np.array([2.0 ** -7, -0.025, 0.0, 0.0])
-    _close(gc.rel_rms_bf16out(got, _REF4), 0.00375, 1e-9, "bf16 output metric")
+    _close(O.bf16_out_err_over_rms(got, _REF4), 0.00375, 1e-9, "bf16 output metric")
     got = _REF4 + np.array([2.0 ** -7, -2.0 ** -6, 0.0, 0.0])
-    assert gc.rel_rms_bf16out(got, _REF4) == 0.0, "a correct rounding scores 0"
+    assert O.bf16_out_err_over_rms(got, _REF4) == 0.0, "a correct rounding scores 0"
 
 
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

@@ -65,3 +65,18 @@ def test_host_entry_rejects_host_arena():
     x = host_inputs()
     with pytest.raises(ValueError, match="arena"):
         call_host(x, arena=torch.zeros(1 << 20, dtype=torch.uint8))
+
+
+class _FakeStream:
+    def __init__(self, device):
+        self.device = torch.device(device)
+        self.cuda_stream = 0
+
+
+def test_stream_of_another_device_is_refused():
+    """The library launches on the current device, which the binding sets to
+    the tensors' device for each call; a stream of a different device would
+    put the kernels on one GPU and the pointers on another."""
+    with pytest.raises(ValueError, match="stream"):
+        gla._stream(_FakeStream("cuda:1"), torch.device("cuda", 0))
+    assert gla._stream(_FakeStream("cuda:0"), torch.device("cuda", 0)).value in (None, 0)

@@ -99,3 +99,28 @@ def test_output_rows_have_unit_rms():
     # Rounding to bf16 (8 significant bits) moves each element, and so a row's
     # RMS, by at most 2^-8 relative.
     assert np.all(np.abs(rms - expect) <= 2.0 ** -8 * expect + 1e-5), np.abs(rms - expect).max()
+
+
+def test_host_step_entry_matches_device_steps():
+    """gla_block_causal_step_host (host inputs and output, device-resident
+    state) gives the device entry's outputs and state bit for bit, over three
+    consecutive blocks."""
+    T, H, W, B, HH, n = 2, 5, 9, 1, 3, 3
+    L = T * H * W
+    inp = workloads.draw(B, n * L, HH, 128, "bf16", seed=41)
+    blocks = [{k: v[:, i * L:(i + 1) * L].contiguous() for k, v in inp.items()} for i in range(n)]
+    S_d = torch.zeros(B, HH, 128, 128, device="cuda")
+    z_d = torch.zeros(B, HH, 128, device="cuda")
+    S_h, z_h = S_d.clone(), z_d.clone()
+    for i, blk in enumerate(blocks):
+        d = {k: v.cuda() for k, v in blk.items()}
+        o_d = gla.gla_block_causal_step(S_d, z_d, d["q"], d["k"], d["v"], d["beta"], d["g"],
+                                        T, H, W, i * T)
+        p = {k: v.pin_memory() for k, v in blk.items()}
+        o_h = torch.empty_like(p["q"]).pin_memory()
+        gla.gla_block_causal_step_host(S_h, z_h, p["q"], p["k"], p["v"], p["beta"], p["g"],
+                                       T, H, W, i * T, out=o_h)
+        torch.cuda.synchronize()
+        assert gla.gla_get_device_status() == gla.GLA_OK
+        assert torch.equal(o_h, o_d.cpu())
+    assert torch.equal(S_h, S_d) and torch.equal(z_h, z_d)

@@ -3,7 +3,6 @@ pins catch every one of them: each mutant must fail at least one check."""
 import numpy as np
 import pytest
 
-import gpu_common
 import oracle.gla_oracle as O
 import oracle_pins
 
@@ -175,7 +174,7 @@ def test_mutant_is_caught(name, monkeypatch):
     assert failed, f"mutant {name} passed every pin"
 
 
-# Mistakes in the tolerance metrics (the oracle's and the GPU tests' helpers).
+# Mistakes in the tolerance metrics every GPU parity test goes through.
 
 def _rms_of_got(got, ref):
     return _orig["max_err_over_rms"](ref, got)
@@ -213,9 +212,6 @@ def _floor_rms_only(got, ref):
     return float(np.max(np.abs(got - ref)) / np.sqrt(np.mean(ref * ref)))
 
 
-_orig_gc = {name: getattr(gpu_common, name) for name in ("bf16_half_ulp", "rel_rms_bf16out")}
-
-
 def _half_ulp_exp7(ref):
     a = np.maximum(np.abs(np.asarray(ref, dtype=np.float64)), 2.0 ** -126)
     return np.ldexp(1.0, (np.floor(np.log2(a)) - 7).astype(int))
@@ -233,14 +229,14 @@ def _bf16out_no_rounding_allowance(got, ref):
 def _bf16out_rms_of_got(got, ref):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
-    excess = np.maximum(np.abs(got - ref) - _orig_gc["bf16_half_ulp"](ref), 0.0)
+    excess = np.maximum(np.abs(got - ref) - _orig["bf16_half_ulp"](ref), 0.0)
     return float(np.max(excess) / np.sqrt(np.mean(got * got)))
 
 
 def _bf16out_full_ulp(got, ref):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
-    excess = np.maximum(np.abs(got - ref) - 2.0 * _orig_gc["bf16_half_ulp"](ref), 0.0)
+    excess = np.maximum(np.abs(got - ref) - 2.0 * _orig["bf16_half_ulp"](ref), 0.0)
     return float(np.max(excess) / np.sqrt(np.mean(ref * ref)))
 
 
@@ -251,11 +247,11 @@ METRIC_MUTANTS = {
     "floor_no_abs": (O, "max_rel_err_rms_floor", _floor_no_abs),
     "floor_rms_of_got": (O, "max_rel_err_rms_floor", _floor_rms_of_got),
     "floor_missing": (O, "max_rel_err_rms_floor", _floor_rms_only),
-    "half_ulp_exp7": (gpu_common, "bf16_half_ulp", _half_ulp_exp7),
-    "half_ulp_ceil": (gpu_common, "bf16_half_ulp", _half_ulp_ceil),
-    "bf16out_no_allowance": (gpu_common, "rel_rms_bf16out", _bf16out_no_rounding_allowance),
-    "bf16out_rms_of_got": (gpu_common, "rel_rms_bf16out", _bf16out_rms_of_got),
-    "bf16out_full_ulp": (gpu_common, "rel_rms_bf16out", _bf16out_full_ulp),
+    "half_ulp_exp7": (O, "bf16_half_ulp", _half_ulp_exp7),
+    "half_ulp_ceil": (O, "bf16_half_ulp", _half_ulp_ceil),
+    "bf16out_no_allowance": (O, "bf16_out_err_over_rms", _bf16out_no_rounding_allowance),
+    "bf16out_rms_of_got": (O, "bf16_out_err_over_rms", _bf16out_rms_of_got),
+    "bf16out_full_ulp": (O, "bf16_out_err_over_rms", _bf16out_full_ulp),
 }
 
 

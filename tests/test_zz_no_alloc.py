@@ -35,13 +35,36 @@ def test_noalloc_matches_forward_bf16_720p():
     _both(wl, workloads.make_inputs(wl), BF16_TOL, rel_rms)
 
 
+def _scratch_bytes():
+    """GLA_NOALLOC_SCRATCH_BYTES as include/gla.h defines it."""
+    import os
+    import re
+    hdr = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                       "include", "gla.h")
+    m = re.search(r"#define GLA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", open(hdr).read())
+    assert m, "GLA_NOALLOC_SCRATCH_BYTES not found in gla.h"
+    return int(m.group(1)) << int(m.group(2))
+
+
+def test_noalloc_matches_forward_fp32_720p_simt():
+    """fp32 inputs at the 720p shape run on the CUDA-core path, whose scratch
+    (no fp16 image, no read-out table) fits the array."""
+    wl = workloads.WORKLOADS["720p"]
+    inp = workloads.draw(wl.batch, wl.tokens, wl.heads, wl.head_dim, "f32", wl.seed)
+    _both(wl, inp, F32_TOL, rel_floor)
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    # 4 x 64 heads of d = 128: the combined states alone exceed the array.
-    d = torch.empty(16, dtype=torch.bfloat16, device="cuda")
+    # Enough heads that the combined fp32 states alone (heads x d x d x 4
+    # bytes, one part of the scratch) take twice the array; one token each.
+    # Every buffer passed has the problem's real size, and the host checks
+    # from the same formula that the problem is beyond the array.
+    cap, d = _scratch_bytes(), 128
+    heads = 2 * cap // (d * d * 4) + 32
+    assert heads * d * d * 4 > 2 * cap
+    x = workloads.draw(1, 1, heads, d, "bf16", seed=3)
+    x = to_device(x)
+    out = torch.empty_like(x["q"])
     with pytest.raises(gla.GlaError) as e:
-        gla.lib()
-        st = gla.lib().gla_forward_noalloc(d.data_ptr(), d.data_ptr(), d.data_ptr(),
-                                           d.data_ptr(), d.data_ptr(), 4, 64, 128, 1, 4, 32,
-                                           1e4, 1e-6, gla.GLA_DTYPE_BF16, d.data_ptr(), None)
-        gla._check(st, "gla_forward_noalloc")
+        gla.gla_forward_noalloc(x["q"], x["k"], x["v"], x["beta"], x["g"], 1, 1, 1, out=out)
     assert e.value.status == gla.GLA_ERR_WORKSPACE
