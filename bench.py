@@ -491,6 +491,16 @@ def run_block_causal(args, wl, gla, dev, dist, world, rank, local):
                                       wl.W, i * wl.T, wl.rope_theta, wl.eps, out=outs[i],
                                       workspace=ws, stream=stream)
 
+    if args.profile:
+        for _ in range(args.warmup + args.steps):
+            sequence()
+        torch.cuda.synchronize(dev)
+        status = gla.gla_get_device_status(stream)
+        print(json.dumps({"profile_run": wl.name, "sequences": args.warmup + args.steps,
+                          "status": gla.status_string(status)}))
+        if status != gla.GLA_OK:
+            sys.exit(1)
+        return
     for _ in range(max(args.warmup, 3)):
         sequence()
     torch.cuda.synchronize(dev)
