@@ -297,6 +297,39 @@ def causal_forward(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
     return dict(den=den, pre=pre, x=x, out=rms_normalize(x))
 
 
+def causal_forward_at(q, k, v, beta, g, T, H, W, rope_theta, eps, tokens, t0=0,
+                      S0=None, z0=None):
+    """The token-level causal read-out at the selected tokens only, each from
+    its own prefix (the definition above, token by token, with no running
+    sums):  S_j = S0 + sum_{n<=j} v_n (beta_n k_til_n)^T,
+    z_j = z0 + sum_{n<=j} k_pls_n, and the read-out of token j against them.
+    S0 [B, Hh, d, d] and z0 [B, Hh, d] are a state carried in from earlier
+    tokens (zero if None), as a streaming call continues a sequence.  Memory
+    stays O(N d), so it serves full-size inputs.  Returns den, pre, x, out of
+    shape [B, len(tokens), Hh(, d)] and the state after the last token,
+    S_end / z_end."""
+    d = q.shape[-1]
+    B, N, Hh, _ = q.shape
+    assert N == T * H * W
+    angles = _angles_or_none(d, T, H, W, rope_theta, t0)
+    q_pls, q_til = feature_maps(q, angles)
+    k_pls, k_til = feature_maps(k, angles)
+    S0 = np.zeros((B, Hh, d, d)) if S0 is None else S0
+    z0 = np.zeros((B, Hh, d)) if z0 is None else z0
+    tokens = list(tokens)
+    den = np.empty((B, len(tokens), Hh))
+    u = np.empty((B, len(tokens), Hh, d))
+    for i, j in enumerate(tokens):
+        S, z = state_and_keysum(k_til[:, :j + 1], k_pls[:, :j + 1], v[:, :j + 1],
+                                beta[:, :j + 1])
+        r = read_out(S0 + S, z0 + z, q_pls[:, j:j + 1], q_til[:, j:j + 1], g[:, j:j + 1], eps)
+        den[:, i] = r["den"][:, 0]
+        u[:, i] = r["pre"][:, 0]
+    x = sigmoid(g[:, tokens]) * u
+    S, z = state_and_keysum(k_til, k_pls, v, beta)
+    return dict(den=den, pre=u, x=x, out=rms_normalize(x), S_end=S0 + S, z_end=z0 + z)
+
+
 def causal_bruteforce(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
     """Prefix-masked pair sum: token j sees token n iff n <= j."""
     return forward_bruteforce(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=t0,

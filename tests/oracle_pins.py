@@ -361,6 +361,37 @@ def check_causal_time_shift_invariance():
     _close(a["out"], b["out"], 1e-10, "causal time shift")
 
 
+def check_causal_at_selected_tokens():
+    """The token-by-token prefix form at selected tokens equals the running
+    sums (two computations of the same definition: per-token prefixes
+    against cumulative sums), and its end state is the full-sequence state."""
+    (q, k, v, beta, g), (T, H, W) = _causal_inputs()
+    toks = [0, 1, 5, 11, T * H * W - 1]
+    a = O.causal_forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5)
+    b = O.causal_forward_at(q, k, v, beta, g, T, H, W, 10000.0, 1e-5, toks)
+    for key in ("den", "pre", "out"):
+        _close(b[key], a[key][:, toks], 1e-12, f"causal at tokens: {key}")
+    full = O.forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5)
+    _close(b["S_end"], full["S"], 1e-12, "causal end state")
+    _close(b["z_end"], full["z"], 1e-12, "causal end key sum")
+
+
+def check_causal_carried_state():
+    """Streaming: running the second half of a sequence from the first
+    half's end state (with the time offset of the second half) gives the
+    whole sequence's causal outputs for the second half."""
+    (q, k, v, beta, g), (T, H, W) = _causal_inputs(T=4)
+    L = (T // 2) * H * W
+    whole = O.causal_forward(q, k, v, beta, g, T, H, W, 10000.0, 1e-5)
+    first = O.causal_forward_at(q[:, :L], k[:, :L], v[:, :L], beta[:, :L], g[:, :L], T // 2,
+                                H, W, 10000.0, 1e-5, [L - 1])
+    sl = slice(L, None)
+    second = O.causal_forward_at(q[:, sl], k[:, sl], v[:, sl], beta[:, sl], g[:, sl], T // 2,
+                                 H, W, 10000.0, 1e-5, range(L), t0=T // 2,
+                                 S0=first["S_end"], z0=first["z_end"])
+    _close(second["out"], whole["out"][:, L:], 1e-12, "carried causal state")
+
+
 # ---------------------------------------------------- MXFP8 input decoding
 
 def check_e4m3_format_values():

@@ -94,15 +94,17 @@ def _causal_exclusive(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
     k_pls, k_til = O.feature_maps(k, angles)
     B, N, Hh, _ = q.shape
     pre = np.empty_like(q)
+    dens = np.empty((B, N, Hh))
     for b in range(B):
         for h in range(Hh):
             per = v[b, :, h, :, None] * (beta[b, :, h, None, None] * k_til[b, :, h, None, :])
             S_run = np.cumsum(per, axis=0) - per
             z_run = np.cumsum(k_pls[b, :, h, :], axis=0) - k_pls[b, :, h, :]
             den = np.einsum("nc,nc->n", z_run, q_pls[b, :, h, :]) + eps
+            dens[b, :, h] = den
             pre[b, :, h, :] = np.einsum("nac,nc->na", S_run, q_til[b, :, h, :]) / den[:, None]
     x = O.sigmoid(g) * pre
-    return dict(pre=pre, x=x, out=O.rms_normalize(x))
+    return dict(den=dens, pre=pre, x=x, out=O.rms_normalize(x))
 
 
 def _causal_suffix(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
@@ -111,6 +113,21 @@ def _causal_suffix(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
     r = _orig["causal_forward"](flip(q), flip(k), flip(v), flip(beta), flip(g), T, H, W,
                                 rope_theta, eps, t0)
     return {key: flip(val) for key, val in r.items()}
+
+
+def _causal_at_exclusive(q, k, v, beta, g, T, H, W, rope_theta, eps, tokens, t0=0, S0=None,
+                         z0=None):
+    """Each selected token read out against the tokens before it only."""
+    tokens = list(tokens)
+    r = _orig["causal_forward_at"](q, k, v, beta, g, T, H, W, rope_theta, eps,
+                                   [max(j - 1, 0) for j in tokens], t0, S0, z0)
+    return r
+
+
+def _causal_at_no_carry(q, k, v, beta, g, T, H, W, rope_theta, eps, tokens, t0=0, S0=None,
+                        z0=None):
+    """The carried-in state dropped."""
+    return _orig["causal_forward_at"](q, k, v, beta, g, T, H, W, rope_theta, eps, tokens, t0)
 
 
 def _e4m3_bias8(codes):
@@ -154,6 +171,8 @@ MUTANTS = {
     "sigmoid_sign": ("sigmoid", _neg_sigmoid),
     "causal_exclusive": ("causal_forward", _causal_exclusive),
     "causal_suffix": ("causal_forward", _causal_suffix),
+    "causal_at_exclusive": ("causal_forward_at", _causal_at_exclusive),
+    "causal_at_no_carry": ("causal_forward_at", _causal_at_no_carry),
     "e4m3_bias8": ("e4m3_decode", _e4m3_bias8),
     "e4m3_no_subnormals": ("e4m3_decode", _e4m3_no_subnormals),
     "e8m0_bias128": ("e8m0_decode", _e8m0_bias128),
