@@ -44,6 +44,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="720p", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--variant", default="bidirectional", choices=["bidirectional", "causal"],
+                    help="causal: the token-level causal read-out (gla_causal_step) of the "
+                         "workload, one step = one call from a zero state")
     ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
@@ -319,6 +322,9 @@ def main():
     if wl.n_blocks > 1:
         run_block_causal(args, wl, gla, dev, dist, world, rank, local)
         return
+    if args.variant == "causal":
+        run_causal(args, wl, gla, dev, dist, world, rank, local)
+        return
 
     inp = workloads.make_inputs(wl, seed=replicas.replica_seed(wl.seed, rank))
     d = {k: v.to(dev) for k, v in inp.items()}
@@ -456,6 +462,158 @@ def main():
             "step_frac_of_nominal_8tbs": step_gbs / 8000.0,
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": th * hd * esz * 4 + th * esz,
+                    "d2h_bytes_per_step": th * hd * esz, "steps": e2e_steps},
+            "gpu_launches": 3 * args.steps,
+            "clocks": mon.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_causal(args, wl, gla, dev, dist, world, rank, local):
+    """One step = one gla_causal_step over the whole workload from a zero
+    state (a new sequence): the token-level causal variant's own measurement."""
+    inp = workloads.make_inputs(wl, seed=replicas.replica_seed(wl.seed, rank))
+    d = {k: v.to(dev) for k, v in inp.items()}
+    B, N, Hh, hd = d["q"].shape
+    code = gla.GLA_DTYPE_BF16 if d["q"].dtype == torch.bfloat16 else gla.GLA_DTYPE_F32
+    S = torch.zeros(B, Hh, hd, hd, dtype=torch.float32, device=dev)
+    z = torch.zeros(B, Hh, hd, dtype=torch.float32, device=dev)
+    out = torch.empty_like(d["q"])
+    ws = gla.alloc_workspace(gla.gla_causal_workspace_size(B, Hh, hd, wl.T, wl.H, wl.W, code), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        S.zero_()
+        z.zero_()
+        if events is None:
+            gla.gla_causal_step(S, z, d["q"], d["k"], d["v"], d["beta"], d["g"], wl.T, wl.H, wl.W,
+                                0, wl.rope_theta, wl.eps, out=out, workspace=ws, stream=stream)
+        else:
+            gla.gla_causal_step_timed(S, z, d["q"], d["k"], d["v"], d["beta"], d["g"], wl.T,
+                                      wl.H, wl.W, events, 0, wl.rope_theta, wl.eps, out=out,
+                                      workspace=ws, stream=stream)
+
+    if args.profile:
+        for _ in range(args.warmup + args.steps):
+            step()
+        torch.cuda.synchronize(dev)
+        status = gla.gla_get_device_status(stream)
+        print(json.dumps({"profile_run": wl.name, "variant": "causal",
+                          "steps": args.warmup + args.steps, "status": gla.status_string(status)}))
+        if status != gla.GLA_OK:
+            sys.exit(1)
+        return
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert gla.gla_get_device_status(stream) == gla.GLA_OK
+
+    def sync():
+        torch.cuda.synchronize(dev)
+
+    def timed_steps():
+        for _ in range(args.steps):
+            step()
+
+    with ClockMonitor(local) as mon:
+        elapsed_ms, reps = timed_repeats(timed_steps, stream, dist, sync, dev, args.repeats)
+    if gla.gla_get_device_status(stream) != gla.GLA_OK:
+        raise RuntimeError("device status after the timed region")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e4 in evs:
+        for e in e4:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    k_state = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    k_prefix = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    k_read = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+
+    # End to end through the host entry: inputs from pinned host memory, the
+    # call, the output back; the state stays on the device.
+    pinned = {k: v.pin_memory() for k, v in inp.items()}
+    out_h = torch.empty_like(pinned["q"]).pin_memory()
+    arena = gla.alloc_workspace(gla.gla_causal_host_arena_size(B, Hh, hd, wl.T, wl.H, wl.W, code),
+                                dev)
+
+    def host_step():
+        S.zero_()
+        z.zero_()
+        gla.gla_causal_step_host(S, z, pinned["q"], pinned["k"], pinned["v"], pinned["beta"],
+                                 pinned["g"], wl.T, wl.H, wl.W, 0, wl.rope_theta, wl.eps,
+                                 out=out_h, arena=arena, stream=stream)
+
+    e2e_steps = max(3, min(args.steps, 100))
+    for _ in range(2):
+        host_step()
+
+    def host_steps():
+        for _ in range(e2e_steps):
+            host_step()
+
+    e2e_ms = replicas.timed(host_steps, replicas.CudaTimer(stream), dist, sync, dev)
+
+    th = B * N * Hh
+    esz = 2 if code == gla.GLA_DTYPE_BF16 else 4
+    ms_per_step = elapsed_ms / args.steps
+    peak, peak_kind = measured_peaks()
+    alg = wl.alg_bytes_per_call()                  # q, k, v, g, beta read + out written
+    read_gbs = alg / (k_read * 1e-3) / 1e9
+    step_gbs = alg / (ms_per_step * 1e-3) / 1e9
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            import oracle.gla_oracle as O
+            from threadpoolctl import threadpool_info
+            # The oracle's running-sum form on whole heads of the first two
+            # frames (its memory grows as N d^2), scaled to the layer.
+            T_s = min(2, wl.T)
+            n_s = T_s * wl.H * wl.W
+            secs, heads = 0.0, 0
+            while secs < args.cpu_sample_seconds:
+                x = workloads.as_f64(workloads.draw(1, n_s, 1, hd, wl.dtype, 3000 + heads))
+                c0 = time.perf_counter()
+                O.causal_forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T_s, wl.H, wl.W,
+                                 wl.rope_theta, wl.eps)
+                secs += time.perf_counter() - c0
+                heads += 1
+            blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+            cpu = {"value": heads * n_s / secs / wl.heads, "unit": "tokens/s",
+                   "cores": blas[0] if blas else 1, "kind": "oracle",
+                   "sample": (f"oracle.causal_forward on {heads} heads of the first {T_s} frames "
+                              f"({n_s} tokens each) of the {wl.name} grid, {secs:.1f} s; tokens/s "
+                              f"of the full layer = token-heads/s / {wl.heads}; cores = BLAS "
+                              f"threads"),
+                   "host": host_info()}
+        line = {
+            "metric": (f"gla_causal_step tokens/s ({wl.heads}x{hd} heads, {wl.tokens} tok, "
+                       "token-level causal)"),
+            "value": replicas.aggregate_rate(world, B * N, args.steps, elapsed_ms),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "repeats": len(reps),
+            "repeat_ms_per_step": [round(r / args.steps, 5) for r in reps],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if code == gla.GLA_DTYPE_BF16 else "f32", "data": "synthetic",
+            "config": dict(workload_config(wl), variant="token-level causal from a zero state",
+                           parallelism=f"replicas x{world}"),
+            "roofline": {"bound": "hbm", "kernel": "tc_causal_kernel", "achieved": read_gbs,
+                         "peak": peak, "unit": "GB/s", "frac": read_gbs / peak,
+                         "peak_kind": peak_kind,
+                         "traffic": traffic_for("tc_causal_kernel", wl.name),
+                         "alg_bytes_per_launch": alg, "ms_per_launch": k_read},
+            "kernels_ms": {"tc_state_kernel": k_state, "combine_prefix_kernel": k_prefix,
+                           "tc_causal_kernel": k_read,
+                           "how": "second timed pass of the same K steps, events around each kernel"},
+            "step_gbs_at_min_bytes": step_gbs, "step_frac_of_peak": step_gbs / peak,
+            "e2e": {"value": replicas.aggregate_rate(world, B * N, e2e_steps, e2e_ms),
+                    "unit": "tokens/s", "h2d_bytes_per_step": th * hd * esz * 4 + th * esz,
                     "d2h_bytes_per_step": th * hd * esz, "steps": e2e_steps},
             "gpu_launches": 3 * args.steps,
             "clocks": mon.summary(),

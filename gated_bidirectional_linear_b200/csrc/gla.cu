@@ -15,6 +15,7 @@
 #include "combine.cuh"
 #include "simt.cuh"
 #include "tc.cuh"
+#include "causal.cuh"
 
 using namespace gla;
 
@@ -312,6 +313,102 @@ gla_status run_call(Call& c) {
   return GLA_OK;
 }
 
+// Workspace of a causal call (tensor path): the state partials and, per
+// partial slot, the state before it.
+struct CausalWs {
+  size_t part_S, part_z, S_start, z_start, total;
+};
+
+CausalWs causal_ws(int BH, int d) {
+  CausalWs L;
+  const size_t slots = (size_t)kMaxStateCtas + BH;
+  size_t off = 0;
+  L.part_S = off; off = align_up(off + slots * d * d * 4, kAlign);
+  L.part_z = off; off = align_up(off + slots * kMaxZParts * d * 4, kAlign);
+  L.S_start = off; off = align_up(off + slots * d * d * 4, kAlign);
+  L.z_start = off; off = align_up(off + slots * d * 4, kAlign);
+  L.total = off;
+  return L;
+}
+
+bool causal_tensor_fits(const Geom& g, int sms) {
+  if (g.H >= (1 << kPosBits) || g.W >= (1 << kPosBits) || g.T >= (1 << kPosBits)) return false;
+  if (!tc_rope_lanes_ok(g)) return false;
+  const int stab = tc_table_entries(g, tc_state_partition(g, sms));
+  return tc_state_smem(stab) <= kMaxSmem && tc_causal_smem(stab) <= kMaxSmem;
+}
+
+template <int D, typename Tin>
+gla_status run_simt_causal(const Geom& g, const void* q, const void* k, const void* v,
+                           const void* beta, const void* gate, void* out, float* S, float* z,
+                           float* den_out, float* x_out, cudaStream_t stream) {
+  SimtCausalParams sp;
+  sp.g = g;
+  sp.q = q; sp.k = k; sp.v = v; sp.beta = beta; sp.gate = gate; sp.out = out;
+  sp.S = S; sp.z = z; sp.den_out = den_out; sp.x_out = x_out;
+  const size_t smem = simt_causal_smem<D>();
+  if (set_smem(simt_causal_kernel<D, Tin>, smem) != cudaSuccess) return GLA_ERR_CUDA;
+  simt_causal_kernel<D, Tin><<<g.B * g.Hh, kSimtCausalThreads, smem, stream>>>(sp);
+  return cudaGetLastError() == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+}
+
+template <typename Tin>
+gla_status run_simt_causal_dim(const Geom& g, const void* q, const void* k, const void* v,
+                               const void* beta, const void* gate, void* out, float* S,
+                               float* z, float* den_out, float* x_out, cudaStream_t stream) {
+  switch (g.d) {
+    case 32: return run_simt_causal<32, Tin>(g, q, k, v, beta, gate, out, S, z, den_out, x_out, stream);
+    case 64: return run_simt_causal<64, Tin>(g, q, k, v, beta, gate, out, S, z, den_out, x_out, stream);
+    case 128: return run_simt_causal<128, Tin>(g, q, k, v, beta, gate, out, S, z, den_out, x_out, stream);
+  }
+  return GLA_ERR_UNSUPPORTED;
+}
+
+// Device bytes of one call's five inputs and its output, staged in an arena
+// for the host entry points of the stateful variants.
+size_t staged_inputs_bytes(int batch, int heads, int head_dim, int T, int H, int W, int dtype) {
+  const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
+  const size_t th = (size_t)batch * T * H * W * heads;
+  return 5 * align_up(th * head_dim * esz, kAlign) + align_up(th * esz, kAlign);
+}
+
+// Copies one call's host inputs into the device arena, runs `step` on them
+// (the state stays in device memory) and copies the output back, all
+// enqueued on `stream`.
+template <typename Step>
+gla_status staged_step(const void* q_h, const void* k_h, const void* v_h, const void* beta_h,
+                       const void* g_h, void* out_h, int batch, int heads, int head_dim, int T,
+                       int H, int W, int dtype, void* arena, size_t arena_bytes, size_t need,
+                       void* stream, Step step) {
+  const void* hp[6] = {q_h, k_h, v_h, beta_h, g_h, out_h};
+  for (const void* p : hp)
+    if (!p) return GLA_ERR_INVALID_ARG;
+  if (!arena || ((uintptr_t)arena % kAlign) != 0 || arena_bytes < need) return GLA_ERR_WORKSPACE;
+  const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
+  const size_t th = (size_t)batch * T * H * W * heads;
+  const size_t big = th * head_dim * esz, small = th * esz;
+  unsigned char* a = static_cast<unsigned char*>(arena);
+  unsigned char* dq = a;
+  unsigned char* dk = dq + align_up(big, kAlign);
+  unsigned char* dv = dk + align_up(big, kAlign);
+  unsigned char* dg = dv + align_up(big, kAlign);
+  unsigned char* dout = dg + align_up(big, kAlign);
+  unsigned char* dbeta = dout + align_up(big, kAlign);
+  unsigned char* dws = dbeta + align_up(small, kAlign);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(dq, q_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dg, g_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dbeta, beta_h, small, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  const gla_status st = step(dq, dk, dv, dbeta, dg, dout, dws, arena_bytes - (size_t)(dws - a));
+  if (st != GLA_OK) return st;
+  if (cudaMemcpyAsync(out_h, dout, big, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  return GLA_OK;
+}
+
 gla_status forward_common(const void* q, const void* k, const void* v, const void* beta,
                           const void* g, int batch, int heads, int head_dim, int T, int H,
                           int W, float rope_theta, float eps, int dtype, void* out,
@@ -456,6 +553,75 @@ gla_status gla_block_causal_step(float* state, float* z, const void* q, const vo
                                   workspace_bytes, stream, GLA_PATH_AUTO);
 }
 
+size_t gla_causal_workspace_size(int batch, int heads, int head_dim, int T, int H, int W,
+                                 int dtype) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W)) return 0;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return 0;
+  return causal_ws(batch * heads, head_dim).total;
+}
+
+gla_status gla_causal_step_timed(float* state, float* z, const void* q, const void* k,
+                                 const void* v, const void* beta, const void* g, int batch,
+                                 int heads, int head_dim, int T, int H, int W, int t0,
+                                 float rope_theta, float eps, int dtype, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream, int path,
+                                 float* den_out, float* x_out, void* const* events) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W) || t0 < 0) return GLA_ERR_INVALID_ARG;
+  if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+  if (!(eps > 0.f) || !isfinite(eps) || !isfinite(rope_theta)) return GLA_ERR_INVALID_ARG;
+  const void* ptrs[8] = {state, z, q, k, v, beta, g, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
+  if (resolve_path(path, dtype, head_dim) < 0) return GLA_ERR_UNSUPPORTED;
+  const Geom geom = make_geom(batch, heads, head_dim, T, H, W, t0, rope_theta, eps);
+  const int sms = device_sm_count();
+  if (sms <= 0) return GLA_ERR_CUDA;
+  int used = resolve_path(path, dtype, head_dim);
+  if (used == GLA_PATH_TENSOR && !causal_tensor_fits(geom, sms)) {
+    if (path == GLA_PATH_TENSOR) return GLA_ERR_UNSUPPORTED;
+    used = GLA_PATH_SIMT;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (used == GLA_PATH_SIMT && events && events[0] &&
+      cudaEventRecord(static_cast<cudaEvent_t>(events[0]), st) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  if (used == GLA_PATH_SIMT)
+    return dtype == GLA_DTYPE_F32
+               ? run_simt_causal_dim<float>(geom, q, k, v, beta, g, out, state, z, den_out, x_out, st)
+               : run_simt_causal_dim<__nv_bfloat16>(geom, q, k, v, beta, g, out, state, z, den_out,
+                                                    x_out, st);
+  const CausalWs L = causal_ws(batch * heads, head_dim);
+  if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < L.total)
+    return GLA_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  return run_causal_tensor(geom, q, k, v, beta, g, out, state, z,
+                           reinterpret_cast<float*>(ws + L.part_S),
+                           reinterpret_cast<float*>(ws + L.part_z),
+                           reinterpret_cast<float*>(ws + L.S_start),
+                           reinterpret_cast<float*>(ws + L.z_start), den_out, x_out, sms, st,
+                           events);
+}
+
+gla_status gla_causal_step_ex(float* state, float* z, const void* q, const void* k,
+                              const void* v, const void* beta, const void* g, int batch,
+                              int heads, int head_dim, int T, int H, int W, int t0,
+                              float rope_theta, float eps, int dtype, void* out,
+                              void* workspace, size_t workspace_bytes, void* stream, int path,
+                              float* den_out, float* x_out) {
+  return gla_causal_step_timed(state, z, q, k, v, beta, g, batch, heads, head_dim, T, H, W, t0,
+                               rope_theta, eps, dtype, out, workspace, workspace_bytes, stream,
+                               path, den_out, x_out, nullptr);
+}
+
+gla_status gla_causal_step(float* state, float* z, const void* q, const void* k, const void* v,
+                           const void* beta, const void* g, int batch, int heads, int head_dim,
+                           int T, int H, int W, int t0, float rope_theta, float eps, int dtype,
+                           void* out, void* workspace, size_t workspace_bytes, void* stream) {
+  return gla_causal_step_ex(state, z, q, k, v, beta, g, batch, heads, head_dim, T, H, W, t0,
+                            rope_theta, eps, dtype, out, workspace, workspace_bytes, stream,
+                            GLA_PATH_AUTO, nullptr, nullptr);
+}
+
 size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, int T, int H, int W,
                                    int dtype) {
   const size_t ws = gla_forward_workspace_size(batch, heads, head_dim, T, H, W, dtype);
@@ -555,9 +721,7 @@ size_t gla_block_causal_host_arena_size(int batch, int heads, int head_dim, int 
                                         int W, int dtype) {
   const size_t ws = gla_block_causal_workspace_size(batch, heads, head_dim, T_blk, H, W, dtype);
   if (!ws) return 0;
-  const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
-  const size_t th = (size_t)batch * T_blk * H * W * heads;
-  return 5 * align_up(th * head_dim * esz, kAlign) + align_up(th * esz, kAlign) + ws;
+  return staged_inputs_bytes(batch, heads, head_dim, T_blk, H, W, dtype) + ws;
 }
 
 gla_status gla_block_causal_step_host(float* state, float* z, const void* q_h, const void* k_h,
@@ -569,35 +733,39 @@ gla_status gla_block_causal_step_host(float* state, float* z, const void* q_h, c
   const size_t need =
       gla_block_causal_host_arena_size(batch, heads, head_dim, T_blk, H, W, dtype);
   if (!need) return GLA_ERR_INVALID_ARG;
-  const void* hp[6] = {q_h, k_h, v_h, beta_h, g_h, out_h};
-  for (const void* p : hp)
-    if (!p) return GLA_ERR_INVALID_ARG;
-  if (!arena || ((uintptr_t)arena % kAlign) != 0 || arena_bytes < need) return GLA_ERR_WORKSPACE;
-  const size_t esz = dtype == GLA_DTYPE_F32 ? 4 : 2;
-  const size_t th = (size_t)batch * T_blk * H * W * heads;
-  const size_t big = th * head_dim * esz, small = th * esz;
-  unsigned char* a = static_cast<unsigned char*>(arena);
-  unsigned char* dq = a;
-  unsigned char* dk = dq + align_up(big, kAlign);
-  unsigned char* dv = dk + align_up(big, kAlign);
-  unsigned char* dg = dv + align_up(big, kAlign);
-  unsigned char* dout = dg + align_up(big, kAlign);
-  unsigned char* dbeta = dout + align_up(big, kAlign);
-  unsigned char* dws = dbeta + align_up(small, kAlign);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(dq, q_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dg, g_h, big, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dbeta, beta_h, small, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return GLA_ERR_CUDA;
-  const gla_status st = gla_block_causal_step(
-      state, z, dq, dk, dv, dbeta, dg, batch, heads, head_dim, T_blk, H, W, t0, rope_theta, eps,
-      dtype, dout, dws, arena_bytes - (size_t)(dws - a), stream);
-  if (st != GLA_OK) return st;
-  if (cudaMemcpyAsync(out_h, dout, big, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return GLA_ERR_CUDA;
-  return GLA_OK;
+  return staged_step(
+      q_h, k_h, v_h, beta_h, g_h, out_h, batch, heads, head_dim, T_blk, H, W, dtype, arena,
+      arena_bytes, need, stream,
+      [&](const void* dq, const void* dk, const void* dv, const void* db, const void* dg,
+          void* dout, void* dws, size_t ws_bytes) {
+        return gla_block_causal_step(state, z, dq, dk, dv, db, dg, batch, heads, head_dim,
+                                     T_blk, H, W, t0, rope_theta, eps, dtype, dout, dws,
+                                     ws_bytes, stream);
+      });
+}
+
+size_t gla_causal_host_arena_size(int batch, int heads, int head_dim, int T, int H, int W,
+                                  int dtype) {
+  const size_t ws = gla_causal_workspace_size(batch, heads, head_dim, T, H, W, dtype);
+  if (!ws) return 0;
+  return staged_inputs_bytes(batch, heads, head_dim, T, H, W, dtype) + ws;
+}
+
+gla_status gla_causal_step_host(float* state, float* z, const void* q_h, const void* k_h,
+                                const void* v_h, const void* beta_h, const void* g_h, int batch,
+                                int heads, int head_dim, int T, int H, int W, int t0,
+                                float rope_theta, float eps, int dtype, void* out_h,
+                                void* arena, size_t arena_bytes, void* stream) {
+  const size_t need = gla_causal_host_arena_size(batch, heads, head_dim, T, H, W, dtype);
+  if (!need) return GLA_ERR_INVALID_ARG;
+  return staged_step(
+      q_h, k_h, v_h, beta_h, g_h, out_h, batch, heads, head_dim, T, H, W, dtype, arena,
+      arena_bytes, need, stream,
+      [&](const void* dq, const void* dk, const void* dv, const void* db, const void* dg,
+          void* dout, void* dws, size_t ws_bytes) {
+        return gla_causal_step(state, z, dq, dk, dv, db, dg, batch, heads, head_dim, T, H, W,
+                               t0, rope_theta, eps, dtype, dout, dws, ws_bytes, stream);
+      });
 }
 
 // ---------------------------------------------------------------------------

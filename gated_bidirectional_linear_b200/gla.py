@@ -40,6 +40,14 @@ _SIGS = {
     "gla_forward_host": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
     "gla_block_causal_host_arena_size": (_sz, [_i] * 7),
     "gla_block_causal_step_host": (_i, [_vp] * 7 + [_i] * 7 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
+    "gla_causal_workspace_size": (_sz, [_i] * 7),
+    "gla_causal_step": (_i, [_vp] * 7 + [_i] * 7 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
+    "gla_causal_step_ex": (_i, [_vp] * 7 + [_i] * 7 + [_f, _f, _i, _vp, _vp, _sz, _vp, _i]
+                           + [_vp] * 2),
+    "gla_causal_step_timed": (_i, [_vp] * 7 + [_i] * 7 + [_f, _f, _i, _vp, _vp, _sz, _vp, _i]
+                              + [_vp] * 2 + [ctypes.POINTER(_vp)]),
+    "gla_causal_host_arena_size": (_sz, [_i] * 7),
+    "gla_causal_step_host": (_i, [_vp] * 7 + [_i] * 7 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
     "gla_forward_noalloc": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp]),
     "gla_get_device_status": (_i, [_vp]),
     "gla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
@@ -287,13 +295,32 @@ def gla_block_causal_host_arena_size(batch, heads, head_dim, T_blk, H, W, dtype)
     return lib().gla_block_causal_host_arena_size(batch, heads, head_dim, T_blk, H, W, dtype)
 
 
+def gla_causal_host_arena_size(batch, heads, head_dim, T, H, W, dtype):
+    return lib().gla_causal_host_arena_size(batch, heads, head_dim, T, H, W, dtype)
+
+
 def gla_block_causal_step_host(state, z, q, k, v, beta, g, T_blk, H, W, t0, rope_theta=10000.0,
                                eps=1e-6, out=None, arena=None, stream=None):
     """One block-causal step on host tensors (pin them for asynchronous
     copies): the block's inputs go to the device `arena`, the step updates the
     device-resident state and z in place, and the block's output comes back
     into `out`.  Asynchronous on `stream`; synchronise before reading `out`."""
-    B, Hh, d = _dims(q, T_blk, H, W)
+    return _staged("gla_block_causal_step_host", "gla_block_causal_host_arena_size", state, z,
+                   q, k, v, beta, g, T_blk, H, W, t0, rope_theta, eps, out, arena, stream)
+
+
+def gla_causal_step_host(state, z, q, k, v, beta, g, T, H, W, t0=0, rope_theta=10000.0,
+                         eps=1e-6, out=None, arena=None, stream=None):
+    """gla_causal_step on host tensors (pin them for asynchronous copies), the
+    state (state, z) resident on the GPU and updated in place.  Asynchronous
+    on `stream`; synchronise before reading `out`."""
+    return _staged("gla_causal_step_host", "gla_causal_host_arena_size", state, z, q, k, v,
+                   beta, g, T, H, W, t0, rope_theta, eps, out, arena, stream)
+
+
+def _staged(entry, arena_size, state, z, q, k, v, beta, g, T, H, W, t0, rope_theta, eps, out,
+            arena, stream):
+    B, Hh, d = _dims(q, T, H, W)
     code = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
@@ -305,17 +332,87 @@ def gla_block_causal_step_host(state, z, q, k, v, beta, g, T_blk, H, W, t0, rope
         if tuple(t.shape) != shape or t.dtype != torch.float32 or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous fp32 tensor of shape {shape}")
     if arena is None:
-        arena = alloc_workspace(gla_block_causal_host_arena_size(B, Hh, d, T_blk, H, W, code),
-                                dev)
+        arena = alloc_workspace(getattr(lib(), arena_size)(B, Hh, d, T, H, W, code), dev)
     if arena.device != dev or arena.dtype != torch.uint8 or not arena.is_contiguous():
         raise ValueError(f"arena must be a contiguous uint8 tensor on {dev}")
     with _on(dev):
-        st = lib().gla_block_causal_step_host(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v),
-                                              _ptr(beta), _ptr(g), B, Hh, d, T_blk, H, W, t0,
-                                              rope_theta, eps, code, _ptr(out), _ptr(arena),
-                                              arena.numel(), _stream(stream, dev))
-    _check(st, "gla_block_causal_step_host")
+        st = getattr(lib(), entry)(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                   _ptr(g), B, Hh, d, T, H, W, t0, rope_theta, eps, code,
+                                   _ptr(out), _ptr(arena), arena.numel(), _stream(stream, dev))
+    _check(st, entry)
     return out
+
+
+def gla_causal_workspace_size(batch, heads, head_dim, T, H, W, dtype):
+    return lib().gla_causal_workspace_size(batch, heads, head_dim, T, H, W, dtype)
+
+
+def gla_causal_step(state, z, q, k, v, beta, g, T, H, W, t0=0, rope_theta=10000.0, eps=1e-6,
+                    out=None, workspace=None, stream=None, path=GLA_PATH_AUTO, den_out=None,
+                    x_out=None):
+    """Token-level causal read-out of one segment of a sequence: token j sees
+    the carried (state, z) plus tokens 0..j of this call; (state, z) are
+    updated in place to the sums after the call.  state [B,Hh,d,d], z [B,Hh,d]
+    fp32 on the GPU; den_out [B,N,Hh] / x_out [B,N,Hh,d] fp32 optional exports."""
+    B, Hh, d = _dims(q, T, H, W)
+    N = q.shape[1]
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    extra = dict(state=(state, (B, Hh, d, d), torch.float32), z=(z, (B, Hh, d), torch.float32))
+    if den_out is not None:
+        extra["den_out"] = (den_out, (B, N, Hh), torch.float32)
+    if x_out is not None:
+        extra["x_out"] = (x_out, (B, N, Hh, d), torch.float32)
+    _validate(q, k, v, beta, g, out, **extra)
+    if workspace is None:
+        workspace = alloc_workspace(gla_causal_workspace_size(B, Hh, d, T, H, W, code), q.device)
+    _check_workspace(workspace, q.device)
+    with _on(q.device):
+        st = lib().gla_causal_step_ex(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v),
+                                      _ptr(beta), _ptr(g), B, Hh, d, T, H, W, t0, rope_theta,
+                                      eps, code, _ptr(out), _ptr(workspace), workspace.numel(),
+                                      _stream(stream, q.device), path, _ptr(den_out),
+                                      _ptr(x_out))
+    _check(st, "gla_causal_step")
+    return out
+
+
+def gla_causal_step_timed(state, z, q, k, v, beta, g, T, H, W, events, t0=0,
+                          rope_theta=10000.0, eps=1e-6, out=None, workspace=None, stream=None,
+                          path=GLA_PATH_AUTO):
+    """gla_causal_step recording four torch.cuda.Event objects around its
+    kernels (before the state partials, after them, after their prefix,
+    after the causal read-out)."""
+    B, Hh, d = _dims(q, T, H, W)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out, state=(state, (B, Hh, d, d), torch.float32),
+              z=(z, (B, Hh, d), torch.float32))
+    if workspace is None:
+        workspace = alloc_workspace(gla_causal_workspace_size(B, Hh, d, T, H, W, code), q.device)
+    _check_workspace(workspace, q.device)
+    ev = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) if e is not None else None
+                                 for e in events])
+    with _on(q.device):
+        st = lib().gla_causal_step_timed(_ptr(state), _ptr(z), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(beta), _ptr(g), B, Hh, d, T, H, W, t0, rope_theta,
+                                         eps, code, _ptr(out), _ptr(workspace),
+                                         workspace.numel(), _stream(stream, q.device), path,
+                                         None, None, ev)
+    _check(st, "gla_causal_step_timed")
+    return out
+
+
+def gla_causal_forward(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, out=None,
+                       workspace=None, stream=None, path=GLA_PATH_AUTO):
+    """The causal read-out of a whole sequence (zero state before it)."""
+    B, Hh, d = _dims(q, T, H, W)
+    state = torch.zeros(B, Hh, d, d, dtype=torch.float32, device=q.device)
+    z = torch.zeros(B, Hh, d, dtype=torch.float32, device=q.device)
+    return gla_causal_step(state, z, q, k, v, beta, g, T, H, W, 0, rope_theta, eps, out=out,
+                           workspace=workspace, stream=stream, path=path)
 
 
 def gla_forward_noalloc(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, out=None,

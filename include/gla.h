@@ -180,6 +180,77 @@ GLA_API gla_status gla_block_causal_step_ex(float* state, float* z, const void* 
                                     void* out, void* workspace, size_t workspace_bytes,
                                     void* stream, int path);
 
+/* Workspace bytes of gla_causal_step / gla_causal_step_ex (the tensor path's
+ * state partials and per-partial starting states; independent of the GPU). */
+GLA_API size_t gla_causal_workspace_size(int batch, int heads, int head_dim, int T, int H,
+                                         int W, int dtype);
+
+/* Token-level causal variant over one call of T*H*W tokens, continuing a
+ * sequence (SANA-Video notes, key design 2: causal linear attention needs only
+ * the running sums of the per-token states v_n (beta_n k_til_n)^T and of the
+ * key features k_pls_n).  Token j is read out against
+ *   S_j = state + sum_{n <= j} v_n (beta_n k_til_n)^T,
+ *   z_j = z     + sum_{n <= j} k_pls_n              (a token sees itself),
+ * with den_j = z_j . q_pls_j + eps and the rest of the read-out as in
+ * gla_forward.  state [batch][heads][d][d] fp32 and z [batch][heads][d] fp32
+ * are caller-owned device memory holding the sums before the call's first
+ * token (zero them to start a sequence); on return they hold the sums after
+ * its last token, so consecutive calls over consecutive segments give the
+ * causal read-out of the whole sequence.  RoPE time positions are t0 + local
+ * frame.  Workspace: gla_causal_workspace_size() bytes, 256-byte aligned (the
+ * CUDA-core path uses none and accepts NULL).  Other layouts, errors and
+ * stream semantics as for gla_forward; the state is reduced in a fixed order,
+ * so results are bitwise reproducible. */
+GLA_API gla_status gla_causal_step(float* state, float* z, const void* q, const void* k,
+                                   const void* v, const void* beta, const void* g, int batch,
+                                   int heads, int head_dim, int T, int H, int W, int t0,
+                                   float rope_theta, float eps, int dtype, void* out,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* gla_causal_step with an explicit path (gla_path) and optional exports of the
+ * hidden intermediates (tests): den_out [batch][N][heads] fp32 (den_j) and
+ * x_out [batch][N][heads][d] fp32 (sigmoid(g_j) * S_j q_til_j / den_j, before
+ * the output RMSNorm); either may be NULL. */
+GLA_API gla_status gla_causal_step_ex(float* state, float* z, const void* q, const void* k,
+                                      const void* v, const void* beta, const void* g,
+                                      int batch, int heads, int head_dim, int T, int H, int W,
+                                      int t0, float rope_theta, float eps, int dtype, void* out,
+                                      void* workspace, size_t workspace_bytes, void* stream,
+                                      int path, float* den_out, float* x_out);
+
+/* gla_causal_step_ex that also records caller-created CUDA events (cudaEvent_t
+ * passed as void*) on `stream` around the tensor path's kernels: events[0]
+ * before the state partials, events[1] after them, events[2] after their
+ * prefix, events[3] after the causal read-out (the CUDA-core path records
+ * events[0] only).  For per-kernel timing in benchmarks; `events` and any of
+ * its entries may be NULL. */
+GLA_API gla_status gla_causal_step_timed(float* state, float* z, const void* q, const void* k,
+                                         const void* v, const void* beta, const void* g,
+                                         int batch, int heads, int head_dim, int T, int H, int W,
+                                         int t0, float rope_theta, float eps, int dtype,
+                                         void* out, void* workspace, size_t workspace_bytes,
+                                         void* stream, int path, float* den_out, float* x_out,
+                                         void* const* events);
+
+/* Bytes of the device arena gla_causal_step_host needs: room for the call's
+ * five inputs, its output and its workspace. */
+GLA_API size_t gla_causal_host_arena_size(int batch, int heads, int head_dim, int T, int H,
+                                          int W, int dtype);
+
+/* gla_causal_step on HOST buffers: q_h .. g_h and out_h are host memory
+ * (pinned memory gives asynchronous copies); state and z stay in the caller's
+ * DEVICE memory, carried between calls.  Enqueues on `stream` the
+ * host-to-device copies of the inputs into the caller's device `arena` (at
+ * least gla_causal_host_arena_size() bytes, 256-byte aligned), the step, and
+ * the device-to-host copy of the output; returns after enqueueing.  The output
+ * equals gla_causal_step's on the same inputs bit for bit. */
+GLA_API gla_status gla_causal_step_host(float* state, float* z, const void* q_h, const void* k_h,
+                                        const void* v_h, const void* beta_h, const void* g_h,
+                                        int batch, int heads, int head_dim, int T, int H, int W,
+                                        int t0, float rope_theta, float eps, int dtype,
+                                        void* out_h, void* arena, size_t arena_bytes,
+                                        void* stream);
+
 /* Bytes of the device arena gla_forward_host needs: room for the five inputs,
  * the output and the workspace. */
 GLA_API size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, int T, int H, int W,
