@@ -497,8 +497,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
     if (iw.more()) fetch_beta(iw);
     for (; iw.more(); iw.next(), rq.next(), ++it) {
       const int s = rq.s;
-      bool ok = mbar_wait(&qkfree[s], rq.ph ^ 1u, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!mbar_wait_warp(&qkfree[s], rq.ph ^ 1u, abort_flag)) break;
       const int b = iw.b, h = iw.h, n0 = iw.ti * kCaTile;
       if (lane == 0) {
         mbar_arrive_expect_tx(&qkfull[s], 2 * kCaTileBytes);
@@ -526,8 +525,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         tile_rowrec<kCaTile>(g, win, n0, lane, sm + TcCausalSmem::ROWREC + s * kCaTile * kRecBytes);
       __syncwarp();
       if (lane == 0) mbar_arrive(&qkfull[s]);
-      ok = mbar_wait(vfree, (uint32_t)((it & 1) ^ 1), abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!mbar_wait_warp(vfree, (uint32_t)((it & 1) ^ 1), abort_flag)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(vfull, kCaTileBytes);
         unsigned char* vt = sm + TcCausalSmem::V;
@@ -649,9 +647,9 @@ __global__ void __launch_bounds__(kCaThreads, 1)
           zr[2 * q + 1] = f2(t.z, t.w);
         }
       }
-      bool ok = mbar_wait(&qkfull[s], rq.ph, abort_flag);
-      ok = ok && mbar_wait(kffree, (uint32_t)((i & 1) ^ 1), abort_flag);
-      ok = ok && mbar_wait(&denfree[s], rq.ph ^ 1u, abort_flag);
+      bool ok = mbar_wait_warp(&qkfull[s], rq.ph, abort_flag);
+      ok = ok && mbar_wait_warp(kffree, (uint32_t)((i & 1) ^ 1), abort_flag);
+      ok = ok && mbar_wait_warp(&denfree[s], rq.ph ^ 1u, abort_flag);
       if (!bar_red_and(2, kCaTW * 32, ok && !*abort_flag)) break;
       const uint32_t qt = sbase + TcCausalSmem::Q + s * kCaTileBytes;
       const uint32_t kt = sbase + TcCausalSmem::K + s * kCaTileBytes;
@@ -812,8 +810,9 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(imgready);
       }
-      // (a) P = mask(A) * scale, over the chunk's q slot.
-      ok = ok && mbar_wait(afull, par, abort_flag);
+      // (a) P = mask(A) * scale, over the chunk's q slot.  Wait outcomes are
+      // made warp-uniform: the tcgen05 loads below are warp-collective.
+      ok = ok && mbar_wait_warp(afull, par, abort_flag);
       if (ok && row < kCaTile) {
         tc_fence_after();
         const uint32_t pslot = sbase + TcCausalSmem::Q + s * kCaTileBytes;
@@ -846,7 +845,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
       if (lane == 0) mbar_arrive(pready);
       // (c) the image of the state after the chunk, for the next chunk of
       // the segment.
-      ok = ok && mbar_wait(sfull, par, abort_flag);
+      ok = ok && mbar_wait_warp(sfull, par, abort_flag);
       tc_fence_after();
       const float chunk_scale = cur_scale;
       if (!iw.last) {
@@ -860,13 +859,14 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         if (!ok) break;
       }
       // (d) the read-out: x = sigmoid(g) * U / (den * scale), RMSNorm, bf16.
-      ok = mbar_wait(&ufull[s], rq.ph, abort_flag);
+      ok = mbar_wait_warp(&ufull[s], rq.ph, abort_flag);
       const int n = n0 + row;
-      if (ok && row < kCaTile && n < g.N) {
+      const bool valid = n < g.N;   // per lane: guards global memory only
+      if (ok && row < kCaTile) {
         tc_fence_after();
         const float hc = 0.5f / (den_ring[s * kCaTile + row] * chunk_scale);
         const uint32_t tU = tmem + kCaTmU + (uint32_t)s * 128u + lane_off;
-        const size_t rowoff = (((size_t)b * g.N + n) * g.Hh + h) * 128;
+        const size_t rowoff = (((size_t)b * g.N + (valid ? n : 0)) * g.Hh + h) * 128;
         const __nv_bfloat16* grow = p.gate + rowoff;
         const f2_t hc2 = f2(hc, hc), half2 = f2(0.5f, 0.5f);
         f2_t ss2 = 0ull;
@@ -874,7 +874,8 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         for (int cb = 0; cb < 4; ++cb) {
           uint4 gv[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) gv[q] = ldg_nc128(grow + cb * 32 + 8 * q);
+          for (int q = 0; q < 4; ++q)
+            gv[q] = valid ? ldg_nc128(grow + cb * 32 + 8 * q) : make_uint4(0u, 0u, 0u, 0u);
           float u[32];
           tmem_ld32(tU + cb * 32, u);
           tmem_wait_ld();
@@ -892,7 +893,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
               u[q * 8 + 2 * e + 1] = f2_hi(x);
             }
           }
-          if (kDebug && p.x_out) {
+          if (kDebug && p.x_out && valid) {
             float* xo = p.x_out + rowoff + cb * 32;
 #pragma unroll
             for (int i2 = 0; i2 < 32; i2 += 4)
@@ -917,7 +918,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
               const f2_t y = f2_mul(f2(x[q * 8 + 2 * e], x[q * 8 + 2 * e + 1]), rstd2);
               o[e] = pack_bf16(f2_lo(y), f2_hi(y));
             }
-            stg128(orow + cb * 32 + 8 * q, make_uint4(o[0], o[1], o[2], o[3]));
+            if (valid) stg128(orow + cb * 32 + 8 * q, make_uint4(o[0], o[1], o[2], o[3]));
           }
         }
       }

@@ -101,6 +101,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
+// mbar_wait for a whole warp: every lane gets the same answer (false if any
+// lane gave up), so that a warp leaves its loop together and never reaches a
+// warp-collective instruction (shuffles, tcgen05 loads) with lanes missing.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+
 // ------------------------------------------------ programmatic dependent launch
 
 // Let the next kernel of the stream (launched with programmatic stream

@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       if (iw.more()) fetch_beta(iw);
       for (; iw.more(); iw.next(), rp.next(), ++it) {
         const int s = rp.s;
-        if (!mbar_wait(&empty[s], rp.ph ^ 1u, abort_flag)) break;
+        if (!mbar_wait_warp(&empty[s], rp.ph ^ 1u, abort_flag)) break;
         const int b = iw.b, h = iw.h;
         const int n0 = iw.ti * kStTile;
         // Lane 0 starts the tile copies first; then the warp stores beta,
@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       const int s = rp.s;
       const uint32_t ph = rp.ph;
       const int bh = iw.bh;
-      if (!mbar_wait(&full[s], ph, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&full[s], ph, abort_flag)) { ok = false; break; }
       const uint32_t kt = sbase + TcStateSmem::K + s * kStTileBytes;
       const float* bs = reinterpret_cast<const float*>(sm + TcStateSmem::BETA + s * kStTile * 4);
       const uint32_t rec_s = sbase + TcStateSmem::ROWREC + s * kStTile * kRecBytes;
@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
           const int third = tw >> 2;
           const int a = q4 * 32 + lane;
           const int ab = seg & 1;
-          if (!mbar_wait(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag)) { ok = false; break; }
           tc_fence_after();
           // Chunk-major partial: columns 8cb .. 8cb+7 of row a at (cb * 128 + a) * 8,
           // so the warp's 32 rows of a chunk are 1 KB of contiguous stores.
@@ -744,7 +744,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
           ahead.next();
         }
         const int s = rq.s;
-        if (!mbar_wait(&qempty[s], rq.ph ^ 1u, abort_flag)) break;
+        if (!mbar_wait_warp(&qempty[s], rq.ph ^ 1u, abort_flag)) break;
         const int n0 = iw.ti * kTcTile;
         if (g.rope_on)
           tile_rowrec<kTcTile>(g, win, n0, lane, sm + TcApplySmem::ROWREC + s * kTcTile * kRecBytes);
@@ -762,7 +762,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
             combined = true;
           }
           // Every lane waits, so the warp leaves the loop together on a timeout.
-          if (!mbar_wait(sfree, (uint32_t)((seg & 1) ^ 1), abort_flag)) break;
+          if (!mbar_wait_warp(sfree, (uint32_t)((seg & 1) ^ 1), abort_flag)) break;
           if (lane == 0) {
             // Smallest first: z and the scale (the transform warps' only
             // dependence on the combine), the RoPE table, then the S image.
@@ -886,7 +886,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
     // ------------------------------------ transform warps: q -> q_til, den
     // The RoPE table comes by bulk copy from the whole-call table that the
     // state kernel's producer warps write.
-    const bool tab_ok = wb >= we || mbar_wait(tfull, 0u, abort_flag);
+    const bool tab_ok = wb >= we || mbar_wait_warp(tfull, 0u, abort_flag);
     const int tw = warp - kApTW0;
     const int rg = tw_row(lane), j = tw_chunk(lane);
     LaneRope lr;
@@ -902,14 +902,14 @@ __global__ void __launch_bounds__(kApThreads, 1)
     for (; tab_ok && iw.more(); iw.next(), rq.next(), rd.next()) {
       const int b = iw.b, h = iw.h;
       if (iw.first) {
-        if (!mbar_wait(zfull, (uint32_t)(seg & 1), abort_flag)) break;
+        if (!mbar_wait_warp(zfull, (uint32_t)(seg & 1), abort_flag)) break;
 #pragma unroll
         for (int i = 0; i < 8; ++i) zr[i] = f2(zs[16 * j + 2 * i], zs[16 * j + 2 * i + 1]);
         hscale = scl_s[0];
         ++seg;
       }
       const int s = rq.s;
-      if (!mbar_wait(&qfull[s], rq.ph, abort_flag)) break;
+      if (!mbar_wait_warp(&qfull[s], rq.ph, abort_flag)) break;
       const int n0 = iw.ti * kTcTile;
       const uint32_t qt = sbase + TcApplySmem::Q + s * kTileBytes;
       float* den = den_ring + rd.s * 128;
@@ -983,10 +983,10 @@ __global__ void __launch_bounds__(kApThreads, 1)
       const int b = iw.b, h = iw.h;
       const int n0 = iw.ti * kTcTile;
       const int ab = ra.s;
-      if (!mbar_wait(&accfull[ab], ra.ph, abort_flag)) break;
+      if (!mbar_wait_warp(&accfull[ab], ra.ph, abort_flag)) break;
       tc_fence_after();
       const int gsl = rg_.s;
-      if (!mbar_wait(&gfull[gsl], rg_.ph, abort_flag)) break;
+      if (!mbar_wait_warp(&gfull[gsl], rg_.ph, abort_flag)) break;
       // sigma(g) / den' = (0.5 tanh(g/2) + 0.5) / den' = fma(hc, tanh(g/2), hc)
       const float hc = 0.5f / den_ring[rd.s * 128 + row];
       const uint32_t taddr = tmem + (uint32_t)(ab * 128) + ((uint32_t)(q4 * 32) << 16);
