@@ -419,3 +419,15 @@ def bf16_out_err_over_rms(got, ref):
     ref = np.asarray(ref, dtype=np.float64)
     excess = np.maximum(np.abs(got - ref) - bf16_half_ulp(ref), 0.0)
     return float(np.max(excess) / np.sqrt(np.mean(ref * ref)))
+
+
+def max_err_over_row_rms(got, ref):
+    """max over rows r and elements i of |got_ri - ref_ri| / rms(ref_r), rows
+    being the last axis (a token's d channels): the error relative to each
+    token's own RMS.  The causal read-out's pre-norm values differ in scale
+    from token to token (an early token averages few values), so its
+    tolerance is stated per token, as the output's is after its RMSNorm."""
+    ref = np.asarray(ref, dtype=np.float64)
+    got = np.asarray(got, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
+    return float(np.max(np.abs(got - ref) / rms))

@@ -46,6 +46,11 @@ def rel_floor(got, ref):
     return O.max_rel_err_rms_floor(got, ref)
 
 
+def rel_row_rms(got, ref):
+    """Error over each token's own RMS (the oracle's max_err_over_row_rms)."""
+    return O.max_err_over_row_rms(got, ref)
+
+
 def bf16_half_ulp(ref):
     """Half the spacing of bf16 numbers at |ref| (the oracle's metric helper)."""
     return O.bf16_half_ulp(ref)

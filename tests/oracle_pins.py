@@ -486,6 +486,17 @@ def check_metric_rel_rms_floor():
     _close(O.max_rel_err_rms_floor(got, _REF4), 0.5, 1e-12, "rel err above the RMS")
 
 
+def check_metric_row_rms():
+    """Per-row errors over per-row RMS: rows (3, -4, 0, 0) (rms 2.5) and
+    (30, -40, 0, 0) (rms 25) with errors (0, 0.5, 0, 0) and (1, 0, 0, -2)
+    give max(0.5/2.5, 2/25) = 0.2; a global RMS would give 2/17.77."""
+    ref = np.array([[3.0, -4.0, 0.0, 0.0], [30.0, -40.0, 0.0, 0.0]])
+    got = ref + np.array([[0.0, 0.5, 0.0, 0.0], [1.0, 0.0, 0.0, -2.0]])
+    _close(O.max_err_over_row_rms(got, ref), 0.2, 1e-12, "row-RMS metric")
+    got = ref + np.array([[0.0, 0.0, 0.0, 0.0], [0.0, 0.0, 0.0, -5.0]])
+    _close(O.max_err_over_row_rms(got, ref), 0.2, 1e-12, "row-RMS metric, second row")
+
+
 def check_metric_bf16_half_ulp():
     """Half the bf16 spacing (8 significant bits) at hand-picked values, then
     against torch's round-to-nearest-even bf16 conversion: a value halfway

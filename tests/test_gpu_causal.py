@@ -1,7 +1,9 @@
 """Token-level causal variant (gla_causal_step) against the fp64 oracle.
 
 Small shapes are compared on every output and on the exported denominator and
-pre-norm read-out (oracle.causal_forward, running sums); the 480p shape on
+pre-norm read-out (oracle.causal_forward, running sums); the pre-norm read-out
+is measured against each token's own RMS, since its scale varies from token
+to token (an early token averages a few values, a late one many); the 480p shape on
 every token of sampled heads; the full 720p shape on sampled tokens of sampled
 heads, each recomputed by the oracle from its own prefix
 (oracle.causal_forward_at).  The state after the call is compared with the
@@ -14,7 +16,7 @@ import torch
 import oracle.gla_oracle as O
 from gated_bidirectional_linear_b200 import gla, workloads
 from gpu_common import (BF16_TOL, F32_TOL, S_TOL_BF16, ZDEN_TOL, head_slice, np64, rel_elem,
-                        rel_floor, rel_rms, rel_rms_bf16out, to_device)
+                        rel_floor, rel_rms, rel_rms_bf16out, rel_row_rms, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -50,7 +52,7 @@ def _check(got, ref, dtype):
         assert rel_floor(got["S"], ref["S"]) <= F32_TOL
     else:
         assert rel_rms_bf16out(got["out"], ref["out"]) <= BF16_TOL
-        assert rel_rms(got["x"], ref["x"]) <= BF16_TOL
+        assert rel_row_rms(got["x"], ref["x"]) <= BF16_TOL
         assert rel_floor(got["S"], ref["S"]) <= S_TOL_BF16
     assert rel_floor(got["z"], ref["z"]) <= ZDEN_TOL
     assert rel_elem(got["den"], ref["den"]) <= ZDEN_TOL
@@ -103,7 +105,7 @@ def test_480p_sampled_heads_every_token(c480, path):
         sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
         worst["out"] = max(worst["out"], rel_rms_bf16out(got["out"][sl], ref["out"]))
         worst["raw"] = max(worst["raw"], rel_rms(got["out"][sl], ref["out"]))
-        worst["x"] = max(worst["x"], rel_rms(got["x"][sl], ref["x"]))
+        worst["x"] = max(worst["x"], rel_row_rms(got["x"][sl], ref["x"]))
         worst["den"] = max(worst["den"], rel_elem(got["den"][sl], ref["den"]))
     # the state after the call, every head
     x = workloads.as_f64(inp)
@@ -164,7 +166,8 @@ def test_streaming_two_calls_equal_one():
              z=torch.from_numpy(a["z"]).float())
     both = np.concatenate([a["out"], b["out"]], axis=1)
     assert rel_rms(both, one["out"]) <= BF16_TOL
-    assert rel_floor(b["S"], one["S"]) <= 1e-5
+    # the same fp32 sums grouped differently (two partitions of the tokens)
+    assert rel_floor(b["S"], one["S"]) <= 1e-4
     x = workloads.as_f64(inp)
     ref = O.causal_forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T, H, W, 1e4, 1e-6)
     assert rel_rms_bf16out(both, ref["out"]) <= BF16_TOL
@@ -183,7 +186,7 @@ def test_tensor_and_cuda_core_paths_agree(c480):
     wl, inp = c480
     a = _run(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, TENSOR)
     b = _run(inp, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, SIMT)
-    assert rel_rms(a["x"], b["x"]) <= BF16_TOL
+    assert rel_row_rms(a["x"], b["x"]) <= BF16_TOL
     assert rel_elem(a["den"], b["den"]) <= ZDEN_TOL
 
 

@@ -259,7 +259,17 @@ def _bf16out_full_ulp(got, ref):
     return float(np.max(excess) / np.sqrt(np.mean(ref * ref)))
 
 
+def _row_rms_global(got, ref):
+    return _orig["max_err_over_rms"](got, ref)
+
+
+def _row_rms_of_got(got, ref):
+    return _orig["max_err_over_row_rms"](ref, got)
+
+
 METRIC_MUTANTS = {
+    "row_rms_global": (O, "max_err_over_row_rms", _row_rms_global),
+    "row_rms_of_got": (O, "max_err_over_row_rms", _row_rms_of_got),
     "err_rms_of_got": (O, "max_err_over_rms", _rms_of_got),
     "err_no_abs": (O, "max_err_over_rms", _err_no_abs),
     "err_mean_abs": (O, "max_err_over_rms", _err_mean_abs),
