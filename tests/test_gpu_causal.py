@@ -38,7 +38,7 @@ def _run(inp, T, H, W, theta, eps, path, t0=0, state=None, z=None):
 
 
 def _oracle(inp, T, H, W, theta, eps, t0=0):
-    x = workloads.as_f64(inp)
+    x = inp if isinstance(inp["q"], np.ndarray) else workloads.as_f64(inp)
     r = O.causal_forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T, H, W, theta, eps, t0)
     f = O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T, H, W, theta, eps, t0)
     r.update(S=f["S"], z=f["z"])       # the state after the last token
