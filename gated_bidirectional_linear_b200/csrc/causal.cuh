@@ -177,9 +177,8 @@ __global__ void __launch_bounds__(kSimtCausalThreads) simt_causal_kernel(SimtCau
 
 struct PrefixParams {
   Partition part;
-  int zparts;            // z partials per slot, added in index order
   const float* part_S;   // [slots][128*128] chunk-major partials (tc_state_kernel)
-  const float* part_z;   // [slots][zparts][128]
+  const float* part_z;   // [slots][kStTW][128], added in index order
   const float* S_in;     // carried state [BH][128][128] row-major (may alias S_out)
   const float* z_in;     // [BH][128] (may alias z_out)
   float* S_start;        // [slots][128*128] chunk-major: the state before the slot
@@ -244,12 +243,17 @@ __global__ void __launch_bounds__(kPrefixThreads) combine_prefix_kernel(PrefixPa
     *reinterpret_cast<float4*>(p.S_out + (size_t)bh * dd + row_major(e)) = acc[k];
   }
   if (slice == 0 && threadIdx.x < 128) {
+    // A slot's kStTW z partials are loaded together, then added in order.
     const int t = threadIdx.x;
     float zr = p.z_in ? p.z_in[(size_t)bh * 128 + t] : 0.f;
     for (int c = c_lo; c <= c_hi; ++c) {
       const size_t slot = (size_t)c + bh;
+      float zp[kStTW];
+#pragma unroll
+      for (int w = 0; w < kStTW; ++w) zp[w] = p.part_z[(slot * kStTW + w) * 128 + t];
       p.z_start[slot * 128 + t] = zr;
-      for (int w = 0; w < p.zparts; ++w) zr += p.part_z[(slot * p.zparts + w) * 128 + t];
+#pragma unroll
+      for (int w = 0; w < kStTW; ++w) zr += zp[w];
     }
     p.z_out[(size_t)bh * 128 + t] = zr;
   }
@@ -260,14 +264,18 @@ __global__ void __launch_bounds__(kPrefixThreads) combine_prefix_kernel(PrefixPa
 constexpr int kCaTile = kStTile;                 // tokens per chunk: the state partition's tile
 constexpr uint32_t kCaBox = kStBox;              // 96 rows x 128 bytes
 constexpr uint32_t kCaTileBytes = kStTileBytes;  // two boxes
-constexpr int kCaTW = 8;                         // transform warps 2..9
+constexpr int kCaTW = 6;                         // transform warps 2..7
 constexpr int kCaTW0 = 2;
-constexpr int kCaEW0 = kCaTW0 + kCaTW;           // epilogue warps 10..13
-constexpr int kCaEW = 4;
-constexpr int kCaThreads = (kCaEW0 + kCaEW) * 32;
-constexpr int kCaGroups = kCaTile / (kCaTW * 4); // row groups of 4 per transform warp
-static_assert(kCaGroups * kCaTW * 4 == kCaTile, "whole row groups per chunk");
-static_assert((kCaTW * 4) % 8 == 0, "row groups keep the 8-row swizzle phase");
+constexpr int kCaEW0 = kCaTW0 + kCaTW;           // chain warps 8..11: P and the state image
+constexpr int kCaEW = 4;                         // one per TMEM lane quarter
+constexpr int kCaOW0 = kCaEW0 + kCaEW;           // output warps 12..14: lane quarters 0..2
+constexpr int kCaOW = kCaTile / 32;              // (rows 0..95)
+constexpr int kCaThreads = (kCaOW0 + kCaOW) * 32;
+static_assert(kCaEW0 % 4 == 0 && kCaOW0 % 4 == 0, "role warps start on a lane quarter");
+constexpr int kCaRowsW = kCaTile / kCaTW;         // contiguous rows per transform warp
+constexpr int kCaGroups = kCaRowsW / 4;          // its row groups of 4
+static_assert(kCaGroups * 4 * kCaTW == kCaTile, "whole row groups per chunk");
+static_assert(kCaRowsW % 8 == 0, "a warp's rows start on the 8-row swizzle phase");
 
 // TMEM columns: A = Q_til (beta K_til)^T, two read-out accumulators U, the state.
 constexpr uint32_t kCaTmA = 0, kCaTmU = 128, kCaTmS = 384;
@@ -281,9 +289,11 @@ struct TcCausalSmem {
   static constexpr uint32_t ROWREC = SIMG + kTileBytes;         // [2][96] RoPE row records
   static constexpr uint32_t BETA = ROWREC + 2 * kCaTile * kRecBytes;   // [2][96] f32
   static constexpr uint32_t DEN = BETA + 2 * kCaTile * 4;      // [2][96] f32
-  static constexpr uint32_t GTOT = DEN + 2 * kCaTile * 4;      // [2][8 warps][128] f32 group sums
-  static constexpr uint32_t RED = GTOT + 2 * kCaTW * 128 * 4;   // [2][4] f32 image maxima
-  static constexpr uint32_t BAR = RED + 32;
+  static constexpr uint32_t GTOT = DEN + 2 * kCaTile * 4;      // [2][warp][128] f32 key sums
+  static constexpr uint32_t ZRUN = GTOT + 2 * kCaTW * 128 * 4;  // [2][128] f32 key sum before a chunk
+  static constexpr uint32_t RED = ZRUN + 2 * 128 * 4;           // [2][4] f32 image maxima
+  static constexpr uint32_t SCL = RED + 32;                    // [4] f32 image scale per chunk
+  static constexpr uint32_t BAR = SCL + 16;
   static constexpr uint32_t NBAR = 19;
   static constexpr uint32_t MISC = BAR + NBAR * 8;
   static constexpr uint32_t TAB = (MISC + 16 + 15) & ~15u;
@@ -433,6 +443,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
   float2* tab = reinterpret_cast<float2*>(sm + TcCausalSmem::TAB);
   float* den_ring = reinterpret_cast<float*>(sm + TcCausalSmem::DEN);
   float* gtot = reinterpret_cast<float*>(sm + TcCausalSmem::GTOT);
+  float* zrun = reinterpret_cast<float*>(sm + TcCausalSmem::ZRUN);
   float* red = reinterpret_cast<float*>(sm + TcCausalSmem::RED);
 
   const Geom& g = p.g;
@@ -448,8 +459,8 @@ __global__ void __launch_bounds__(kCaThreads, 1)
       mbar_init(&qkfull[s], 2);
       mbar_init(&qkfree[s], 1);
       mbar_init(&ufull[s], 1);
-      mbar_init(&ufree[s], kCaEW);
-      mbar_init(&denfree[s], kCaEW);
+      mbar_init(&ufree[s], kCaOW);
+      mbar_init(&denfree[s], kCaOW);
     }
     mbar_init(vfull, 1);
     mbar_init(vfree, 1);
@@ -610,43 +621,37 @@ __global__ void __launch_bounds__(kCaThreads, 1)
   } else if (warp < kCaEW0) {
     // --------------------------------------------------- transform warps
     // q -> q_til (fp16), k -> beta k_til (bf16 in place, fp16 copy), and the
-    // denominator of every row from the running sum of k_pls.
+    // denominator of every row from the running sum of k_pls.  Warp tw owns
+    // the chunk's rows 16 tw .. 16 tw + 15 (four row groups of four).  A
+    // first pass sums the warp's k_pls; after one barrier each warp knows the
+    // key sum before its rows (the sum before the chunk plus the earlier
+    // warps' sums), and the main pass carries it row group by row group.
+    // Warp sums are stored with 16-byte chunk q of lane j at float4 index
+    // q * 8 + j, so that the 8 lanes that read one chunk read 128 contiguous
+    // bytes.
     rope_build(tab, g, win, threadIdx.x - kCaTW0 * 32, kCaTW * 32);
     named_barrier(1, kCaTW * 32);
     const int tw = warp - kCaTW0;
     const int rg = tw_row(lane), j = tw_chunk(lane);
     LaneRope lr;
     lane_rope(g, j, smem_u32(tab), lr);
-    uint32_t ch0, ch1;
-    lane_chunks(0, kCaBox, tw * 4 + rg, j, ch0, ch1);
-    // Lanes of the row group above: rg - 1 (rg = lane bit 2 | lane bit 4 << 1)
-    // and rg - 2.
+    // The lane's two 16-byte chunks in the first row of each group parity:
+    // rows 16 tw + 4 u + rg have swizzle phase 4 (u & 1) + rg.
+    uint32_t ch0[2], ch1[2];
+    lane_chunks(0, kCaBox, rg, j, ch0[0], ch1[0]);
+    lane_chunks(0, kCaBox, 4 + rg, j, ch0[1], ch1[1]);
+    // Lanes of the row group above: rg - 1 (rg = lane bit 2 | lane bit 4 << 1),
+    // rg - 2, and the group's last row (rg = 3).
     const int src1 = (rg & 1) ? (lane ^ 4) : (lane ^ 20);
     const int src2 = lane ^ 16;
-    f2_t zr[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) zr[i] = 0ull;
+    const int src3 = lane | 20;
     bool waited_grid = false;
-    uint32_t gpar = 0;
     ItemWalk iw(wb, we, tph, g.Hh);
     RingPos<2> rq;
     long long i = 0;
     for (; iw.more(); iw.next(), rq.next(), ++i) {
       const int s = rq.s;
-      if (iw.first) {
-        // The running key sum of the head starts at its slot's z_start.
-        if (!waited_grid) {
-          pdl_wait();
-          waited_grid = true;
-        }
-        const float* zs = p.z_start + ((size_t)c + iw.bh) * 128 + 16 * j;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 t = *reinterpret_cast<const float4*>(zs + 4 * q);
-          zr[2 * q] = f2(t.x, t.y);
-          zr[2 * q + 1] = f2(t.z, t.w);
-        }
-      }
+      const int par = (int)(i & 1);
       bool ok = mbar_wait_warp(&qkfull[s], rq.ph, abort_flag);
       ok = ok && mbar_wait_warp(kffree, (uint32_t)((i & 1) ^ 1), abort_flag);
       ok = ok && mbar_wait_warp(&denfree[s], rq.ph ^ 1u, abort_flag);
@@ -658,14 +663,92 @@ __global__ void __launch_bounds__(kCaThreads, 1)
       const uint32_t rec_s = sbase + TcCausalSmem::ROWREC + s * kCaTile * kRecBytes;
       float* den = den_ring + s * kCaTile;
       const int n0 = iw.ti * kCaTile;
+      float* zr_now = zrun + par * 128;
+      if (iw.first && tw == 0 && rg == 0) {
+        // The key sum of the head starts at its slot's z_start.
+        if (!waited_grid) {
+          pdl_wait();
+          waited_grid = true;
+        }
+        const float* zs = p.z_start + ((size_t)c + iw.bh) * 128 + 16 * j;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<float4*>(zr_now + 16 * j + 4 * q) =
+              *reinterpret_cast<const float4*>(zs + 4 * q);
+      }
+      // Pass 1: this warp's sum of k_pls over its 16 rows.
+      f2_t ta[8];
+#pragma unroll
+      for (int i2 = 0; i2 < 8; ++i2) ta[i2] = 0ull;
 #pragma unroll 1
       for (int u = 0; u < kCaGroups; ++u) {
-        const int r = u * kCaTW * 4 + tw * 4 + rg;
-        const uint32_t roff = (uint32_t)(u * kCaTW * 4) * 128u;
+        const uint32_t roff = (uint32_t)(kCaRowsW * tw + 4 * (u & ~1)) * 128u;
+        f2_t x[8];
+        unpack8(lds128(kt + ch0[u & 1] + roff), lds128(kt + ch1[u & 1] + roff), x);
+        const float rstd = row_rstd(x);
+        const f2_t rstd2 = f2(rstd, rstd);
+#pragma unroll
+        for (int i2 = 0; i2 < 8; ++i2) ta[i2] = f2_fma(f2_relu(x[i2]), rstd2, ta[i2]);
+      }
+#pragma unroll
+      for (int i2 = 0; i2 < 8; ++i2) {
+        ta[i2] = f2_add(ta[i2], shfl_f2(ta[i2], lane ^ 4));
+        ta[i2] = f2_add(ta[i2], shfl_f2(ta[i2], lane ^ 16));
+      }
+      float* gt = gtot + par * (kCaTW * 128);
+      if (rg == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<float4*>(gt + tw * 128 + (q * 8 + j) * 4) =
+              make_float4(f2_lo(ta[2 * q]), f2_hi(ta[2 * q]), f2_lo(ta[2 * q + 1]),
+                          f2_hi(ta[2 * q + 1]));
+      }
+      named_barrier(2, kCaTW * 32);
+      // The key sum before the warp's first row; warp 0 also records the sum
+      // after the chunk for the next one.
+      f2_t off[8], tot[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 t = *reinterpret_cast<const float4*>(zr_now + 16 * j + 4 * q);
+        off[2 * q] = f2(t.x, t.y);
+        off[2 * q + 1] = f2(t.z, t.w);
+        tot[2 * q] = off[2 * q];
+        tot[2 * q + 1] = off[2 * q + 1];
+      }
+#pragma unroll 1
+      for (int w2 = 0; w2 < kCaTW; ++w2) {
+        f2_t gv[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 t = *reinterpret_cast<const float4*>(gt + w2 * 128 + (q * 8 + j) * 4);
+          gv[2 * q] = f2(t.x, t.y);
+          gv[2 * q + 1] = f2(t.z, t.w);
+        }
+        if (w2 < tw) {
+#pragma unroll
+          for (int i2 = 0; i2 < 8; ++i2) off[i2] = f2_add(off[i2], gv[i2]);
+        }
+#pragma unroll
+        for (int i2 = 0; i2 < 8; ++i2) tot[i2] = f2_add(tot[i2], gv[i2]);
+      }
+      if (tw == 0 && rg == 0) {
+        float* zr_next = zrun + (par ^ 1) * 128 + 16 * j;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<float4*>(zr_next + 4 * q) =
+              make_float4(f2_lo(tot[2 * q]), f2_hi(tot[2 * q]), f2_lo(tot[2 * q + 1]),
+                          f2_hi(tot[2 * q + 1]));
+      }
+      // Pass 2: the transforms and the denominators, row group by row group.
+#pragma unroll 1
+      for (int u = 0; u < kCaGroups; ++u) {
+        const int r = kCaRowsW * tw + 4 * u + rg;
+        const uint32_t roff = (uint32_t)(kCaRowsW * tw + 4 * (u & ~1)) * 128u;
+        const uint32_t c0 = ch0[u & 1] + roff, c1 = ch1[u & 1] + roff;
         uint32_t t012 = 0, t345 = 0, t67 = 0;
         if (g.rope_on) lane_rope_row(lr, rec_s + r * kRecBytes, t012, t345, t67);
-        const uint4 k0 = lds128(kt + ch0 + roff), k1 = lds128(kt + ch1 + roff);
-        const uint4 q0 = lds128(qt + ch0 + roff), q1 = lds128(qt + ch1 + roff);
+        const uint4 k0 = lds128(kt + c0), k1 = lds128(kt + c1);
+        const uint4 q0 = lds128(qt + c0), q1 = lds128(qt + c1);
         f2_t e[8];
         if (g.rope_on) tab_load8(t012, t345, t67, e);
         const float bet = bs[r];
@@ -683,11 +766,11 @@ __global__ void __launch_bounds__(kCaThreads, 1)
           }
           uint4 o0, o1;
           rope_scale_pack<false>(g.rope_on, e, x, rstd * bet, o0, o1);
-          sts128(kt + ch0 + roff, o0);
-          sts128(kt + ch1 + roff, o1);
+          sts128(kt + c0, o0);
+          sts128(kt + c1, o1);
           rope_scale_pack<true>(g.rope_on, e, x, rstd * bet, o0, o1);
-          sts128(kf + ch0 + roff, o0);
-          sts128(kf + ch1 + roff, o1);
+          sts128(kf + c0, o0);
+          sts128(kf + c1, o1);
         }
         // queries
         f2_t qp[8];
@@ -703,8 +786,8 @@ __global__ void __launch_bounds__(kCaThreads, 1)
           }
           uint4 o0, o1;
           rope_scale_pack<true>(g.rope_on, e, y, rstd, o0, o1);
-          sts128(qt + ch0 + roff, o0);
-          sts128(qt + ch1 + roff, o1);
+          sts128(qt + c0, o0);
+          sts128(qt + c1, o1);
         }
         // Inclusive prefix of k_pls over the group's four rows (rg order).
 #pragma unroll
@@ -717,36 +800,10 @@ __global__ void __launch_bounds__(kCaThreads, 1)
           const f2_t t = shfl_f2(kp[i2], src2);
           if (rg >= 2) kp[i2] = f2_add(kp[i2], t);
         }
-        float* gt = gtot + gpar * (kCaTW * 128);
-        if (rg == 3) {
-#pragma unroll
-          for (int i2 = 0; i2 < 8; i2 += 2)
-            *reinterpret_cast<float4*>(gt + tw * 128 + 16 * j + 2 * i2) =
-                make_float4(f2_lo(kp[i2]), f2_hi(kp[i2]), f2_lo(kp[i2 + 1]), f2_hi(kp[i2 + 1]));
-        }
-        named_barrier(2, kCaTW * 32);
-        // den = q_pls . (z before the chunk + earlier groups' and warps' rows +
-        // this row's prefix) + eps; then z absorbs the whole group.
+        // den = q_pls . (key sum before the group + this row's prefix) + eps
         f2_t dd = 0ull;
 #pragma unroll
-        for (int i2 = 0; i2 < 8; ++i2) dd = f2_fma(qp[i2], f2_add(zr[i2], kp[i2]), dd);
-#pragma unroll 1
-        for (int w2 = 0; w2 < kCaTW; ++w2) {
-          const float* src = gt + w2 * 128 + 16 * j;
-          f2_t gv[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 t = *reinterpret_cast<const float4*>(src + 4 * q);
-            gv[2 * q] = f2(t.x, t.y);
-            gv[2 * q + 1] = f2(t.z, t.w);
-          }
-          if (w2 < tw) {
-#pragma unroll
-            for (int i2 = 0; i2 < 8; ++i2) dd = f2_fma(qp[i2], gv[i2], dd);
-          }
-#pragma unroll
-          for (int i2 = 0; i2 < 8; ++i2) zr[i2] = f2_add(zr[i2], gv[i2]);
-        }
+        for (int i2 = 0; i2 < 8; ++i2) dd = f2_fma(qp[i2], f2_add(off[i2], kp[i2]), dd);
         const float dn = row_sum(f2_lo(dd) + f2_hi(dd)) + g.eps;
         if (j == 0) {
           den[r] = dn;
@@ -754,21 +811,26 @@ __global__ void __launch_bounds__(kCaThreads, 1)
           if (kDebug && p.den_out && n < g.N)
             p.den_out[((size_t)iw.b * g.N + n) * g.Hh + iw.h] = dn;
         }
-        gpar ^= 1u;
+        // The next group starts after this group's last row.
+#pragma unroll
+        for (int i2 = 0; i2 < 8; ++i2) off[i2] = f2_add(off[i2], shfl_f2(kp[i2], src3));
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(tready);
     }
-  } else {
-    // ----------------------------------------------------- epilogue warps
-    // Thread = TMEM lane = token row (rows 96..127 take part in the state
-    // image only).
+  } else if (warp < kCaOW0) {
+    // -------------------------------------------------------- chain warps
+    // The two steps the MMA chain waits on: P = mask(A) * scale after the
+    // first MMAs of a chunk, and the image of the state after its state MMA
+    // (the next chunk's read-out operand).  Thread = TMEM lane = state row;
+    // rows 96..127 take part in the image only.
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tmem + kCaTmS + lane_off;
     unsigned char* simg = sm + TcCausalSmem::SIMG;
+    float* scl = reinterpret_cast<float*>(sm + TcCausalSmem::SCL);
     bool waited_grid = false;
     bool ok = true;
     uint32_t rpar = 0;
@@ -779,7 +841,6 @@ __global__ void __launch_bounds__(kCaThreads, 1)
     for (; iw.more(); iw.next(), rq.next(), ++i) {
       const uint32_t par = (uint32_t)(i & 1);
       const int s = rq.s;
-      const int b = iw.b, h = iw.h, n0 = iw.ti * kCaTile;
       if (iw.first) {
         // The state before the segment: this slot's S_start into TMEM, then
         // its image.  The previous segment's last state MMA was waited for
@@ -807,11 +868,12 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         cur_scale = causal_image(tS, simg, red, (int)rpar, q4, lane, ok);
         rpar ^= 1u;
         if (!ok) break;
+        if (threadIdx.x == kCaEW0 * 32) scl[i & 3] = cur_scale;
         __syncwarp();
         if (lane == 0) mbar_arrive(imgready);
       }
       // (a) P = mask(A) * scale, over the chunk's q slot.  Wait outcomes are
-      // made warp-uniform: the tcgen05 loads below are warp-collective.
+      // warp-uniform: the tcgen05 loads below are warp-collective.
       ok = ok && mbar_wait_warp(afull, par, abort_flag);
       if (ok && row < kCaTile) {
         tc_fence_after();
@@ -847,79 +909,108 @@ __global__ void __launch_bounds__(kCaThreads, 1)
       // the segment.
       ok = ok && mbar_wait_warp(sfull, par, abort_flag);
       tc_fence_after();
-      const float chunk_scale = cur_scale;
       if (!iw.last) {
         cur_scale = causal_image(tS, simg, red, (int)rpar, q4, lane, ok);
         rpar ^= 1u;
         if (!ok) break;
+        if (threadIdx.x == kCaEW0 * 32) scl[(i + 1) & 3] = cur_scale;
         __syncwarp();
         if (lane == 0) mbar_arrive(imgready);
       } else {
         ok = bar_red_and(3, kCaEW * 32, ok);
         if (!ok) break;
       }
-      // (d) the read-out: x = sigmoid(g) * U / (den * scale), RMSNorm, bf16.
-      ok = mbar_wait_warp(&ufull[s], rq.ph, abort_flag);
+    }
+  } else {
+    // ------------------------------------------------------- output warps
+    // Thread = TMEM lane = token row 0..95 of the chunk:
+    // x = sigmoid(g) * U / (den * scale), the output RMSNorm, bf16 stores.
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const float* scl = reinterpret_cast<const float*>(sm + TcCausalSmem::SCL);
+    ItemWalk iw(wb, we, tph, g.Hh);
+    RingPos<2> rq;
+    long long i = 0;
+    for (; iw.more(); iw.next(), rq.next(), ++i) {
+      const uint32_t par = (uint32_t)(i & 1);
+      const int s = rq.s;
+      const int b = iw.b, h = iw.h, n0 = iw.ti * kCaTile;
+      // den (transform warps) and the scale (chain warps) of the chunk: their
+      // barriers have completed for this chunk and at most one chunk more, so
+      // waiting on them is immediate and orders the reads after the writes.
+      bool ok = mbar_wait_warp(tready, par, abort_flag);
+      ok = ok && mbar_wait_warp(imgready, par, abort_flag);
+      ok = ok && mbar_wait_warp(&ufull[s], rq.ph, abort_flag);
+      if (!ok) break;
       const int n = n0 + row;
       const bool valid = n < g.N;   // per lane: guards global memory only
-      if (ok && row < kCaTile) {
-        tc_fence_after();
-        const float hc = 0.5f / (den_ring[s * kCaTile + row] * chunk_scale);
-        const uint32_t tU = tmem + kCaTmU + (uint32_t)s * 128u + lane_off;
-        const size_t rowoff = (((size_t)b * g.N + (valid ? n : 0)) * g.Hh + h) * 128;
-        const __nv_bfloat16* grow = p.gate + rowoff;
-        const f2_t hc2 = f2(hc, hc), half2 = f2(0.5f, 0.5f);
-        f2_t ss2 = 0ull;
+      tc_fence_after();
+      const float hc = 0.5f / (den_ring[s * kCaTile + row] * scl[i & 3]);
+      const uint32_t tU = tmem + kCaTmU + (uint32_t)s * 128u + lane_off;
+      const size_t rowoff = (((size_t)b * g.N + (valid ? n : 0)) * g.Hh + h) * 128;
+      const __nv_bfloat16* grow = p.gate + rowoff;
+      const f2_t hc2 = f2(hc, hc), half2 = f2(0.5f, 0.5f);
+      f2_t ss2 = 0ull;
+      // Gate loads run one 32-channel block ahead of their use (the producer
+      // has prefetched the chunk's gate tile into L2).
+      uint4 gv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        gv[q] = valid ? ldg_nc128(grow + 8 * q) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
-          uint4 gv[4];
+      for (int cb = 0; cb < 4; ++cb) {
+        uint4 gn[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            gv[q] = valid ? ldg_nc128(grow + cb * 32 + 8 * q) : make_uint4(0u, 0u, 0u, 0u);
-          float u[32];
-          tmem_ld32(tU + cb * 32, u);
-          tmem_wait_ld();
+        for (int q = 0; q < 4; ++q)
+          gn[q] = (valid && cb < 3) ? ldg_nc128(grow + (cb + 1) * 32 + 8 * q)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        float u[32];
+        tmem_ld32(tU + cb * 32, u);
+        tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t wv[4] = {gv[q].x, gv[q].y, gv[q].z, gv[q].w};
+        for (int q = 0; q < 4; ++q) {
+          const uint4 gq = gv[q];
+          const uint32_t wv[4] = {gq.x, gq.y, gq.z, gq.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const f2_t hg = f2_mul(f2_bf(wv[e]), half2);
-              const f2_t t = f2(tanh_approx(f2_lo(hg)), tanh_approx(f2_hi(hg)));
-              const f2_t sg = f2_fma(hc2, t, hc2);
-              const f2_t x = f2_mul(sg, f2(u[q * 8 + 2 * e], u[q * 8 + 2 * e + 1]));
-              ss2 = f2_fma(x, x, ss2);
-              u[q * 8 + 2 * e] = f2_lo(x);
-              u[q * 8 + 2 * e + 1] = f2_hi(x);
-            }
+          for (int e = 0; e < 4; ++e) {
+            const f2_t hg = f2_mul(f2_bf(wv[e]), half2);
+            const f2_t t = f2(tanh_approx(f2_lo(hg)), tanh_approx(f2_hi(hg)));
+            const f2_t sg = f2_fma(hc2, t, hc2);
+            const f2_t x = f2_mul(sg, f2(u[q * 8 + 2 * e], u[q * 8 + 2 * e + 1]));
+            ss2 = f2_fma(x, x, ss2);
+            u[q * 8 + 2 * e] = f2_lo(x);
+            u[q * 8 + 2 * e + 1] = f2_hi(x);
           }
-          if (kDebug && p.x_out && valid) {
-            float* xo = p.x_out + rowoff + cb * 32;
-#pragma unroll
-            for (int i2 = 0; i2 < 32; i2 += 4)
-              *reinterpret_cast<float4*>(xo + i2) = make_float4(u[i2], u[i2 + 1], u[i2 + 2], u[i2 + 3]);
-          }
-          tmem_st32(tU + cb * 32, u);
         }
-        tmem_wait_st();
-        const float rstd = rsqrtf((f2_lo(ss2) + f2_hi(ss2)) * (1.f / 128.f) + kRmsEps);
-        const f2_t rstd2 = f2(rstd, rstd);
-        __nv_bfloat16* orow = p.out + rowoff;
+        if (kDebug && p.x_out && valid) {
+          float* xo = p.x_out + rowoff + cb * 32;
+#pragma unroll
+          for (int i2 = 0; i2 < 32; i2 += 4)
+            *reinterpret_cast<float4*>(xo + i2) = make_float4(u[i2], u[i2 + 1], u[i2 + 2], u[i2 + 3]);
+        }
+        tmem_st32(tU + cb * 32, u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) gv[q] = gn[q];
+      }
+      tmem_wait_st();
+      const float rstd = rsqrtf((f2_lo(ss2) + f2_hi(ss2)) * (1.f / 128.f) + kRmsEps);
+      const f2_t rstd2 = f2(rstd, rstd);
+      __nv_bfloat16* orow = p.out + rowoff;
 #pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
-          float x[32];
-          tmem_ld32(tU + cb * 32, x);
-          tmem_wait_ld();
+      for (int cb = 0; cb < 4; ++cb) {
+        float x[32];
+        tmem_ld32(tU + cb * 32, x);
+        tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t o[4];
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const f2_t y = f2_mul(f2(x[q * 8 + 2 * e], x[q * 8 + 2 * e + 1]), rstd2);
-              o[e] = pack_bf16(f2_lo(y), f2_hi(y));
-            }
-            if (valid) stg128(orow + cb * 32 + 8 * q, make_uint4(o[0], o[1], o[2], o[3]));
+          for (int e = 0; e < 4; ++e) {
+            const f2_t y = f2_mul(f2(x[q * 8 + 2 * e], x[q * 8 + 2 * e + 1]), rstd2);
+            o[e] = pack_bf16(f2_lo(y), f2_hi(y));
           }
+          if (valid) stg128(orow + cb * 32 + 8 * q, make_uint4(o[0], o[1], o[2], o[3]));
         }
       }
       tc_fence_before();
@@ -978,6 +1069,8 @@ inline gla_status run_causal_tensor(const Geom& g, const void* q, const void* k,
   sp.beta = static_cast<const __nv_bfloat16*>(beta);
   sp.part_S = part_S; sp.part_z = part_z; sp.tab_entries = stab;
   sp.rope_tab = nullptr;
+  sp.wait_ns = kWaitLimitNs;
+  sp.stall_item = -1;
   if (!ensure_max_smem(tc_state_kernel, 0)) return GLA_ERR_CUDA;
   cudaLaunchConfig_t sc = {};
   sc.gridDim = dim3(spart.grid);
@@ -991,7 +1084,7 @@ inline gla_status run_causal_tensor(const Geom& g, const void* q, const void* k,
     return GLA_ERR_CUDA;
 
   PrefixParams pp = {};
-  pp.part = spart; pp.zparts = kStTW;
+  pp.part = spart;
   pp.part_S = part_S; pp.part_z = part_z;
   pp.S_in = S; pp.z_in = z;
   pp.S_start = S_start; pp.z_start = z_start;

@@ -202,6 +202,7 @@ struct Call {
   cudaStream_t stream;
   float *S_dbg, *z_dbg, *den_dbg, *x_dbg;
   void* const* events;   // optional [4] cudaEvent_t records around the kernels
+  unsigned long long stall_limit_ns = 0;   // self-test of the abort path (0: off)
 };
 
 inline cudaError_t mark(const Call& c, int i) {
@@ -298,7 +299,7 @@ gla_status run_call(Call& c) {
                     reinterpret_cast<__half*>(c.ws + c.L.S_img),
                     reinterpret_cast<float*>(c.ws + c.L.S_scale),
                     reinterpret_cast<float2*>(c.ws + c.L.rope_tab), c.den_dbg, c.x_dbg,
-                    device_sm_count(), c.stream, c.events);
+                    device_sm_count(), c.stream, c.events, c.stall_limit_ns);
   } else {
     st = c.dtype == GLA_DTYPE_F32 ? run_simt_dtype<float>(c)
                                   : run_simt_dtype<__nv_bfloat16>(c);
@@ -414,7 +415,8 @@ gla_status forward_common(const void* q, const void* k, const void* v, const voi
                           int W, float rope_theta, float eps, int dtype, void* out,
                           void* workspace, size_t workspace_bytes, void* stream, int path,
                           float* S_out, float* z_out, float* den_out, float* x_out,
-                          void* const* events = nullptr) {
+                          void* const* events = nullptr,
+                          unsigned long long stall_limit_ns = 0) {
   if (!dims_ok(batch, heads, head_dim, T, H, W)) return GLA_ERR_INVALID_ARG;
   if (dtype != GLA_DTYPE_F32 && dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
   if (!(eps > 0.f) || !isfinite(eps) || !isfinite(rope_theta)) return GLA_ERR_INVALID_ARG;
@@ -439,6 +441,7 @@ gla_status forward_common(const void* q, const void* k, const void* v, const voi
   c.stream = static_cast<cudaStream_t>(stream);
   c.S_dbg = S_out; c.z_dbg = z_out; c.den_dbg = den_out; c.x_dbg = x_out;
   c.events = events;
+  c.stall_limit_ns = stall_limit_ns;
   return run_call(c);
 }
 
@@ -855,6 +858,19 @@ gla_status gla_forward_noalloc(const void* q, const void* k, const void* v, cons
   c.S_dbg = c.z_dbg = c.den_dbg = c.x_dbg = nullptr;
   c.events = nullptr;
   return run_call(c);
+}
+
+gla_status gla_selftest_pipeline_stall(const void* q, const void* k, const void* v,
+                                       const void* beta, const void* g, int batch, int heads,
+                                       int head_dim, int T, int H, int W, float rope_theta,
+                                       float eps, void* out, void* workspace,
+                                       size_t workspace_bytes, unsigned int limit_us,
+                                       void* stream) {
+  if (limit_us < 1 || limit_us > 1000000u) return GLA_ERR_INVALID_ARG;
+  return forward_common(q, k, v, beta, g, batch, heads, head_dim, T, H, W, rope_theta, eps,
+                        GLA_DTYPE_BF16, out, workspace, workspace_bytes, stream, GLA_PATH_TENSOR,
+                        nullptr, nullptr, nullptr, nullptr, nullptr,
+                        (unsigned long long)limit_us * 1000ull);
 }
 
 gla_status gla_selftest_wait_timeout(unsigned int limit_us, void* stream) {

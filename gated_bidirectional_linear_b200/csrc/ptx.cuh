@@ -109,6 +109,13 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
+// The same with an explicit limit.
+__device__ __forceinline__ bool mbar_wait_warp_for(uint64_t* bar, uint32_t parity,
+                                                   volatile int* abort,
+                                                   unsigned long long limit_ns) {
+  return __all_sync(0xffffffffu, mbar_wait_for(bar, parity, abort, limit_ns));
+}
+
 // ------------------------------------------------ programmatic dependent launch
 
 // Let the next kernel of the stream (launched with programmatic stream

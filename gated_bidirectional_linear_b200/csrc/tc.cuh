@@ -75,6 +75,9 @@ struct TcStateParams {
   float* part_z;
   float2* rope_tab;   // optional: the call's whole RoPE table for the read-out
   int tab_entries;
+  unsigned long long wait_ns;   // limit of every wait (kWaitLimitNs)
+  long long stall_item;         // self-test only: CTA 0 withholds this item's
+                                // arrival (-1: never)
 };
 
 // A CTA's items in order, advanced without divisions: head bh (batch b and
@@ -382,7 +385,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       if (iw.more()) fetch_beta(iw);
       for (; iw.more(); iw.next(), rp.next(), ++it) {
         const int s = rp.s;
-        if (!mbar_wait_warp(&empty[s], rp.ph ^ 1u, abort_flag)) break;
+        if (!mbar_wait_warp_for(&empty[s], rp.ph ^ 1u, abort_flag, p.wait_ns)) break;
         const int b = iw.b, h = iw.h;
         const int n0 = iw.ti * kStTile;
         // Lane 0 starts the tile copies first; then the warp stores beta,
@@ -410,7 +413,8 @@ __global__ void __launch_bounds__(kStThreads, 1)
           tile_rowrec<kStTile>(g, win, n0, lane,
                                sm + TcStateSmem::ROWREC + s * kStTile * kRecBytes);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
+        // (the self-test withholds one arrival so that the consumers' waits run out)
+        if (lane == 0 && !(c == 0 && it == p.stall_item)) mbar_arrive(&full[s]);
         ++issued;
         // While the first tiles land: this CTA's rows of the whole-call RoPE
         // table the read-out copies.  Written after the wait above, so the
@@ -423,8 +427,8 @@ __global__ void __launch_bounds__(kStThreads, 1)
         long long first = it - (issued < kStStages ? issued : kStStages);
         for (long long i2 = first; i2 < it; ++i2) {
           int dummy = 0;
-          mbar_wait(&full[i2 % kStStages], (uint32_t)((i2 / kStStages) & 1),
-                    reinterpret_cast<volatile int*>(&dummy));
+          mbar_wait_for(&full[i2 % kStStages], (uint32_t)((i2 / kStStages) & 1),
+                        reinterpret_cast<volatile int*>(&dummy), p.wait_ns);
         }
       }
     }
@@ -440,9 +444,10 @@ __global__ void __launch_bounds__(kStThreads, 1)
         const uint32_t ph = rp.ph;
         const bool first = iw.first, last = iw.last;
         const int ab = seg & 1;
-        if (first && !mbar_wait(&accempty[ab], (uint32_t)(((seg >> 1) & 1) ^ 1), abort_flag))
+        if (first && !mbar_wait_for(&accempty[ab], (uint32_t)(((seg >> 1) & 1) ^ 1), abort_flag,
+                                    p.wait_ns))
           break;
-        if (!mbar_wait(&kready[s], ph, abort_flag)) break;
+        if (!mbar_wait_for(&kready[s], ph, abort_flag, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t kt = sbase + TcStateSmem::K + s * kStTileBytes;
         const uint32_t vt = sbase + TcStateSmem::V + s * kStTileBytes;
@@ -461,7 +466,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       // Every MMA issued above has completed before TMEM is released.
       umma_commit(drain);
       int dummy = 0;
-      mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy));
+      mbar_wait_for(drain, 0, reinterpret_cast<volatile int*>(&dummy), p.wait_ns);
     }
   } else {
     // ------------------------------------------- transform warps: k -> beta k_til
@@ -487,7 +492,7 @@ __global__ void __launch_bounds__(kStThreads, 1)
       const int s = rp.s;
       const uint32_t ph = rp.ph;
       const int bh = iw.bh;
-      if (!mbar_wait_warp(&full[s], ph, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp_for(&full[s], ph, abort_flag, p.wait_ns)) { ok = false; break; }
       const uint32_t kt = sbase + TcStateSmem::K + s * kStTileBytes;
       const float* bs = reinterpret_cast<const float*>(sm + TcStateSmem::BETA + s * kStTile * 4);
       const uint32_t rec_s = sbase + TcStateSmem::ROWREC + s * kStTile * kRecBytes;
@@ -566,7 +571,10 @@ __global__ void __launch_bounds__(kStThreads, 1)
           const int third = tw >> 2;
           const int a = q4 * 32 + lane;
           const int ab = seg & 1;
-          if (!mbar_wait_warp(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp_for(&accfull[ab], (uint32_t)((seg >> 1) & 1), abort_flag, p.wait_ns)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           // Chunk-major partial: columns 8cb .. 8cb+7 of row a at (cb * 128 + a) * 8,
           // so the warp's 32 rows of a chunk are 1 KB of contiguous stores.
@@ -1177,7 +1185,7 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
                              float* z, bool carry, bool write_state, float* part_S,
                              float* part_z, __half* S_img, float* S_scale, float2* rope_tab,
                              float* den_dbg, float* x_dbg, int sms, cudaStream_t stream,
-                             void* const* events) {
+                             void* const* events, unsigned long long stall_limit_ns = 0) {
   auto mark = [&](int i) {
     if (!events || !events[i]) return cudaSuccess;
     return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream);
@@ -1203,6 +1211,8 @@ inline gla_status run_tensor(const Geom& g, const void* q, const void* k, const 
   sp.beta = static_cast<const __nv_bfloat16*>(beta);
   sp.part_S = part_S; sp.part_z = part_z; sp.tab_entries = stab;
   sp.rope_tab = g.rope_on ? rope_tab : nullptr;
+  sp.wait_ns = stall_limit_ns ? stall_limit_ns : kWaitLimitNs;
+  sp.stall_item = stall_limit_ns ? 0 : -1;
   if (!ensure_max_smem(tc_state_kernel, 0)) return GLA_ERR_CUDA;
   if (mark(0) != cudaSuccess) return GLA_ERR_CUDA;
   cudaLaunchAttribute pdl[1];

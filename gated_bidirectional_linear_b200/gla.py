@@ -51,6 +51,8 @@ _SIGS = {
     "gla_forward_noalloc": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp]),
     "gla_get_device_status": (_i, [_vp]),
     "gla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
+    "gla_selftest_pipeline_stall": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _vp, _vp, _sz,
+                                                               ctypes.c_uint, _vp]),
     "gla_plan": (_i, [_i] * 9 + [ctypes.POINTER(_i)] * 3),
     "gla_check_rope_copy": (_i, [_i] * 7),
 }
@@ -449,6 +451,28 @@ def gla_selftest_wait_timeout(limit_us, stream=None):
     with _on(dev):
         st = lib().gla_selftest_wait_timeout(int(limit_us), _stream(stream, dev))
     _check(st, "gla_selftest_wait_timeout")
+
+
+def gla_selftest_pipeline_stall(q, k, v, beta, g, T, H, W, limit_us, rope_theta=10000.0,
+                                eps=1e-6, out=None, workspace=None, stream=None):
+    """Run gla_forward (tensor path) with the state kernel's waits limited to
+    `limit_us` and one producer arrival withheld, so that its pipeline abort
+    path runs for real; read the outcome with gla_get_device_status()."""
+    B, Hh, d = _dims(q, T, H, W)
+    if out is None:
+        out = torch.empty_like(q)
+    _validate(q, k, v, beta, g, out)
+    if workspace is None:
+        workspace = alloc_workspace(gla_forward_workspace_size(B, Hh, d, T, H, W,
+                                                               _dtype_code(q)), q.device)
+    _check_workspace(workspace, q.device)
+    with _on(q.device):
+        st = lib().gla_selftest_pipeline_stall(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g),
+                                               B, Hh, d, T, H, W, rope_theta, eps, _ptr(out),
+                                               _ptr(workspace), workspace.numel(),
+                                               int(limit_us), _stream(stream, q.device))
+    _check(st, "gla_selftest_pipeline_stall")
+    return out
 
 
 def gla_plan(batch, heads, head_dim, T, H, W, dtype, path, num_sms):

@@ -344,6 +344,26 @@ GLA_API gla_status gla_get_device_status(void* stream);
  * GLA_ERR_CUDA if the launch fails, else GLA_OK. */
 GLA_API gla_status gla_selftest_wait_timeout(unsigned int limit_us, void* stream);
 
+/* Self-test of the tensor pipelines' abort path (tests only; no fault, no
+ * hang).  Runs gla_forward on the tensor path (bf16, head_dim 128; arguments
+ * as gla_forward) with two changes in the state-reduction kernel: every
+ * pipeline wait gives up after `limit_us` microseconds (1 .. 1000000) instead
+ * of 2 s, and the producer of CTA 0 withholds the arrival that announces its
+ * first tile.  The transform warps' wait for that tile runs out: the kernel
+ * records GLA_ERR_TIMEOUT in the device error word, raises its abort flag, and
+ * every role leaves its loop, lets its copies and MMAs in flight complete,
+ * frees TMEM and returns; the rest of the call runs to completion on the
+ * partial sums it has.  `out` then holds no meaningful result, a later
+ * gla_get_device_status() reports GLA_ERR_TIMEOUT (and clears it), and the
+ * next call computes normally.  Returns GLA_ERR_INVALID_ARG for a limit out
+ * of range, GLA_ERR_UNSUPPORTED where the tensor path does not apply. */
+GLA_API gla_status gla_selftest_pipeline_stall(const void* q, const void* k, const void* v,
+                                               const void* beta, const void* g, int batch,
+                                               int heads, int head_dim, int T, int H, int W,
+                                               float rope_theta, float eps, void* out,
+                                               void* workspace, size_t workspace_bytes,
+                                               unsigned int limit_us, void* stream);
+
 /* Host-only self-check of the tensor read-out's RoPE table copies (tests; no
  * GPU needed): for every read-out CTA of this problem on num_sms SMs, the bulk
  * copies that bring its table window from the whole-call table are 16-byte

@@ -44,3 +44,26 @@ def test_library_still_computes_after_a_timeout():
     ref = O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], wl.T, wl.H, wl.W, 1e4, 1e-6)
     err = O.max_rel_err_rms_floor(out.cpu().double().numpy(), ref["out"])
     assert np.isfinite(err) and err <= 1e-5
+
+
+def test_state_pipeline_abort_path_then_recovery():
+    """The state kernel's own abort path: CTA 0's producer withholds one
+    arrival, the transform warps' wait runs out after 2 ms, and every role
+    leaves, drains its copies and MMAs and frees TMEM; the call ends, the
+    status reads GLA_ERR_TIMEOUT once, and the next call matches the oracle."""
+    torch.cuda.set_device(0)
+    assert gla.gla_get_device_status() == gla.GLA_OK
+    T, H, W, B, HH = 2, 6, 16, 1, 3
+    inp = workloads.draw(B, T * H * W, HH, 128, "bf16", seed=61)
+    d = {k: v.cuda() for k, v in inp.items()}
+    t0 = time.monotonic()
+    gla.gla_selftest_pipeline_stall(d["q"], d["k"], d["v"], d["beta"], d["g"], T, H, W, 2000)
+    assert gla.gla_get_device_status() == gla.GLA_ERR_TIMEOUT
+    assert time.monotonic() - t0 < 10.0
+    assert gla.gla_get_device_status() == gla.GLA_OK
+    out = gla.gla_forward(d["q"], d["k"], d["v"], d["beta"], d["g"], T, H, W)
+    torch.cuda.synchronize()
+    assert gla.gla_get_device_status() == gla.GLA_OK
+    x = workloads.as_f64(inp)
+    ref = O.forward(x["q"], x["k"], x["v"], x["beta"], x["g"], T, H, W, 1e4, 1e-6)
+    assert O.bf16_out_err_over_rms(out.cpu().double().numpy(), ref["out"]) <= 2e-2
