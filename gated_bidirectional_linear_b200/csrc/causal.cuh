@@ -264,18 +264,27 @@ __global__ void __launch_bounds__(kPrefixThreads) combine_prefix_kernel(PrefixPa
 constexpr int kCaTile = kStTile;                 // tokens per chunk: the state partition's tile
 constexpr uint32_t kCaBox = kStBox;              // 96 rows x 128 bytes
 constexpr uint32_t kCaTileBytes = kStTileBytes;  // two boxes
-constexpr int kCaTW = 6;                         // transform warps 2..7
-constexpr int kCaTW0 = 2;
-constexpr int kCaEW0 = kCaTW0 + kCaTW;           // chain warps 8..11: P and the state image
-constexpr int kCaEW = 4;                         // one per TMEM lane quarter
-constexpr int kCaOW0 = kCaEW0 + kCaEW;           // output warps 12..14: lane quarters 0..2
-constexpr int kCaOW = kCaTile / 32;              // (rows 0..95)
-constexpr int kCaThreads = (kCaOW0 + kCaOW) * 32;
+// Warp roles: 0 producer, 1 MMA, 2..7 transform, 8..11 chain (P and the
+// state image; one per TMEM lane quarter), 12..14 output (lane quarters 0..2:
+// rows 0..95).  15 warps keep every scheduler at four warps or fewer, so each
+// thread may hold 128 registers (a 16th or 17th warp would cut that).
+constexpr int kCaTW = 6;
+constexpr int kCaEW0 = 8;
+constexpr int kCaEW = 4;
+constexpr int kCaOW0 = 12;
+constexpr int kCaOW = kCaTile / 32;
+constexpr int kCaWarps = kCaOW0 + kCaOW;
+constexpr int kCaThreads = kCaWarps * 32;
 static_assert(kCaEW0 % 4 == 0 && kCaOW0 % 4 == 0, "role warps start on a lane quarter");
+static_assert(2 + kCaTW == kCaEW0, "transform warps 2 .. kCaEW0-1");
+// Index of a transform warp (0 .. kCaTW-1), or -1.
+__host__ __device__ constexpr int ca_transform_index(int warp) {
+  return warp >= 2 && warp < kCaEW0 ? warp - 2 : -1;
+}
 constexpr int kCaRowsW = kCaTile / kCaTW;         // contiguous rows per transform warp
 constexpr int kCaGroups = kCaRowsW / 4;          // its row groups of 4
 static_assert(kCaGroups * 4 * kCaTW == kCaTile, "whole row groups per chunk");
-static_assert(kCaRowsW % 8 == 0, "a warp's rows start on the 8-row swizzle phase");
+static_assert(kCaRowsW % 4 == 0, "row groups start on a multiple of four rows");
 
 // TMEM columns: A = Q_til (beta K_til)^T, two read-out accumulators U, the state.
 constexpr uint32_t kCaTmA = 0, kCaTmU = 128, kCaTmS = 384;
@@ -618,25 +627,25 @@ __global__ void __launch_bounds__(kCaThreads, 1)
       int dummy = 0;
       mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy));
     }
-  } else if (warp < kCaEW0) {
+  } else if (ca_transform_index(warp) >= 0) {
     // --------------------------------------------------- transform warps
     // q -> q_til (fp16), k -> beta k_til (bf16 in place, fp16 copy), and the
     // denominator of every row from the running sum of k_pls.  Warp tw owns
-    // the chunk's rows 16 tw .. 16 tw + 15 (four row groups of four).  A
+    // kCaRowsW contiguous rows of the chunk (row groups of four).  A
     // first pass sums the warp's k_pls; after one barrier each warp knows the
     // key sum before its rows (the sum before the chunk plus the earlier
     // warps' sums), and the main pass carries it row group by row group.
     // Warp sums are stored with 16-byte chunk q of lane j at float4 index
     // q * 8 + j, so that the 8 lanes that read one chunk read 128 contiguous
     // bytes.
-    rope_build(tab, g, win, threadIdx.x - kCaTW0 * 32, kCaTW * 32);
+    const int tw = ca_transform_index(warp);
+    rope_build(tab, g, win, tw * 32 + lane, kCaTW * 32);
     named_barrier(1, kCaTW * 32);
-    const int tw = warp - kCaTW0;
     const int rg = tw_row(lane), j = tw_chunk(lane);
     LaneRope lr;
     lane_rope(g, j, smem_u32(tab), lr);
-    // The lane's two 16-byte chunks in the first row of each group parity:
-    // rows 16 tw + 4 u + rg have swizzle phase 4 (u & 1) + rg.
+    // The lane's two 16-byte chunks in rows rg and 4 + rg: a row group
+    // starting at row R (a multiple of 4) has swizzle phase 4 ((R >> 2) & 1) + rg.
     uint32_t ch0[2], ch1[2];
     lane_chunks(0, kCaBox, rg, j, ch0[0], ch1[0]);
     lane_chunks(0, kCaBox, 4 + rg, j, ch0[1], ch1[1]);
@@ -676,15 +685,17 @@ __global__ void __launch_bounds__(kCaThreads, 1)
           *reinterpret_cast<float4*>(zr_now + 16 * j + 4 * q) =
               *reinterpret_cast<const float4*>(zs + 4 * q);
       }
-      // Pass 1: this warp's sum of k_pls over its 16 rows.
+      // Pass 1: this warp's sum of k_pls over its rows.
       f2_t ta[8];
 #pragma unroll
       for (int i2 = 0; i2 < 8; ++i2) ta[i2] = 0ull;
 #pragma unroll 1
       for (int u = 0; u < kCaGroups; ++u) {
-        const uint32_t roff = (uint32_t)(kCaRowsW * tw + 4 * (u & ~1)) * 128u;
+        const int R = kCaRowsW * tw + 4 * u;
+        const uint32_t roff = (uint32_t)(R & ~7) * 128u;
+        const int ph = (R >> 2) & 1;
         f2_t x[8];
-        unpack8(lds128(kt + ch0[u & 1] + roff), lds128(kt + ch1[u & 1] + roff), x);
+        unpack8(lds128(kt + ch0[ph] + roff), lds128(kt + ch1[ph] + roff), x);
         const float rstd = row_rstd(x);
         const f2_t rstd2 = f2(rstd, rstd);
 #pragma unroll
@@ -742,9 +753,11 @@ __global__ void __launch_bounds__(kCaThreads, 1)
       // Pass 2: the transforms and the denominators, row group by row group.
 #pragma unroll 1
       for (int u = 0; u < kCaGroups; ++u) {
-        const int r = kCaRowsW * tw + 4 * u + rg;
-        const uint32_t roff = (uint32_t)(kCaRowsW * tw + 4 * (u & ~1)) * 128u;
-        const uint32_t c0 = ch0[u & 1] + roff, c1 = ch1[u & 1] + roff;
+        const int R = kCaRowsW * tw + 4 * u;
+        const int r = R + rg;
+        const uint32_t roff = (uint32_t)(R & ~7) * 128u;
+        const int ph = (R >> 2) & 1;
+        const uint32_t c0 = ch0[ph] + roff, c1 = ch1[ph] + roff;
         uint32_t t012 = 0, t345 = 0, t67 = 0;
         if (g.rope_on) lane_rope_row(lr, rec_s + r * kRecBytes, t012, t345, t67);
         const uint4 k0 = lds128(kt + c0), k1 = lds128(kt + c1);
@@ -820,7 +833,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
       if (lane == 0) mbar_arrive(tready);
     }
   } else if (warp < kCaOW0) {
-    // -------------------------------------------------------- chain warps
+    // -------------------------------------------------------- chain warps (8..11)
     // The two steps the MMA chain waits on: P = mask(A) * scale after the
     // first MMAs of a chunk, and the image of the state after its state MMA
     // (the next chunk's read-out operand).  Thread = TMEM lane = state row;
@@ -921,7 +934,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         if (!ok) break;
       }
     }
-  } else {
+  } else if (warp < kCaOW0 + kCaOW) {
     // ------------------------------------------------------- output warps
     // Thread = TMEM lane = token row 0..95 of the chunk:
     // x = sigmoid(g) * U / (den * scale), the output RMSNorm, bf16 stores.
