@@ -44,9 +44,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="720p", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", default="bidirectional", choices=["bidirectional", "causal"],
+    ap.add_argument("--variant", default="bidirectional", choices=["bidirectional", "causal", "mx"],
                     help="causal: the token-level causal read-out (gla_causal_step) of the "
-                         "workload, one step = one call from a zero state")
+                         "workload, one step = one call from a zero state; mx: gla_forward on "
+                         "FP8 (OCP MX) inputs")
     ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
@@ -324,6 +325,9 @@ def main():
         return
     if args.variant == "causal":
         run_causal(args, wl, gla, dev, dist, world, rank, local)
+        return
+    if args.variant == "mx":
+        run_mx(args, wl, gla, dev, dist, world, rank, local)
         return
 
     inp = workloads.make_inputs(wl, seed=replicas.replica_seed(wl.seed, rank))
@@ -618,6 +622,127 @@ def run_causal(args, wl, gla, dev, dist, world, rank, local):
             "gpu_launches": 3 * args.steps,
             "clocks": mon.summary(),
             "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_mx(args, wl, gla, dev, dist, world, rank, local):
+    """One step = one gla_forward_mx call on the workload with q, k, v, g in
+    FP8 (E4M3 codes, one E8M0 scale per 32 channels) and beta in bf16."""
+    xh = workloads.draw_mx(wl.batch, wl.tokens, wl.heads, wl.head_dim,
+                           replicas.replica_seed(wl.seed, rank))
+    x = {k: v.to(dev) for k, v in xh.items()}
+    B, N, Hh, hd = x["q"].shape
+    out = torch.empty(B, N, Hh, hd, dtype=torch.bfloat16, device=dev)
+    ws = gla.alloc_workspace(gla.lib().gla_forward_mx_workspace_size(B, Hh, hd, wl.T, wl.H, wl.W,
+                                                                     gla.GLA_PATH_AUTO), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        gla.gla_forward_mx(x, wl.T, wl.H, wl.W, wl.rope_theta, wl.eps, out=out, workspace=ws,
+                           stream=stream, events=events)
+
+    if args.profile:
+        for _ in range(args.warmup + args.steps):
+            step()
+        torch.cuda.synchronize(dev)
+        status = gla.gla_get_device_status(stream)
+        print(json.dumps({"profile_run": wl.name, "variant": "mx",
+                          "steps": args.warmup + args.steps, "status": gla.status_string(status)}))
+        if status != gla.GLA_OK:
+            sys.exit(1)
+        return
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert gla.gla_get_device_status(stream) == gla.GLA_OK
+
+    def sync():
+        torch.cuda.synchronize(dev)
+
+    def timed_steps():
+        for _ in range(args.steps):
+            step()
+
+    with ClockMonitor(local) as mon:
+        elapsed_ms, reps = timed_repeats(timed_steps, stream, dist, sync, dev, args.repeats)
+    if gla.gla_get_device_status(stream) != gla.GLA_OK:
+        raise RuntimeError("device status after the timed region")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e4 in evs:
+        for e in e4:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    k_state = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    k_comb = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    k_apply = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+
+    # End to end: the inputs from pinned host memory (one copy per tensor),
+    # the call, the output back, every step.
+    pinned = {k: v.pin_memory() for k, v in xh.items()}
+    out_h = torch.empty(B, N, Hh, hd, dtype=torch.bfloat16).pin_memory()
+
+    def host_step():
+        for k in x:
+            x[k].copy_(pinned[k], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 100))
+    host_step()
+
+    def host_steps():
+        for _ in range(e2e_steps):
+            host_step()
+
+    e2e_ms = replicas.timed(host_steps, replicas.CudaTimer(stream), dist, sync, dev)
+
+    th = B * N * Hh
+    ms_per_step = elapsed_ms / args.steps
+    peak, peak_kind = measured_peaks()
+    apply_bytes = th * (hd + 4) * 2 + th * hd * 2      # q, g codes + scales read, out written
+    state_bytes = th * (hd + 4) * 2 + th * 2           # k, v codes + scales, beta
+    alg = apply_bytes + state_bytes                     # 786 B per token-head at d = 128
+    apply_gbs = apply_bytes / (k_apply * 1e-3) / 1e9
+    step_gbs = alg / (ms_per_step * 1e-3) / 1e9
+    if rank == 0:
+        line = {
+            "metric": (f"gla_forward_mx tokens/s ({wl.heads}x{hd} heads, {wl.tokens} tok, "
+                       "FP8 MX inputs)"),
+            "value": replicas.aggregate_rate(world, B * N, args.steps, elapsed_ms),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "repeats": len(reps),
+            "repeat_ms_per_step": [round(r / args.steps, 5) for r in reps],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16",
+            "data": "synthetic",
+            "config": dict(workload_config(wl), inputs="q, k, v, g E4M3 + E8M0 per 32 channels, "
+                           "beta bf16, out bf16", parallelism=f"replicas x{world}"),
+            "roofline": {"bound": "hbm", "kernel": "tc_apply_mx_kernel", "achieved": apply_gbs,
+                         "peak": peak, "unit": "GB/s", "frac": apply_gbs / peak,
+                         "peak_kind": peak_kind,
+                         "traffic": traffic_for("tc_apply_mx_kernel", wl.name),
+                         "alg_bytes_per_launch": apply_bytes, "ms_per_launch": k_apply},
+            "kernels_ms": {"tc_state_mx_kernel": k_state, "combine_kernel": k_comb,
+                           "tc_apply_mx_kernel": k_apply,
+                           "how": "second timed pass of the same K steps, events around each kernel"},
+            "kernels_gbs": {"tc_state_mx_kernel": state_bytes / (k_state * 1e-3) / 1e9,
+                            "tc_apply_mx_kernel": apply_gbs},
+            "hbm_gbs_per_gpu": step_gbs, "step_frac_of_peak": step_gbs / peak,
+            "alg_bytes_per_step": alg,
+            "e2e": {"value": replicas.aggregate_rate(world, B * N, e2e_steps, e2e_ms),
+                    "unit": "tokens/s", "h2d_bytes_per_step": state_bytes + th * (hd + 4) * 2,
+                    "d2h_bytes_per_step": th * hd * 2, "steps": e2e_steps,
+                    "via": "one torch copy per input tensor from pinned memory, gla_forward_mx, "
+                           "one copy of the output back"},
+            "gpu_launches": 3 * args.steps,
+            "clocks": mon.summary(),
+            "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)
     if dist:

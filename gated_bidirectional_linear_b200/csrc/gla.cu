@@ -16,6 +16,7 @@
 #include "simt.cuh"
 #include "tc.cuh"
 #include "causal.cuh"
+#include "mx.cuh"
 
 using namespace gla;
 
@@ -623,6 +624,94 @@ gla_status gla_causal_step(float* state, float* z, const void* q, const void* k,
   return gla_causal_step_ex(state, z, q, k, v, beta, g, batch, heads, head_dim, T, H, W, t0,
                             rope_theta, eps, dtype, out, workspace, workspace_bytes, stream,
                             GLA_PATH_AUTO, nullptr, nullptr);
+}
+
+size_t gla_forward_mx_workspace_size(int batch, int heads, int head_dim, int T, int H, int W,
+                                     int path) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W) || head_dim != 128) return 0;
+  const size_t ws = ws_layout(batch * heads, head_dim, true, T, H, W).total;
+  if (path != GLA_PATH_SIMT) return ws;
+  // The CUDA-core path decodes q, k, v and g to bf16 first.
+  const size_t n = (size_t)batch * T * H * W * heads * head_dim;
+  return 4 * align_up(n * 2, kAlign) + ws;
+}
+
+gla_status gla_forward_mx_ex(const void* q, const void* q_scale, const void* k,
+                             const void* k_scale, const void* v, const void* v_scale,
+                             const void* beta, const void* g, const void* g_scale, int batch,
+                             int heads, int head_dim, int T, int H, int W, float rope_theta,
+                             float eps, void* out, void* workspace, size_t workspace_bytes,
+                             void* stream, int path, float* S_out, float* z_out,
+                             float* den_out, float* x_out, void* const* events) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W)) return GLA_ERR_INVALID_ARG;
+  if (head_dim != 128) return GLA_ERR_UNSUPPORTED;
+  if (!(eps > 0.f) || !isfinite(eps) || !isfinite(rope_theta)) return GLA_ERR_INVALID_ARG;
+  const void* ptrs[10] = {q, q_scale, k, k_scale, v, v_scale, beta, g, g_scale, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return GLA_ERR_INVALID_ARG;
+  if (path != GLA_PATH_AUTO && path != GLA_PATH_SIMT && path != GLA_PATH_TENSOR)
+    return GLA_ERR_UNSUPPORTED;
+  const size_t need = gla_forward_mx_workspace_size(batch, heads, head_dim, T, H, W, path);
+  if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < need)
+    return GLA_ERR_WORKSPACE;
+  const Geom geom = make_geom(batch, heads, head_dim, T, H, W, 0, rope_theta, eps);
+  const int sms = device_sm_count();
+  if (sms <= 0) return GLA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (path == GLA_PATH_SIMT) {
+    // Decode to bf16 (exact: E4M3 values times powers of two), then the
+    // bf16 CUDA-core kernels.
+    const size_t n = (size_t)batch * T * H * W * heads * head_dim;
+    const void* codes[4] = {q, k, v, g};
+    const void* scales[4] = {q_scale, k_scale, v_scale, g_scale};
+    unsigned char* dec[4];
+    for (int i = 0; i < 4; ++i) {
+      dec[i] = ws + i * align_up(n * 2, kAlign);
+      mx_decode_kernel<<<4 * sms, 256, 0, st>>>(static_cast<const uint8_t*>(codes[i]),
+                                                static_cast<const uint8_t*>(scales[i]),
+                                                reinterpret_cast<__nv_bfloat16*>(dec[i]), n);
+      if (cudaGetLastError() != cudaSuccess) return GLA_ERR_CUDA;
+    }
+    unsigned char* rest = ws + 4 * align_up(n * 2, kAlign);
+    return forward_common(dec[0], dec[1], dec[2], beta, dec[3], batch, heads, head_dim, T, H, W,
+                          rope_theta, eps, GLA_DTYPE_BF16, out, rest,
+                          workspace_bytes - (size_t)(rest - ws), stream, GLA_PATH_SIMT, S_out,
+                          z_out, den_out, x_out, events);
+  }
+  const WsLayout L = ws_layout(batch * heads, head_dim, true, T, H, W);
+  MxInputs in = {q, q_scale, k, k_scale, v, v_scale, g, g_scale};
+  float* S = reinterpret_cast<float*>(ws + L.S);
+  float* z = reinterpret_cast<float*>(ws + L.z);
+  gla_status r = run_tensor_mx(geom, in, beta, out, S, z, S_out != nullptr,
+                               reinterpret_cast<float*>(ws + L.part_S),
+                               reinterpret_cast<float*>(ws + L.part_z),
+                               reinterpret_cast<__half*>(ws + L.S_img),
+                               reinterpret_cast<float*>(ws + L.S_scale),
+                               reinterpret_cast<float2*>(ws + L.rope_tab), den_out, x_out, sms, st,
+                               events);
+  if (r == GLA_ERR_UNSUPPORTED && path == GLA_PATH_AUTO)
+    return gla_forward_mx_ex(q, q_scale, k, k_scale, v, v_scale, beta, g, g_scale, batch, heads,
+                             head_dim, T, H, W, rope_theta, eps, out, workspace, workspace_bytes,
+                             stream, GLA_PATH_SIMT, S_out, z_out, den_out, x_out, events);
+  if (r != GLA_OK) return r;
+  const size_t dd = (size_t)batch * heads * head_dim * head_dim;
+  const size_t dz = (size_t)batch * heads * head_dim;
+  if (S_out && cudaMemcpyAsync(S_out, S, dd * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  if (z_out && cudaMemcpyAsync(z_out, z, dz * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return GLA_ERR_CUDA;
+  return GLA_OK;
+}
+
+gla_status gla_forward_mx(const void* q, const void* q_scale, const void* k, const void* k_scale,
+                          const void* v, const void* v_scale, const void* beta, const void* g,
+                          const void* g_scale, int batch, int heads, int head_dim, int T, int H,
+                          int W, float rope_theta, float eps, void* out, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  return gla_forward_mx_ex(q, q_scale, k, k_scale, v, v_scale, beta, g, g_scale, batch, heads,
+                           head_dim, T, H, W, rope_theta, eps, out, workspace, workspace_bytes,
+                           stream, GLA_PATH_AUTO, nullptr, nullptr, nullptr, nullptr, nullptr);
 }
 
 size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, int T, int H, int W,

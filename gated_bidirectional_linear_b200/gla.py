@@ -48,6 +48,10 @@ _SIGS = {
                               + [_vp] * 2 + [ctypes.POINTER(_vp)]),
     "gla_causal_host_arena_size": (_sz, [_i] * 7),
     "gla_causal_step_host": (_i, [_vp] * 7 + [_i] * 7 + [_f, _f, _i, _vp, _vp, _sz, _vp]),
+    "gla_forward_mx_workspace_size": (_sz, [_i] * 7),
+    "gla_forward_mx": (_i, [_vp] * 9 + [_i] * 6 + [_f, _f, _vp, _vp, _sz, _vp]),
+    "gla_forward_mx_ex": (_i, [_vp] * 9 + [_i] * 6 + [_f, _f, _vp, _vp, _sz, _vp, _i]
+                          + [_vp] * 4 + [ctypes.POINTER(_vp)]),
     "gla_forward_noalloc": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp]),
     "gla_get_device_status": (_i, [_vp]),
     "gla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
@@ -415,6 +419,64 @@ def gla_causal_forward(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, 
     z = torch.zeros(B, Hh, d, dtype=torch.float32, device=q.device)
     return gla_causal_step(state, z, q, k, v, beta, g, T, H, W, 0, rope_theta, eps, out=out,
                            workspace=workspace, stream=stream, path=path)
+
+
+MX_NAMES = ("q", "q_scale", "k", "k_scale", "v", "v_scale", "beta", "g", "g_scale")
+
+
+def gla_forward_mx(x, T, H, W, rope_theta=10000.0, eps=1e-6, out=None, workspace=None,
+                   stream=None, path=GLA_PATH_AUTO, debug=False, events=None):
+    """The operator on FP8 (OCP MX) inputs.  x: dict with uint8 codes q, k, v,
+    g [B, N, Hh, 128] and uint8 E8M0 scales q_scale .. g_scale [B, N, Hh, 4]
+    (one per 32 channels), and bf16 beta [B, N, Hh], all on one GPU.  Returns
+    the bf16 output, or with debug=True dict(out, S, z, den, x) like
+    gla_forward_debug.  events: four torch.cuda.Event objects recorded around
+    the kernels (as gla_forward_timed)."""
+    q = x["q"]
+    if q.dim() != 4 or q.shape[-1] != 128:
+        raise ValueError(f"q codes must be [B, N, heads, 128], got {tuple(q.shape)}")
+    B, N, Hh, d = q.shape
+    if N != T * H * W:
+        raise ValueError(f"q has {N} tokens, grid {T}x{H}x{W} has {T * H * W}")
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError(f"q is on {dev}; this entry point takes GPU tensors")
+    shapes = {"q": (B, N, Hh, d), "k": (B, N, Hh, d), "v": (B, N, Hh, d), "g": (B, N, Hh, d),
+              "q_scale": (B, N, Hh, d // 32), "k_scale": (B, N, Hh, d // 32),
+              "v_scale": (B, N, Hh, d // 32), "g_scale": (B, N, Hh, d // 32), "beta": (B, N, Hh)}
+    for name, shape in shapes.items():
+        t = x.get(name)
+        want = torch.bfloat16 if name == "beta" else torch.uint8
+        if t is None:
+            raise ValueError(f"{name} is missing")
+        if tuple(t.shape) != shape or t.dtype != want or t.device != dev or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {want} tensor of shape {shape} on {dev}")
+    if out is None:
+        out = torch.empty(B, N, Hh, d, dtype=torch.bfloat16, device=dev)
+    if tuple(out.shape) != (B, N, Hh, d) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor of the input shape")
+    if workspace is None:
+        workspace = alloc_workspace(lib().gla_forward_mx_workspace_size(B, Hh, d, T, H, W, path),
+                                    dev)
+    _check_workspace(workspace, dev)
+    dbg = {}
+    if debug:
+        dbg = dict(S=torch.empty(B, Hh, d, d, dtype=torch.float32, device=dev),
+                   z=torch.empty(B, Hh, d, dtype=torch.float32, device=dev),
+                   den=torch.empty(B, N, Hh, dtype=torch.float32, device=dev),
+                   x=torch.empty(B, N, Hh, d, dtype=torch.float32, device=dev))
+    ev = None
+    if events is not None:
+        ev = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) if e is not None else None
+                                     for e in events])
+    with _on(dev):
+        st = lib().gla_forward_mx_ex(*[_ptr(x[n]) for n in MX_NAMES], B, Hh, d, T, H, W,
+                                     rope_theta, eps, _ptr(out), _ptr(workspace),
+                                     workspace.numel(), _stream(stream, dev), path,
+                                     _ptr(dbg.get("S")), _ptr(dbg.get("z")), _ptr(dbg.get("den")),
+                                     _ptr(dbg.get("x")), ev)
+    _check(st, "gla_forward_mx")
+    return dict(out=out, **dbg) if debug else out
 
 
 def gla_forward_noalloc(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, out=None,

@@ -91,6 +91,45 @@ def draw(batch, tokens, heads, head_dim, dtype, seed):
     return out
 
 
+MX_BLOCK = 32          # elements per shared scale (OCP MX)
+E4M3_EMAX = 8          # exponent of E4M3's largest power of two (448 = 1.75 * 2^8)
+
+
+def mx_encode(x):
+    """OCP MX encoding of a float array along its last axis, as the inputs of
+    the FP8 operator arrive: per block of 32 consecutive elements one E8M0
+    shared exponent X = floor(log2(max |x|)) - 8 (biased by 127; a block of
+    zeros takes the smallest), elements x / 2^X rounded to nearest-even E4M3
+    and clamped to +-448.  Returns (codes uint8 [..., d], scales uint8
+    [..., d/32]) as CPU torch tensors."""
+    x = np.asarray(x, dtype=np.float32)
+    d = x.shape[-1]
+    blocks = x.reshape(x.shape[:-1] + (d // MX_BLOCK, MX_BLOCK))
+    amax = np.max(np.abs(blocks), axis=-1)
+    with np.errstate(divide="ignore"):
+        e = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))), -127.0)
+    X = np.clip(e - E4M3_EMAX, -127, 127)
+    elems = np.clip(blocks / np.exp2(X)[..., None], -448.0, 448.0).astype(np.float32)
+    codes = torch.from_numpy(np.ascontiguousarray(elems.reshape(x.shape))).to(
+        torch.float8_e4m3fn).view(torch.uint8)
+    scales = torch.from_numpy((X + 127).astype(np.uint8))
+    return codes, scales
+
+
+def draw_mx(batch, tokens, heads, head_dim, seed):
+    """Seeded MX inputs: the same draws as draw() (q, k, v, g ~ N(0, 1), beta
+    = logistic(N(0, 1))) with q, k, v and g MX-encoded and beta in bf16.
+    Returns dict(q, q_scale, k, k_scale, v, v_scale, g, g_scale, beta)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    shape = (batch, tokens, heads, head_dim)
+    out = {}
+    for name in ("q", "k", "v", "g"):
+        out[name], out[name + "_scale"] = mx_encode(rng.standard_normal(shape, dtype=np.float32))
+    logits = rng.standard_normal(shape[:3], dtype=np.float64)
+    out["beta"] = _round((1.0 / (1.0 + np.exp(-logits))).astype(np.float32), "bf16")
+    return out
+
+
 def make_inputs(wl: Workload, seed=None):
     """Inputs of a workload over all of its tokens (all blocks)."""
     return draw(wl.batch, wl.total_tokens, wl.heads, wl.head_dim, wl.dtype,

@@ -232,6 +232,49 @@ GLA_API gla_status gla_causal_step_timed(float* state, float* z, const void* q, 
                                          void* stream, int path, float* den_out, float* x_out,
                                          void* const* events);
 
+/* ------------------------------------------------------------------------
+ * FP8 operator inputs (OCP microscaling "MX" format).  The SANA-Video 2.0
+ * summary (results and limitations) trains with MXFP8 activations for the
+ * GEMMs, keeps attention in BF16 and names low-precision attention kernels as
+ * future work; these entry points take the operator's q, k, v and g in that
+ * activation format.  q, k, v, g: E4M3 codes [batch][N][heads][128], one byte
+ * per element (sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities, S.1111.111 is NaN); q_scale .. g_scale: E8M0 scales
+ * [batch][N][heads][4], one byte per 32 consecutive channels (value
+ * 2^(byte - 127)).  Element i of a row is e4m3(code_i) * 2^(scale[i / 32] -
+ * 127).  beta stays bf16 [batch][N][heads]; out is bf16 [batch][N][heads][128].
+ * The operator is gla_forward's, on the decoded values (which bf16 represents
+ * exactly).  head_dim 128 only.  All pointers 16-byte aligned device memory. */
+
+/* Workspace bytes of gla_forward_mx_ex for `path` (GLA_PATH_SIMT also holds
+ * the inputs decoded to bf16); 0 for invalid sizes. */
+GLA_API size_t gla_forward_mx_workspace_size(int batch, int heads, int head_dim, int T, int H,
+                                             int W, int path);
+
+/* The bidirectional operator on MX inputs (tensor path: the state reduction
+ * and read-out decode the fp8 tiles in their transform warps). */
+GLA_API gla_status gla_forward_mx(const void* q, const void* q_scale, const void* k,
+                                  const void* k_scale, const void* v, const void* v_scale,
+                                  const void* beta, const void* g, const void* g_scale,
+                                  int batch, int heads, int head_dim, int T, int H, int W,
+                                  float rope_theta, float eps, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* gla_forward_mx with an explicit path (GLA_PATH_SIMT decodes the inputs to
+ * bf16 in the workspace and runs the CUDA-core kernels), the hidden
+ * intermediates of gla_forward_debug (S_out, z_out, den_out, x_out, each may
+ * be NULL) and the kernel events of gla_forward_timed (`events` may be NULL).
+ * GLA_PATH_AUTO falls back to the CUDA-core path where the tensor path does
+ * not fit, if the workspace is large enough for it. */
+GLA_API gla_status gla_forward_mx_ex(const void* q, const void* q_scale, const void* k,
+                                     const void* k_scale, const void* v, const void* v_scale,
+                                     const void* beta, const void* g, const void* g_scale,
+                                     int batch, int heads, int head_dim, int T, int H, int W,
+                                     float rope_theta, float eps, void* out, void* workspace,
+                                     size_t workspace_bytes, void* stream, int path,
+                                     float* S_out, float* z_out, float* den_out, float* x_out,
+                                     void* const* events);
+
 /* Bytes of the device arena gla_causal_step_host needs: room for the call's
  * five inputs, its output and its workspace. */
 GLA_API size_t gla_causal_host_arena_size(int batch, int heads, int head_dim, int T, int H,
