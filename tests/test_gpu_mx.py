@@ -69,7 +69,7 @@ EDGE = [
     (1, 2, 2, 4, 4, 1e4),       # 32 tokens
     (2, 3, 1, 1, 1, 1e4),       # one token per head
     (1, 5, 1, 10, 10, 1e4),     # N = 100 < one tile
-    (2, 3, 1, 1, 257, 1e4),     # a one-token ragged tail
+    (2, 3, 5, 7, 11, 1e4),      # N = 385: a one-token tail for 96- and 128-token tiles
     (1, 2, 10, 32, 40, 1e4),    # CTAs straddle the head boundary
     (1, 3, 7, 9, 11, 0.0),      # RoPE off
 ]
