@@ -430,13 +430,13 @@ __global__ void __launch_bounds__(kMxApThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kApQ; ++s) {
-      mbar_init(&qfull[s], 1);
+      mbar_init(&qfull[s], 2);      // TMA bytes + the producer's scales / records
       mbar_init(&q8free[s], kApTW);
       mbar_init(&qtfree[s], 1);
       mbar_init(&qready[s], kApTW);
     }
     for (int s = 0; s < kMxApG; ++s) {
-      mbar_init(&gfull[s], 1);
+      mbar_init(&gfull[s], 2);      // TMA bytes + the producer's scales
       mbar_init(&gempty[s], kApEW);
     }
     for (int a = 0; a < kApAcc; ++a) {
@@ -480,6 +480,11 @@ __global__ void __launch_bounds__(kMxApThreads, 1)
       const int s = rq.s;
       if (!mbar_wait_warp(&q8free[s], rq.ph ^ 1u, abort_flag)) break;
       const int n0 = iw.ti * kTcTile;
+      // The tile copy first; the scales and row records land while it flies.
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&qfull[s], kMxApIn);
+        tma_load_3d(sm + TcApplyMxSmem::Q8 + s * kMxApIn, &tmQ, &qfull[s], h * 128, n0, b, pol);
+      }
       uint32_t* qs = reinterpret_cast<uint32_t*>(sm + TcApplyMxSmem::QSC + s * 512);
 #pragma unroll
       for (int k2 = 0; k2 < kTcTile / 32; ++k2) {
@@ -489,10 +494,7 @@ __global__ void __launch_bounds__(kMxApThreads, 1)
       if (g.rope_on)
         tile_rowrec<kTcTile>(g, win, n0, lane, sm + TcApplyMxSmem::ROWREC + s * kTcTile * kRecBytes);
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&qfull[s], kMxApIn);
-        tma_load_3d(sm + TcApplyMxSmem::Q8 + s * kMxApIn, &tmQ, &qfull[s], h * 128, n0, b, pol);
-      }
+      if (lane == 0) mbar_arrive(&qfull[s]);
       ++issued;
       if (iw.first) {
         if (!combined) {
@@ -559,6 +561,10 @@ __global__ void __launch_bounds__(kMxApThreads, 1)
       }
       if (!mbar_wait_warp(&gempty[s], rg_.ph ^ 1u, abort_flag)) break;
       const int n0 = iw.ti * kTcTile;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&gfull[s], kMxApIn);
+        tma_load_3d(sm + TcApplyMxSmem::G8 + s * kMxApIn, &tmG, &gfull[s], h * 128, n0, b, pol);
+      }
       uint32_t* gs = reinterpret_cast<uint32_t*>(sm + TcApplyMxSmem::GSC + s * 512);
 #pragma unroll
       for (int k2 = 0; k2 < kTcTile / 32; ++k2) {
@@ -566,10 +572,7 @@ __global__ void __launch_bounds__(kMxApThreads, 1)
         gs[r] = n < g.N ? p.g_scale[((size_t)b * g.N + n) * g.Hh + h] : 0u;
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&gfull[s], kMxApIn);
-        tma_load_3d(sm + TcApplyMxSmem::G8 + s * kMxApIn, &tmG, &gfull[s], h * 128, n0, b, pol);
-      }
+      if (lane == 0) mbar_arrive(&gfull[s]);
       ++issued;
     }
     if (*abort_flag && lane == 0) {
