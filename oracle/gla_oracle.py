@@ -384,6 +384,42 @@ def forward_mx(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
     return forward(dq(q), dq(k), dq(v), beta, dq(g), T, H, W, rope_theta, eps, t0)
 
 
+# ----------------------------------------------- the layer's projections
+
+# [GBLA] writes the read-out as o_j = W_o RMSNorm[...]: the heads' normalised
+# read-outs, concatenated over the heads (the width Hh*d), times W_o.  The
+# pages print no input projection; reading: q, k, v, g and the beta logits
+# are one linear map of the layer input x (rows of W_in in that order: Hh*d
+# rows each for q, k, v and g, then Hh rows of beta logits), with beta =
+# sigmoid(logits) and g left as logits (the operator applies its sigmoid).
+
+def project_in(x, W_in, heads, head_dim):
+    """x [B, N, C], W_in [4*Hh*d + Hh, C] -> dict(q, k, v, g [B, N, Hh, d],
+    beta [B, N, Hh]) with beta = sigmoid(x W_beta^T)."""
+    B, N, _ = x.shape
+    hd = heads * head_dim
+    y = x @ W_in.T
+    out = {}
+    for i, name in enumerate("qkvg"):
+        out[name] = y[..., i * hd:(i + 1) * hd].reshape(B, N, heads, head_dim)
+    out["beta"] = sigmoid(y[..., 4 * hd:4 * hd + heads])
+    return out
+
+
+def project_out(o, W_o):
+    """o [B, N, Hh, d] (the operator's output) -> o_flat W_o^T, [B, N, C_out]
+    with W_o [C_out, Hh*d]."""
+    B, N, Hh, d = o.shape
+    return o.reshape(B, N, Hh * d) @ W_o.T
+
+
+def layer_forward(x, W_in, W_o, heads, head_dim, T, H, W, rope_theta, eps):
+    """x -> projections -> the bidirectional operator -> W_o."""
+    p = project_in(x, W_in, heads, head_dim)
+    r = forward(p["q"], p["k"], p["v"], p["beta"], p["g"], T, H, W, rope_theta, eps)
+    return dict(y=project_out(r["out"], W_o), proj=p, op=r)
+
+
 # ------------------------------------------------------------- parity metric
 
 def max_err_over_rms(got, ref):

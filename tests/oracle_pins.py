@@ -392,6 +392,52 @@ def check_causal_carried_state():
     _close(second["out"], whole["out"][:, L:], 1e-12, "carried causal state")
 
 
+# ------------------------------------------------ the layer's projections
+
+def check_project_in_layout():
+    """One token, C = 2, Hh = 2, d = 2: W_in rows in the order q (4 rows), k,
+    v, g, then 2 beta-logit rows.  With x = (1, 2) each output is its row's
+    dot with x; q of head 1 is rows 2..3; beta = sigmoid of the last two."""
+    Hh, d, C = 2, 2, 2
+    rows = 4 * Hh * d + Hh
+    W_in = np.zeros((rows, C))
+    for r in range(rows):
+        W_in[r] = (r, 1.0)                 # row r . (1, 2) = r + 2
+    x = np.array([[[1.0, 2.0]]])
+    p = O.project_in(x, W_in, Hh, d)
+    want = {"q": [2, 3, 4, 5], "k": [6, 7, 8, 9], "v": [10, 11, 12, 13], "g": [14, 15, 16, 17]}
+    for name, w in want.items():
+        _close(p[name].ravel(), w, 0.0, f"project_in {name}")
+    assert p["q"].shape == (1, 1, Hh, d)
+    _close(p["q"][0, 0, 1], [4, 5], 0.0, "q of head 1")
+    _close(p["beta"].ravel(), [1 / (1 + math.exp(-18)), 1 / (1 + math.exp(-19))], 1e-15,
+           "beta = sigmoid(logits)")
+
+
+def check_project_out_layout():
+    """o [1, 1, Hh=2, d=2] = (1, 2 | 3, 4) flattened head-major; W_o rows pick
+    single entries: W_o = [[0,0,1,0], [1,1,1,1]] -> (3, 10)."""
+    o = np.array([1.0, 2.0, 3.0, 4.0]).reshape(1, 1, 2, 2)
+    W_o = np.array([[0.0, 0.0, 1.0, 0.0], [1.0, 1.0, 1.0, 1.0]])
+    _close(O.project_out(o, W_o).ravel(), [3.0, 10.0], 0.0, "project_out")
+
+
+def check_layer_is_the_composition():
+    """layer_forward = W_o applied to the operator of the projections."""
+    rng = np.random.default_rng(3)
+    Hh, d, C, T, H, W = 2, 8, 6, 2, 2, 2
+    N = T * H * W
+    x = rng.standard_normal((1, N, C))
+    W_in = rng.standard_normal((4 * Hh * d + Hh, C)) * 0.3
+    W_o = rng.standard_normal((5, Hh * d))
+    r = O.layer_forward(x, W_in, W_o, Hh, d, T, H, W, 1e4, 1e-5)
+    y = x @ W_in.T
+    q, k, v, g = (y[..., i * Hh * d:(i + 1) * Hh * d].reshape(1, N, Hh, d) for i in range(4))
+    beta = 1 / (1 + np.exp(-y[..., 4 * Hh * d:]))
+    op = O.forward(q, k, v, beta, g, T, H, W, 1e4, 1e-5)
+    _close(r["y"], op["out"].reshape(1, N, Hh * d) @ W_o.T, 1e-12, "layer composition")
+
+
 # ---------------------------------------------------- MXFP8 input decoding
 
 def check_e4m3_format_values():

@@ -130,6 +130,24 @@ def _causal_at_no_carry(q, k, v, beta, g, T, H, W, rope_theta, eps, tokens, t0=0
     return _orig["causal_forward_at"](q, k, v, beta, g, T, H, W, rope_theta, eps, tokens, t0)
 
 
+def _project_in_no_sigmoid(x, W_in, heads, head_dim):
+    p = _orig["project_in"](x, W_in, heads, head_dim)
+    y = x @ W_in.T
+    p["beta"] = y[..., 4 * heads * head_dim:4 * heads * head_dim + heads]
+    return p
+
+
+def _project_in_qk_swapped(x, W_in, heads, head_dim):
+    p = _orig["project_in"](x, W_in, heads, head_dim)
+    p["q"], p["k"] = p["k"], p["q"]
+    return p
+
+
+def _project_out_transposed(o, W_o):
+    B, N, Hh, d = o.shape
+    return np.swapaxes(o, 2, 3).reshape(B, N, Hh * d) @ W_o.T
+
+
 def _e4m3_bias8(codes):
     return _orig["e4m3_decode"](codes) / 2.0
 
@@ -173,6 +191,9 @@ MUTANTS = {
     "causal_suffix": ("causal_forward", _causal_suffix),
     "causal_at_exclusive": ("causal_forward_at", _causal_at_exclusive),
     "causal_at_no_carry": ("causal_forward_at", _causal_at_no_carry),
+    "project_in_no_sigmoid": ("project_in", _project_in_no_sigmoid),
+    "project_in_qk_swapped": ("project_in", _project_in_qk_swapped),
+    "project_out_channel_major": ("project_out", _project_out_transposed),
     "e4m3_bias8": ("e4m3_decode", _e4m3_bias8),
     "e4m3_no_subnormals": ("e4m3_decode", _e4m3_no_subnormals),
     "e8m0_bias128": ("e8m0_decode", _e8m0_bias128),
