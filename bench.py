@@ -44,10 +44,12 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="720p", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--variant", default="bidirectional", choices=["bidirectional", "causal", "mx"],
+    ap.add_argument("--variant", default="bidirectional",
+                    choices=["bidirectional", "causal", "mx", "layer"],
                     help="causal: the token-level causal read-out (gla_causal_step) of the "
                          "workload, one step = one call from a zero state; mx: gla_forward on "
-                         "FP8 (OCP MX) inputs")
+                         "FP8 (OCP MX) inputs; layer: input projection, gla_forward and W_o "
+                         "(gla_layer_forward) at the workload's width")
     ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
@@ -328,6 +330,9 @@ def main():
         return
     if args.variant == "mx":
         run_mx(args, wl, gla, dev, dist, world, rank, local)
+        return
+    if args.variant == "layer":
+        run_layer(args, wl, gla, dev, dist, world, rank, local)
         return
 
     inp = workloads.make_inputs(wl, seed=replicas.replica_seed(wl.seed, rank))
@@ -741,6 +746,122 @@ def run_mx(args, wl, gla, dev, dist, world, rank, local):
                     "via": "one torch copy per input tensor from pinned memory, gla_forward_mx, "
                            "one copy of the output back"},
             "gpu_launches": 3 * args.steps,
+            "clocks": mon.summary(),
+            "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measured_tflops(sustained=True):
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops_sustained" if sustained else "bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return (1400.0 if sustained else 1590.0), "fallback"
+
+
+def run_layer(args, wl, gla, dev, dist, world, rank, local):
+    """One step = gla_layer_forward on the workload: x [tokens, C] (C = heads *
+    head_dim, the model width) -> q, k, v, g, beta by one projection GEMM whose
+    epilogue writes the operator's inputs -> gla_forward -> W_o.  Synthetic
+    bf16 x ~ N(0, 1) and weights ~ N(0, 1/fan_in)."""
+    Hh, d = wl.heads, wl.head_dim
+    C = Hh * d
+    tokens = wl.batch * wl.tokens
+    rng = np.random.Generator(np.random.PCG64(replicas.replica_seed(wl.seed, rank) + 100))
+    mk = lambda shape, sc: torch.from_numpy(rng.standard_normal(shape, dtype=np.float32) * sc).to(
+        torch.bfloat16).to(dev)
+    x = mk((tokens, C), 1.0)
+    W_in = mk((4 * C + Hh, C), C ** -0.5)
+    W_o = mk((C, C), C ** -0.5)
+    y = torch.empty(tokens, C, dtype=torch.bfloat16, device=dev)
+    ws = gla.alloc_workspace(gla.lib().gla_layer_workspace_size(wl.batch, Hh, d, wl.T, wl.H, wl.W),
+                             dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gla.gla_layer_forward(x, W_in, W_o, wl.batch, Hh, d, wl.T, wl.H, wl.W, wl.rope_theta,
+                              wl.eps, out=y, workspace=ws, stream=stream)
+
+    if args.profile:
+        for _ in range(args.warmup + args.steps):
+            step()
+        torch.cuda.synchronize(dev)
+        status = gla.gla_get_device_status(stream)
+        print(json.dumps({"profile_run": wl.name, "variant": "layer",
+                          "steps": args.warmup + args.steps, "status": gla.status_string(status)}))
+        if status != gla.GLA_OK:
+            sys.exit(1)
+        return
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert gla.gla_get_device_status(stream) == gla.GLA_OK
+
+    def sync():
+        torch.cuda.synchronize(dev)
+
+    steps = max(1, args.steps // 10)
+
+    def timed_steps():
+        for _ in range(steps):
+            step()
+
+    with ClockMonitor(local) as mon:
+        elapsed_ms, reps = timed_repeats(timed_steps, stream, dist, sync, dev, args.repeats)
+    if gla.gla_get_device_status(stream) != gla.GLA_OK:
+        raise RuntimeError("device status after the timed region")
+
+    # Per stage, events around the three calls (the stages then do not overlap).
+    p = {}
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    t_in, t_op, t_out = [], [], []
+    for _ in range(steps):
+        ev[0].record(stream)
+        p = gla.gla_project_in(x, W_in, wl.batch, wl.tokens, Hh, d, stream=stream)
+        ev[1].record(stream)
+        o = gla.gla_forward(p["q"], p["k"], p["v"], p["beta"], p["g"], wl.T, wl.H, wl.W,
+                            wl.rope_theta, wl.eps, stream=stream)
+        ev[2].record(stream)
+        gla.gla_gemm_bf16(o.view(tokens, C), W_o, out=y, stream=stream)
+        ev[3].record(stream)
+        torch.cuda.synchronize(dev)
+        t_in.append(ev[0].elapsed_time(ev[1]))
+        t_op.append(ev[1].elapsed_time(ev[2]))
+        t_out.append(ev[2].elapsed_time(ev[3]))
+    k_in, k_op, k_out = (float(np.median(t)) for t in (t_in, t_op, t_out))
+
+    ms_per_step = elapsed_ms / steps
+    flops_in = 2.0 * tokens * (4 * C + Hh) * C
+    flops_out = 2.0 * tokens * C * C
+    peak, peak_kind = measured_tflops(sustained=True)
+    in_tf = flops_in / (k_in * 1e-3) / 1e12
+    if rank == 0:
+        line = {
+            "metric": (f"gla_layer_forward tokens/s (width {C}, {Hh}x{d} heads, {wl.tokens} tok: "
+                       "projection, operator, W_o)"),
+            "value": replicas.aggregate_rate(world, tokens, steps, elapsed_ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "repeats": len(reps), "repeat_ms_per_step": [round(r / steps, 5) for r in reps],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(workload_config(wl), layer=(f"x [{tokens}, {C}], W_in [{4 * C + Hh}, "
+                                                       f"{C}], W_o [{C}, {C}], N(0, 1/fan_in)"),
+                           parallelism=f"replicas x{world}"),
+            "roofline": {"bound": "tensor", "kernel": "gemm_kernel (input projection)",
+                         "achieved": in_tf, "peak": peak, "unit": "TFLOP/s", "frac": in_tf / peak,
+                         "peak_kind": peak_kind + " sustained bf16",
+                         "traffic": None, "alg_flops_per_launch": flops_in, "ms_per_launch": k_in},
+            "stages_ms": {"project_in": k_in, "gla_forward": k_op, "project_out": k_out,
+                          "how": "events around each of the three calls, per step, median"},
+            "stages_tflops": {"project_in": in_tf,
+                              "project_out": flops_out / (k_out * 1e-3) / 1e12},
+            "e2e": None,
+            "gpu_launches": 5 * steps,
             "clocks": mon.summary(),
             "cpu_baseline": None,
         }

@@ -17,6 +17,7 @@
 #include "tc.cuh"
 #include "causal.cuh"
 #include "mx.cuh"
+#include "gemm.cuh"
 
 using namespace gla;
 
@@ -712,6 +713,71 @@ gla_status gla_forward_mx(const void* q, const void* q_scale, const void* k, con
   return gla_forward_mx_ex(q, q_scale, k, k_scale, v, v_scale, beta, g, g_scale, batch, heads,
                            head_dim, T, H, W, rope_theta, eps, out, workspace, workspace_bytes,
                            stream, GLA_PATH_AUTO, nullptr, nullptr, nullptr, nullptr, nullptr);
+}
+
+gla_status gla_gemm_bf16(const void* A, const void* B, void* C, int M, int N, int K,
+                         void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0 || K % 8 || N % 8) return GLA_ERR_INVALID_ARG;
+  if (!A || !B || !C || !aligned16(A) || !aligned16(B) || !aligned16(C)) return GLA_ERR_INVALID_ARG;
+  GemmParams p = {};
+  p.M = M; p.N = N; p.K = K; p.mode = kGemmPlain;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  return run_gemm(A, B, p, device_sm_count(), static_cast<cudaStream_t>(stream));
+}
+
+gla_status gla_project_in(const void* x, const void* W_in, int tokens, int C, int heads,
+                          int head_dim, void* q, void* k, void* v, void* g, void* beta,
+                          void* stream) {
+  if (tokens <= 0 || C <= 0 || C % 8 || heads <= 0 || head_dim <= 0) return GLA_ERR_INVALID_ARG;
+  const int HD = heads * head_dim;
+  if (HD % 32) return GLA_ERR_UNSUPPORTED;
+  const void* ptrs[8] = {x, W_in, q, k, v, g, beta, nullptr};
+  for (int i = 0; i < 7; ++i)
+    if (!ptrs[i] || !aligned16(ptrs[i])) return GLA_ERR_INVALID_ARG;
+  GemmParams p = {};
+  p.M = tokens; p.N = 4 * HD + heads; p.K = C; p.mode = kGemmSplit;
+  p.dst[0] = static_cast<__nv_bfloat16*>(q);
+  p.dst[1] = static_cast<__nv_bfloat16*>(k);
+  p.dst[2] = static_cast<__nv_bfloat16*>(v);
+  p.dst[3] = static_cast<__nv_bfloat16*>(g);
+  p.beta = static_cast<__nv_bfloat16*>(beta);
+  p.HD = HD; p.heads = heads;
+  return run_gemm(x, W_in, p, device_sm_count(), static_cast<cudaStream_t>(stream));
+}
+
+// Layer workspace: q, k, v, g, the operator's output (tokens x HD bf16 each),
+// beta (tokens x heads bf16), then the operator's own workspace.
+size_t gla_layer_workspace_size(int batch, int heads, int head_dim, int T, int H, int W) {
+  const size_t op = gla_forward_workspace_size(batch, heads, head_dim, T, H, W, GLA_DTYPE_BF16);
+  if (!op) return 0;
+  const size_t th = (size_t)batch * T * H * W * heads;
+  return 5 * align_up(th * head_dim * 2, kAlign) + align_up(th * 2, kAlign) + op;
+}
+
+gla_status gla_layer_forward(const void* x, const void* W_in, const void* W_o, int batch, int C,
+                             int C_out, int heads, int head_dim, int T, int H, int W,
+                             float rope_theta, float eps, void* y, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W) || C <= 0 || C_out <= 0) return GLA_ERR_INVALID_ARG;
+  if (C % 8 || C_out % 8 || (heads * head_dim) % 32) return GLA_ERR_UNSUPPORTED;
+  if (!x || !W_in || !W_o || !y || !aligned16(x) || !aligned16(W_in) || !aligned16(W_o) ||
+      !aligned16(y))
+    return GLA_ERR_INVALID_ARG;
+  const size_t need = gla_layer_workspace_size(batch, heads, head_dim, T, H, W);
+  if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < need)
+    return GLA_ERR_WORKSPACE;
+  const int tokens = batch * T * H * W;
+  const size_t th = (size_t)tokens * heads;
+  const size_t big = align_up(th * head_dim * 2, kAlign);
+  unsigned char* w = static_cast<unsigned char*>(workspace);
+  unsigned char *q = w, *k = q + big, *v = k + big, *g = v + big, *o = g + big, *beta = o + big;
+  unsigned char* ows = beta + align_up(th * 2, kAlign);
+  gla_status st = gla_project_in(x, W_in, tokens, C, heads, head_dim, q, k, v, g, beta, stream);
+  if (st != GLA_OK) return st;
+  st = gla_forward(q, k, v, beta, g, batch, heads, head_dim, T, H, W, rope_theta, eps,
+                   GLA_DTYPE_BF16, o, ows, workspace_bytes - (size_t)(ows - w), stream);
+  if (st != GLA_OK) return st;
+  return gla_gemm_bf16(o, W_o, y, tokens, C_out, heads * head_dim, stream);
 }
 
 size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, int T, int H, int W,

@@ -52,6 +52,10 @@ _SIGS = {
     "gla_forward_mx": (_i, [_vp] * 9 + [_i] * 6 + [_f, _f, _vp, _vp, _sz, _vp]),
     "gla_forward_mx_ex": (_i, [_vp] * 9 + [_i] * 6 + [_f, _f, _vp, _vp, _sz, _vp, _i]
                           + [_vp] * 4 + [ctypes.POINTER(_vp)]),
+    "gla_gemm_bf16": (_i, [_vp] * 3 + [_i] * 3 + [_vp]),
+    "gla_project_in": (_i, [_vp] * 2 + [_i] * 4 + [_vp] * 6),
+    "gla_layer_workspace_size": (_sz, [_i] * 6),
+    "gla_layer_forward": (_i, [_vp] * 3 + [_i] * 8 + [_f, _f, _vp, _vp, _sz, _vp]),
     "gla_forward_noalloc": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp]),
     "gla_get_device_status": (_i, [_vp]),
     "gla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
@@ -419,6 +423,80 @@ def gla_causal_forward(q, k, v, beta, g, T, H, W, rope_theta=10000.0, eps=1e-6, 
     z = torch.zeros(B, Hh, d, dtype=torch.float32, device=q.device)
     return gla_causal_step(state, z, q, k, v, beta, g, T, H, W, 0, rope_theta, eps, out=out,
                            workspace=workspace, stream=stream, path=path)
+
+
+def _bf16_matrix(t, name, dev=None):
+    if t.dim() != 2 or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a contiguous 2-D bf16 GPU tensor")
+    if dev is not None and t.device != dev:
+        raise ValueError(f"{name} is on {t.device}, expected {dev}")
+
+
+def gla_gemm_bf16(A, B, out=None, stream=None):
+    """A [M, K] @ B[N, K]^T on the tensor cores (bf16 in and out, fp32 sums)."""
+    _bf16_matrix(A, "A")
+    _bf16_matrix(B, "B", A.device)
+    M, K = A.shape
+    N, K2 = B.shape
+    if K2 != K:
+        raise ValueError(f"A is {tuple(A.shape)}, B is {tuple(B.shape)}: K differs")
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device)
+    _bf16_matrix(out, "out", A.device)
+    if tuple(out.shape) != (M, N):
+        raise ValueError(f"out must be [{M}, {N}]")
+    with _on(A.device):
+        st = lib().gla_gemm_bf16(_ptr(A), _ptr(B), _ptr(out), M, N, K, _stream(stream, A.device))
+    _check(st, "gla_gemm_bf16")
+    return out
+
+
+def gla_project_in(x, W_in, batch, N, heads, head_dim, stream=None):
+    """x [batch*N, C] times W_in^T, split into the operator's inputs: returns
+    dict(q, k, v, g [batch, N, heads, head_dim], beta [batch, N, heads])."""
+    _bf16_matrix(x, "x")
+    _bf16_matrix(W_in, "W_in", x.device)
+    tokens, C = x.shape
+    if tokens != batch * N or tuple(W_in.shape) != (4 * heads * head_dim + heads, C):
+        raise ValueError("x must be [batch*N, C] and W_in [4*heads*head_dim + heads, C]")
+    dev = x.device
+    out = {n: torch.empty(batch, N, heads, head_dim, dtype=torch.bfloat16, device=dev)
+           for n in "qkvg"}
+    out["beta"] = torch.empty(batch, N, heads, dtype=torch.bfloat16, device=dev)
+    with _on(dev):
+        st = lib().gla_project_in(_ptr(x), _ptr(W_in), tokens, C, heads, head_dim, _ptr(out["q"]),
+                                  _ptr(out["k"]), _ptr(out["v"]), _ptr(out["g"]), _ptr(out["beta"]),
+                                  _stream(stream, dev))
+    _check(st, "gla_project_in")
+    return out
+
+
+def gla_layer_forward(x, W_in, W_o, batch, heads, head_dim, T, H, W, rope_theta=10000.0,
+                      eps=1e-6, out=None, workspace=None, stream=None):
+    """y [batch*N, C_out] = W_o applied to the operator of the projections of
+    x [batch*N, C]."""
+    _bf16_matrix(x, "x")
+    _bf16_matrix(W_in, "W_in", x.device)
+    _bf16_matrix(W_o, "W_o", x.device)
+    tokens, C = x.shape
+    C_out, HD = W_o.shape
+    if tokens != batch * T * H * W or HD != heads * head_dim or \
+            tuple(W_in.shape) != (4 * heads * head_dim + heads, C):
+        raise ValueError("shapes do not match the layer")
+    dev = x.device
+    if out is None:
+        out = torch.empty(tokens, C_out, dtype=torch.bfloat16, device=dev)
+    _bf16_matrix(out, "out", dev)
+    if workspace is None:
+        workspace = alloc_workspace(lib().gla_layer_workspace_size(batch, heads, head_dim, T, H, W),
+                                    dev)
+    _check_workspace(workspace, dev)
+    with _on(dev):
+        st = lib().gla_layer_forward(_ptr(x), _ptr(W_in), _ptr(W_o), batch, C, C_out, heads,
+                                     head_dim, T, H, W, rope_theta, eps, _ptr(out),
+                                     _ptr(workspace), workspace.numel(), _stream(stream, dev))
+    _check(st, "gla_layer_forward")
+    return out
 
 
 MX_NAMES = ("q", "q_scale", "k", "k_scale", "v", "v_scale", "beta", "g", "g_scale")

@@ -275,6 +275,43 @@ GLA_API gla_status gla_forward_mx_ex(const void* q, const void* q_scale, const v
                                      float* S_out, float* z_out, float* den_out, float* x_out,
                                      void* const* events);
 
+/* ------------------------------------------------------------------------
+ * The layer around the operator.  The "Gated Bilinear Linear Attention"
+ * prerequisite of the SANA-Video 2.0 summary reads o_j = W_o RMSNorm[...]: the
+ * heads' normalised read-outs, concatenated over the heads (width
+ * heads*head_dim), times W_o.  The pages print no input projection; here q, k,
+ * v, g and the beta logits are one linear map of the layer input x, and beta is
+ * the sigmoid of its logits.  All matrices are bf16, row-major, device memory,
+ * 16-byte aligned; products accumulate in fp32 on the tensor cores (tcgen05). */
+
+/* C [M][N] = A [M][K] B[N][K]^T, bf16 out (rounded to nearest even).  K and N
+ * multiples of 8 (16-byte rows). */
+GLA_API gla_status gla_gemm_bf16(const void* A, const void* B, void* C, int M, int N, int K,
+                                 void* stream);
+
+/* The input projection with the operator's inputs written straight from the
+ * product: x [tokens][C] times W_in [4*heads*head_dim + heads][C]^T, columns
+ * [0, HD) to q, [HD, 2HD) to k, then v and g ([tokens][HD] each, HD =
+ * heads*head_dim, i.e. the operator's [B][N][heads][head_dim] layout), and
+ * the last `heads` columns to beta [tokens][heads] after a sigmoid.  C a
+ * multiple of 8, HD a multiple of 32. */
+GLA_API gla_status gla_project_in(const void* x, const void* W_in, int tokens, int C, int heads,
+                                  int head_dim, void* q, void* k, void* v, void* g, void* beta,
+                                  void* stream);
+
+/* Workspace bytes of gla_layer_forward (q, k, v, g, beta, the operator's output
+ * and the operator's workspace). */
+GLA_API size_t gla_layer_workspace_size(int batch, int heads, int head_dim, int T, int H, int W);
+
+/* y [batch*N][C_out] = W_o applied to gla_forward of the projections of x
+ * [batch*N][C]: gla_project_in, gla_forward, gla_gemm_bf16, each kernel a
+ * programmatic dependent of the one before.  W_in [4*heads*head_dim +
+ * heads][C], W_o [C_out][heads*head_dim]. */
+GLA_API gla_status gla_layer_forward(const void* x, const void* W_in, const void* W_o, int batch,
+                                     int C, int C_out, int heads, int head_dim, int T, int H,
+                                     int W, float rope_theta, float eps, void* y,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of the device arena gla_causal_step_host needs: room for the call's
  * five inputs, its output and its workspace. */
 GLA_API size_t gla_causal_host_arena_size(int batch, int heads, int head_dim, int T, int H,
