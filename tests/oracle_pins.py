@@ -392,6 +392,64 @@ def check_causal_carried_state():
     _close(second["out"], whole["out"][:, L:], 1e-12, "carried causal state")
 
 
+# ---------------------------------------------------- gated softmax anchor
+
+def check_anchor_one_token():
+    """N = 1: the softmax of one score is 1, so out = sigmoid(g) * v exactly."""
+    rng = np.random.default_rng(8)
+    q, k, v, g = (rng.standard_normal((1, 1, 2, 8)) for _ in range(4))
+    r = O.softmax_anchor(q, k, v, g, 1, 1, 1, 1e4)
+    _close(r["out"], (1 / (1 + np.exp(-g))) * v, 1e-15, "anchor, one token")
+
+
+def check_anchor_two_token_closed_form():
+    """T = 2, H = W = 1, d = 2, RoPE off: q0 = (1, 0) -> q_hat0 = (1, 0) /
+    sqrt(0.5 + e_n) ~ (sqrt2, 0); k0 = (1, 0), k1 = (0, 1) likewise; scores of
+    token 0: (c^2 / sqrt2, 0) with c = 1/sqrt(0.5 + e_n); weights
+    (e^a, 1) / (e^a + 1); out = sigma(g) * weighted v."""
+    e_n = 1e-6
+    c = 1 / math.sqrt(0.5 + e_n)
+    q = np.array([[1.0, 0.0], [0.0, 1.0]]).reshape(1, 2, 1, 2)
+    k = np.array([[1.0, 0.0], [0.0, 1.0]]).reshape(1, 2, 1, 2)
+    v = np.array([[1.0, 2.0], [3.0, -1.0]]).reshape(1, 2, 1, 2)
+    g = np.zeros((1, 2, 1, 2))
+    a = c * c / math.sqrt(2)
+    w0 = np.array([math.exp(a), 1.0]) / (math.exp(a) + 1.0)
+    want0 = 0.5 * (w0[0] * np.array([1.0, 2.0]) + w0[1] * np.array([3.0, -1.0]))
+    r = O.softmax_anchor(q, k, v, g, 2, 1, 1, 0.0)
+    _close(r["out"][0, 0, 0], want0, 1e-14, "anchor token 0")
+    want1 = 0.5 * (w0[1] * np.array([1.0, 2.0]) + w0[0] * np.array([3.0, -1.0]))
+    _close(r["out"][0, 1, 0], want1, 1e-14, "anchor token 1")
+
+
+def check_anchor_matches_library_sdpa():
+    """On the normalised, rotated q and k (the oracle's own feature maps are
+    pinned above), the attention equals torch's scaled_dot_product_attention
+    in fp64."""
+    import torch
+    rng = np.random.default_rng(9)
+    T, H, W, d, Hh = 2, 3, 2, 16, 2
+    N = T * H * W
+    q, k, v, g = (rng.standard_normal((1, N, Hh, d)) for _ in range(4))
+    r = O.softmax_anchor(q, k, v, g, T, H, W, 1e4)
+    ang = O.rope_angles(d, T, H, W, 1e4)
+    qt = O.rope_rotate(O.rms_normalize(q), ang)
+    kt = O.rope_rotate(O.rms_normalize(k), ang)
+    to = lambda a: torch.from_numpy(np.ascontiguousarray(a.transpose(0, 2, 1, 3)))
+    lib = torch.nn.functional.scaled_dot_product_attention(to(qt), to(kt), to(v))
+    _close(r["attn"], lib.numpy().transpose(0, 2, 1, 3), 1e-12, "anchor vs torch SDPA")
+
+
+def check_anchor_uniform_scores():
+    """q = 0 gives q_hat = 0 and all scores 0: every token reads the mean of v."""
+    rng = np.random.default_rng(10)
+    k, v, g = (rng.standard_normal((1, 6, 1, 4)) for _ in range(3))
+    q = np.zeros((1, 6, 1, 4))
+    r = O.softmax_anchor(q, k, v, g, 1, 2, 3, 1e4)
+    _close(r["attn"][0, :, 0], np.repeat(v[0, :, 0].mean(axis=0, keepdims=True), 6, axis=0),
+           1e-14, "uniform attention")
+
+
 # ------------------------------------------------ the layer's projections
 
 def check_project_in_layout():

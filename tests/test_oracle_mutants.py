@@ -148,6 +148,16 @@ def _project_out_transposed(o, W_o):
     return np.swapaxes(o, 2, 3).reshape(B, N, Hh * d) @ W_o.T
 
 
+def _anchor_gate_inside(q, k, v, g, T, H, W, rope_theta, t0=0):
+    r = _orig["softmax_anchor"](q, k, v * (1 / (1 + np.exp(-g))), np.full_like(g, 40.0), T, H, W,
+                                rope_theta, t0)
+    return r
+
+
+def _anchor_softmax_over_queries(q, k, v, g, T, H, W, rope_theta, t0=0):
+    return _orig["softmax_anchor"](k, q, v, g, T, H, W, rope_theta, t0)
+
+
 def _e4m3_bias8(codes):
     return _orig["e4m3_decode"](codes) / 2.0
 
@@ -194,6 +204,8 @@ MUTANTS = {
     "project_in_no_sigmoid": ("project_in", _project_in_no_sigmoid),
     "project_in_qk_swapped": ("project_in", _project_in_qk_swapped),
     "project_out_channel_major": ("project_out", _project_out_transposed),
+    "anchor_gate_on_values": ("softmax_anchor", _anchor_gate_inside),
+    "anchor_q_k_swapped": ("softmax_anchor", _anchor_softmax_over_queries),
     "e4m3_bias8": ("e4m3_decode", _e4m3_bias8),
     "e4m3_no_subnormals": ("e4m3_decode", _e4m3_no_subnormals),
     "e8m0_bias128": ("e8m0_decode", _e8m0_bias128),
