@@ -45,11 +45,12 @@ def parse():
     ap.add_argument("--workload", default="720p", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--variant", default="bidirectional",
-                    choices=["bidirectional", "causal", "mx", "layer"],
+                    choices=["bidirectional", "causal", "mx", "layer", "anchor"],
                     help="causal: the token-level causal read-out (gla_causal_step) of the "
                          "workload, one step = one call from a zero state; mx: gla_forward on "
                          "FP8 (OCP MX) inputs; layer: input projection, gla_forward and W_o "
-                         "(gla_layer_forward) at the workload's width")
+                         "(gla_layer_forward) at the workload's width; anchor: the gated softmax "
+                         "anchor layer (gla_softmax_anchor) on the workload's q, k, v, g")
     ap.add_argument("--cpu-sample-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
@@ -333,6 +334,9 @@ def main():
         return
     if args.variant == "layer":
         run_layer(args, wl, gla, dev, dist, world, rank, local)
+        return
+    if args.variant == "anchor":
+        run_anchor(args, wl, gla, dev, dist, world, rank, local)
         return
 
     inp = workloads.make_inputs(wl, seed=replicas.replica_seed(wl.seed, rank))
@@ -864,6 +868,139 @@ def run_layer(args, wl, gla, dev, dist, world, rank, local):
             "gpu_launches": 5 * steps,
             "clocks": mon.summary(),
             "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def anchor_cpu_rate(wl, seconds, rows=256):
+    """The oracle's softmax_anchor, as it stands, on `rows` query rows of one
+    head at a time (all N keys) until `seconds` have passed: returns (tokens/s
+    of the full layer, query rows done, s, BLAS threads)."""
+    import oracle.gla_oracle as O
+    from threadpoolctl import threadpool_info
+    t_used, done, idx = 0.0, 0, 0
+    while t_used < seconds:
+        x = workloads.as_f64(workloads.draw(1, wl.tokens, 1, wl.head_dim, wl.dtype, 2000 + idx))
+        sel = np.linspace(0, wl.tokens - 1, rows).astype(np.int64)
+        t0 = time.perf_counter()
+        O.softmax_anchor(x["q"], x["k"], x["v"], x["g"], wl.T, wl.H, wl.W, wl.rope_theta,
+                         queries=sel)
+        t_used += time.perf_counter() - t0
+        done += rows
+        idx += 1
+    blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+    return done / t_used / wl.heads, done, t_used, (blas[0] if blas else 1)
+
+
+def run_anchor(args, wl, gla, dev, dist, world, rank, local):
+    """One step = gla_softmax_anchor on the workload's q, k, v, g (bf16, the
+    operator's draw): q/k RMSNorm + 3D RoPE, then bidirectional softmax
+    attention over all N tokens with the sigmoid output gate."""
+    x = workloads.draw(wl.batch, wl.tokens, wl.heads, wl.head_dim, wl.dtype,
+                       replicas.replica_seed(wl.seed, rank))
+    d = {n: x[n].to(dev) for n in "qkvg"}
+    out = torch.empty_like(d["q"])
+    ws = gla.alloc_workspace(gla.gla_softmax_anchor_workspace_size(
+        wl.batch, wl.heads, wl.head_dim, wl.T, wl.H, wl.W), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        gla.gla_softmax_anchor(d["q"], d["k"], d["v"], d["g"], wl.T, wl.H, wl.W, wl.rope_theta,
+                               out=out, workspace=ws, stream=stream, events=events)
+
+    if args.profile:
+        for _ in range(args.warmup + args.steps):
+            step()
+        torch.cuda.synchronize(dev)
+        status = gla.gla_get_device_status(stream)
+        print(json.dumps({"profile_run": wl.name, "variant": "anchor",
+                          "steps": args.warmup + args.steps, "status": gla.status_string(status)}))
+        if status != gla.GLA_OK:
+            sys.exit(1)
+        return
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert gla.gla_get_device_status(stream) == gla.GLA_OK
+
+    def sync():
+        torch.cuda.synchronize(dev)
+
+    steps = max(5, args.steps // 100)
+
+    def timed_steps():
+        for _ in range(steps):
+            step()
+
+    with ClockMonitor(local) as mon:
+        elapsed_ms, reps = timed_repeats(timed_steps, stream, dist, sync, dev, args.repeats)
+        # The attention kernel alone: events before and after it, per call.
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        t_prep, t_attn = [], []
+        for _ in range(steps):
+            step(ev)
+            torch.cuda.synchronize(dev)
+            t_prep.append(ev[0].elapsed_time(ev[1]))
+            t_attn.append(ev[1].elapsed_time(ev[2]))
+    if gla.gla_get_device_status(stream) != gla.GLA_OK:
+        raise RuntimeError("device status after the timed region")
+    k_prep, k_attn = float(np.median(t_prep)), float(np.median(t_attn))
+
+    # End to end: pinned host q, k, v, g in, the output back to pinned host memory.
+    host = {n: x[n].pin_memory() for n in "qkvg"}
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_steps():
+        for _ in range(steps):
+            for n in "qkvg":
+                d[n].copy_(host[n], non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+
+    e2e_ms, _ = timed_repeats(e2e_steps, stream, dist, sync, dev, 1)
+
+    tokens = wl.batch * wl.tokens
+    flops = 4.0 * wl.batch * wl.heads * float(wl.tokens) ** 2 * wl.head_dim
+    peak, peak_kind = measured_tflops(sustained=True)
+    tf = flops / (k_attn * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, rows, t_used, cores = anchor_cpu_rate(wl, args.cpu_sample_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": (f"oracle.softmax_anchor on {rows} query rows (256 per call, all "
+                          f"{wl.tokens} keys, one head per call) in {t_used:.1f} s; tokens/s of "
+                          f"the full layer = query-head rows/s / {wl.heads}"),
+               "host": host_info()}
+    if rank == 0:
+        line = {
+            "metric": (f"gla_softmax_anchor tokens/s ({wl.heads}x{wl.head_dim} heads, "
+                       f"{wl.tokens} tok, bidirectional softmax) and TFLOP/s vs B200 peak"),
+            "value": replicas.aggregate_rate(world, tokens, steps, elapsed_ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / steps,
+            "repeats": len(reps), "repeat_ms_per_step": [round(r / steps, 5) for r in reps],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(workload_config(wl), variant="gated softmax anchor",
+                           l2="no flush: K/V of a head are re-read from L2 by design",
+                           parallelism=f"replicas x{world}"),
+            "roofline": {"bound": "tensor", "kernel": "anchor_attn_kernel",
+                         "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "peak_kind": peak_kind + " sustained bf16",
+                         "traffic": traffic_for("anchor_attn_kernel", wl.name),
+                         "alg_flops_per_launch": flops, "ms_per_launch": k_attn},
+            "stages_ms": {"anchor_prep_kernel": k_prep, "anchor_attn_kernel": k_attn,
+                          "how": "events around each kernel, per call, median"},
+            "e2e": {"value": replicas.aggregate_rate(world, tokens, steps, e2e_ms),
+                    "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 2 * steps,
+            "clocks": mon.summary(),
+            "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     if dist:

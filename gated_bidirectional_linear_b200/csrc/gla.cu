@@ -18,6 +18,7 @@
 #include "causal.cuh"
 #include "mx.cuh"
 #include "gemm.cuh"
+#include "anchor.cuh"
 
 using namespace gla;
 
@@ -778,6 +779,42 @@ gla_status gla_layer_forward(const void* x, const void* W_in, const void* W_o, i
                    GLA_DTYPE_BF16, o, ows, workspace_bytes - (size_t)(ows - w), stream);
   if (st != GLA_OK) return st;
   return gla_gemm_bf16(o, W_o, y, tokens, C_out, heads * head_dim, stream);
+}
+
+// Anchor workspace: q_til and k_til, fp16, the inputs' layout.
+size_t gla_softmax_anchor_workspace_size(int batch, int heads, int head_dim, int T, int H,
+                                         int W) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W) || head_dim != 128) return 0;
+  const size_t th = (size_t)batch * T * H * W * heads;
+  return 2 * align_up(th * head_dim * 2, kAlign);
+}
+
+gla_status gla_softmax_anchor_timed(const void* q, const void* k, const void* v, const void* g,
+                                    int batch, int heads, int head_dim, int T, int H, int W,
+                                    float rope_theta, void* out, void* workspace,
+                                    size_t workspace_bytes, void* stream, void* const* events) {
+  if (!dims_ok(batch, heads, head_dim, T, H, W)) return GLA_ERR_INVALID_ARG;
+  if (head_dim != 128 || (long long)batch * heads > 65535) return GLA_ERR_UNSUPPORTED;
+  if (!isfinite(rope_theta)) return GLA_ERR_INVALID_ARG;
+  const void* ptrs[5] = {q, k, v, g, out};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return GLA_ERR_INVALID_ARG;
+  const size_t need = gla_softmax_anchor_workspace_size(batch, heads, head_dim, T, H, W);
+  if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < need)
+    return GLA_ERR_WORKSPACE;
+  if (device_sm_count() <= 0) return GLA_ERR_CUDA;
+  const Geom geom = make_geom(batch, heads, head_dim, T, H, W, 0, rope_theta, 1e-6f);
+  __half* qt = static_cast<__half*>(workspace);
+  __half* kt = reinterpret_cast<__half*>(static_cast<unsigned char*>(workspace) + need / 2);
+  return run_anchor(geom, q, k, v, g, out, qt, kt, static_cast<cudaStream_t>(stream), events);
+}
+
+gla_status gla_softmax_anchor(const void* q, const void* k, const void* v, const void* g,
+                              int batch, int heads, int head_dim, int T, int H, int W,
+                              float rope_theta, void* out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return gla_softmax_anchor_timed(q, k, v, g, batch, heads, head_dim, T, H, W, rope_theta, out,
+                                  workspace, workspace_bytes, stream, nullptr);
 }
 
 size_t gla_forward_host_arena_size(int batch, int heads, int head_dim, int T, int H, int W,

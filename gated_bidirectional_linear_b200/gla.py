@@ -56,6 +56,10 @@ _SIGS = {
     "gla_project_in": (_i, [_vp] * 2 + [_i] * 4 + [_vp] * 6),
     "gla_layer_workspace_size": (_sz, [_i] * 6),
     "gla_layer_forward": (_i, [_vp] * 3 + [_i] * 8 + [_f, _f, _vp, _vp, _sz, _vp]),
+    "gla_softmax_anchor_workspace_size": (_sz, [_i] * 6),
+    "gla_softmax_anchor": (_i, [_vp] * 4 + [_i] * 6 + [_f, _vp, _vp, _sz, _vp]),
+    "gla_softmax_anchor_timed": (_i, [_vp] * 4 + [_i] * 6 + [_f, _vp, _vp, _sz, _vp,
+                                                          ctypes.POINTER(_vp)]),
     "gla_forward_noalloc": (_i, [_vp] * 5 + [_i] * 6 + [_f, _f, _i, _vp, _vp]),
     "gla_get_device_status": (_i, [_vp]),
     "gla_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
@@ -496,6 +500,45 @@ def gla_layer_forward(x, W_in, W_o, batch, heads, head_dim, T, H, W, rope_theta=
                                      head_dim, T, H, W, rope_theta, eps, _ptr(out),
                                      _ptr(workspace), workspace.numel(), _stream(stream, dev))
     _check(st, "gla_layer_forward")
+    return out
+
+
+def gla_softmax_anchor_workspace_size(batch, heads, head_dim, T, H, W):
+    return lib().gla_softmax_anchor_workspace_size(batch, heads, head_dim, T, H, W)
+
+
+def gla_softmax_anchor(q, k, v, g, T, H, W, rope_theta=10000.0, out=None, workspace=None,
+                       stream=None, events=None):
+    """The gated softmax anchor: o_j = sigmoid(g_j) * softmax(q_til_j . K_til^T
+    / sqrt(d)) V over all T*H*W tokens, q_til / k_til the RMS-normalised and
+    3D-rotated q / k.  q, k, v, g: bf16 [B, N, Hh, 128] on one GPU.  events:
+    three torch.cuda.Event objects recorded before the q/k preparation, after
+    it and after the attention kernel."""
+    B, Hh, d = _dims(q, T, H, W)
+    if out is None:
+        out = torch.empty_like(q)
+    shape = tuple(q.shape)
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("out", out)):
+        if tuple(t.shape) != shape or t.dtype != torch.bfloat16 or t.device != q.device \
+                or t.device.type != "cuda" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 GPU tensor of shape {shape} "
+                             f"on {q.device}")
+    if workspace is None:
+        workspace = alloc_workspace(gla_softmax_anchor_workspace_size(B, Hh, d, T, H, W),
+                                    q.device)
+    _check_workspace(workspace, q.device)
+    ev = None
+    if events is not None:
+        for e in events:        # torch creates an event's handle at its first record
+            if e is not None and e.cuda_event == 0:
+                e.record(torch.cuda.current_stream(q.device) if stream is None else stream)
+        ev = (ctypes.c_void_p * 3)(*[ctypes.c_void_p(e.cuda_event) if e is not None else None
+                                     for e in events])
+    with _on(q.device):
+        st = lib().gla_softmax_anchor_timed(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, Hh, d, T, H, W,
+                                            rope_theta, _ptr(out), _ptr(workspace),
+                                            workspace.numel(), _stream(stream, q.device), ev)
+    _check(st, "gla_softmax_anchor")
     return out
 
 

@@ -312,6 +312,43 @@ GLA_API gla_status gla_layer_forward(const void* x, const void* W_in, const void
                                      int W, float rope_theta, float eps, void* y,
                                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The gated softmax anchor.  The "softmax anchors and hybrid attention"
+ * section of the SANA-Video 2.0 summary keeps one full softmax attention
+ * layer in four; its anchor layers normalise q and k, rotate them with the
+ * same 3D RoPE and gate the read-out with sigmoid(g).  Per head:
+ *   q_til = RoPE3D(RMSNorm(q)), k_til = RoPE3D(RMSNorm(k))   (no ReLU here)
+ *   o_j   = sigmoid(g_j) * sum_n softmax_n(q_til_j . k_til_n / sqrt(d)) v_n
+ * over all N tokens of the call (bidirectional).  RMSNorm has no weight and
+ * epsilon 1e-6; q, k, v, g and out are bf16 [batch][N][heads][head_dim]
+ * device buffers (16-byte aligned), N = T*H*W in raster order; head_dim 128
+ * (GLA_ERR_UNSUPPORTED otherwise); rope_theta <= 0 turns the rotation off.
+ * Scores are taken on the tensor cores from fp16 q_til, k_til (fp32
+ * accumulate), the softmax weights are rounded to bf16 for P*V, and the
+ * row sums stay in fp32.  Errors: GLA_ERR_INVALID_ARG for bad sizes or
+ * pointers, GLA_ERR_WORKSPACE for a short or misaligned workspace (256-byte
+ * aligned), GLA_ERR_CUDA for a failed launch. */
+
+/* Workspace bytes of gla_softmax_anchor (fp16 q_til and k_til), 0 for
+ * unsupported sizes. */
+GLA_API size_t gla_softmax_anchor_workspace_size(int batch, int heads, int head_dim, int T, int H,
+                                                 int W);
+
+GLA_API gla_status gla_softmax_anchor(const void* q, const void* k, const void* v, const void* g,
+                                      int batch, int heads, int head_dim, int T, int H, int W,
+                                      float rope_theta, void* out, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/* gla_softmax_anchor that also records caller-created CUDA events (cudaEvent_t
+ * passed as void*) on `stream`: events[0] before the q/k preparation,
+ * events[1] after it, events[2] after the attention kernel.  `events` and any
+ * of its entries may be NULL. */
+GLA_API gla_status gla_softmax_anchor_timed(const void* q, const void* k, const void* v,
+                                            const void* g, int batch, int heads, int head_dim,
+                                            int T, int H, int W, float rope_theta, void* out,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream, void* const* events);
+
 /* Bytes of the device arena gla_causal_step_host needs: room for the call's
  * five inputs, its output and its workspace. */
 GLA_API size_t gla_causal_host_arena_size(int batch, int heads, int head_dim, int T, int H,

@@ -386,7 +386,7 @@ def forward_mx(q, k, v, beta, g, T, H, W, rope_theta, eps, t0=0):
 
 # ------------------------------------------------------ gated softmax anchor
 
-def softmax_anchor(q, k, v, g, T, H, W, rope_theta, t0=0):
+def softmax_anchor(q, k, v, g, T, H, W, rope_theta, t0=0, queries=None):
     """The gated softmax anchor of the hybrid stack ([GBLA]'s page, "softmax
     anchors and hybrid attention"; method: a gated softmax layer every fourth
     depth): bidirectional scaled dot-product attention with QK normalisation,
@@ -395,22 +395,25 @@ def softmax_anchor(q, k, v, g, T, H, W, rope_theta, t0=0):
     and k (no ReLU on this path), scores q_til . k_til / sqrt(d) over every
     token, and o_j = sigmoid(g_j) * sum_n softmax_n(scores_j) v_n, with no
     output norm (W_o is outside).  q, k, v, g [B, N, Hh, d]; returns dict(out,
-    attn) with attn the read-out before the gate."""
+    attn) with attn the read-out before the gate.  queries: indices of the
+    query tokens whose rows are returned ([B, len(queries), Hh, d]); default
+    all tokens."""
     d = q.shape[-1]
     angles = _angles_or_none(d, T, H, W, rope_theta, t0)
     qh, kh = rms_normalize(q), rms_normalize(k)
     qt = qh if angles is None else rope_rotate(qh, angles)
     kt = kh if angles is None else rope_rotate(kh, angles)
     B, N, Hh, _ = q.shape
-    attn = np.empty_like(q)
+    rows = np.arange(N) if queries is None else np.asarray(queries)
+    attn = np.empty((B, len(rows), Hh, d), dtype=np.float64)
     for b in range(B):
         for h in range(Hh):
-            s = qt[b, :, h, :] @ kt[b, :, h, :].T / np.sqrt(d)
+            s = qt[b, rows, h, :] @ kt[b, :, h, :].T / np.sqrt(d)
             s = s - s.max(axis=1, keepdims=True)
             w = np.exp(s)
             w /= w.sum(axis=1, keepdims=True)
             attn[b, :, h, :] = w @ v[b, :, h, :]
-    return dict(attn=attn, out=sigmoid(g) * attn)
+    return dict(attn=attn, out=sigmoid(g[:, rows]) * attn)
 
 
 # ----------------------------------------------- the layer's projections

@@ -450,6 +450,31 @@ def check_anchor_uniform_scores():
            1e-14, "uniform attention")
 
 
+def check_anchor_query_rows():
+    """Selected query rows (queries=...) equal a per-row brute force: for each
+    chosen token j, scores over all n by explicit dot products, max-shifted
+    exponentials, normalised weights, weighted sum of v, times sigmoid(g_j)."""
+    rng = np.random.default_rng(11)
+    T, H, W, d, Hh = 2, 2, 3, 8, 2
+    N = T * H * W
+    q, k, v, g = (rng.standard_normal((1, N, Hh, d)) for _ in range(4))
+    rows = [0, 5, 11, 7]
+    r = O.softmax_anchor(q, k, v, g, T, H, W, 1e4, queries=rows)
+    ang = O.rope_angles(d, T, H, W, 1e4)
+    qt = O.rope_rotate(O.rms_normalize(q), ang)
+    kt = O.rope_rotate(O.rms_normalize(k), ang)
+    for i, j in enumerate(rows):
+        for h in range(Hh):
+            sc = [sum(qt[0, j, h, c] * kt[0, n, h, c] for c in range(d)) / math.sqrt(d)
+                  for n in range(N)]
+            m = max(sc)
+            w = [math.exp(x - m) for x in sc]
+            tot = sum(w)
+            attn = [sum(w[n] * v[0, n, h, c] for n in range(N)) / tot for c in range(d)]
+            gate = 1 / (1 + np.exp(-g[0, j, h]))
+            _close(r["out"][0, i, h], gate * np.array(attn), 1e-13, f"anchor row {j} head {h}")
+
+
 # ------------------------------------------------ the layer's projections
 
 def check_project_in_layout():

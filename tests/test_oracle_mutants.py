@@ -148,14 +148,14 @@ def _project_out_transposed(o, W_o):
     return np.swapaxes(o, 2, 3).reshape(B, N, Hh * d) @ W_o.T
 
 
-def _anchor_gate_inside(q, k, v, g, T, H, W, rope_theta, t0=0):
+def _anchor_gate_inside(q, k, v, g, T, H, W, rope_theta, t0=0, queries=None):
     r = _orig["softmax_anchor"](q, k, v * (1 / (1 + np.exp(-g))), np.full_like(g, 40.0), T, H, W,
-                                rope_theta, t0)
+                                rope_theta, t0, queries)
     return r
 
 
-def _anchor_softmax_over_queries(q, k, v, g, T, H, W, rope_theta, t0=0):
-    return _orig["softmax_anchor"](k, q, v, g, T, H, W, rope_theta, t0)
+def _anchor_softmax_over_queries(q, k, v, g, T, H, W, rope_theta, t0=0, queries=None):
+    return _orig["softmax_anchor"](k, q, v, g, T, H, W, rope_theta, t0, queries)
 
 
 def _e4m3_bias8(codes):
