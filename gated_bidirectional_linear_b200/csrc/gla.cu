@@ -802,11 +802,13 @@ gla_status gla_softmax_anchor_timed(const void* q, const void* k, const void* v,
   const size_t need = gla_softmax_anchor_workspace_size(batch, heads, head_dim, T, H, W);
   if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < need)
     return GLA_ERR_WORKSPACE;
-  if (device_sm_count() <= 0) return GLA_ERR_CUDA;
+  const int sms = device_sm_count();
+  if (sms <= 0) return GLA_ERR_CUDA;
   const Geom geom = make_geom(batch, heads, head_dim, T, H, W, 0, rope_theta, 1e-6f);
   __half* qt = static_cast<__half*>(workspace);
   __half* kt = reinterpret_cast<__half*>(static_cast<unsigned char*>(workspace) + need / 2);
-  return run_anchor(geom, q, k, v, g, out, qt, kt, static_cast<cudaStream_t>(stream), events);
+  return run_anchor(geom, q, k, v, g, out, qt, kt, sms, static_cast<cudaStream_t>(stream),
+                    events);
 }
 
 gla_status gla_softmax_anchor(const void* q, const void* k, const void* v, const void* g,

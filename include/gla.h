@@ -325,7 +325,7 @@ GLA_API gla_status gla_layer_forward(const void* x, const void* W_in, const void
  * (GLA_ERR_UNSUPPORTED otherwise); rope_theta <= 0 turns the rotation off.
  * Scores are taken on the tensor cores from fp16 q_til, k_til (fp32
  * accumulate), the softmax weights are rounded to bf16 for P*V, and the
- * row sums stay in fp32.  Errors: GLA_ERR_INVALID_ARG for bad sizes or
+ * row sums add those rounded weights in fp32.  Errors: GLA_ERR_INVALID_ARG for bad sizes or
  * pointers, GLA_ERR_WORKSPACE for a short or misaligned workspace (256-byte
  * aligned), GLA_ERR_CUDA for a failed launch. */
 
