@@ -32,6 +32,13 @@ struct AnchorPrepParams {
   __half* kt;
 };
 
+// 8-byte read-only global load.
+__device__ __forceinline__ uint2 ldg_u2(const __nv_bfloat16* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
 // One token-head row: RMSNorm, the rotation (c[i], s[i] of this lane's pairs
 // 2l, 2l+1), the scale; lane l holds channels 4l .. 4l+3.
 __device__ __forceinline__ uint2 an_prep_row(uint2 r, const float (&c)[2], const float (&s)[2],
@@ -77,24 +84,22 @@ __global__ void __launch_bounds__(kAnWarpsPrep * 32) anchor_prep_kernel(AnchorPr
       }
     }
     const size_t base = (size_t)bn * g.Hh * 128 + 4 * lane;
-    int h = 0;
-    for (; h + 2 <= g.Hh; h += 2) {
-      const size_t o0 = base + (size_t)h * 128, o1 = o0 + 128;
-      const uint2 q0 = *reinterpret_cast<const uint2*>(p.q + o0);
-      const uint2 q1 = *reinterpret_cast<const uint2*>(p.q + o1);
-      const uint2 k0 = *reinterpret_cast<const uint2*>(p.k + o0);
-      const uint2 k1 = *reinterpret_cast<const uint2*>(p.k + o1);
-      *reinterpret_cast<uint2*>(p.qt + o0) = an_prep_row(q0, c, sn, kQScale);
-      *reinterpret_cast<uint2*>(p.qt + o1) = an_prep_row(q1, c, sn, kQScale);
-      *reinterpret_cast<uint2*>(p.kt + o0) = an_prep_row(k0, c, sn, 1.f);
-      *reinterpret_cast<uint2*>(p.kt + o1) = an_prep_row(k1, c, sn, 1.f);
-    }
-    if (h < g.Hh) {
-      const size_t o0 = base + (size_t)h * 128;
-      const uint2 q0 = *reinterpret_cast<const uint2*>(p.q + o0);
-      const uint2 k0 = *reinterpret_cast<const uint2*>(p.k + o0);
-      *reinterpret_cast<uint2*>(p.qt + o0) = an_prep_row(q0, c, sn, kQScale);
-      *reinterpret_cast<uint2*>(p.kt + o0) = an_prep_row(k0, c, sn, 1.f);
+    // Four heads per step, all eight loads issued before any use.
+    for (int h0 = 0; h0 < g.Hh; h0 += 4) {
+      uint2 qr[4], kr[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const size_t o = base + (size_t)(h0 + u < g.Hh ? h0 + u : h0) * 128;
+        qr[u] = ldg_u2(p.q + o);
+        kr[u] = ldg_u2(p.k + o);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (h0 + u >= g.Hh) break;
+        const size_t o = base + (size_t)(h0 + u) * 128;
+        *reinterpret_cast<uint2*>(p.qt + o) = an_prep_row(qr[u], c, sn, kQScale);
+        *reinterpret_cast<uint2*>(p.kt + o) = an_prep_row(kr[u], c, sn, 1.f);
+      }
     }
   }
 }
@@ -103,9 +108,10 @@ __global__ void __launch_bounds__(kAnWarpsPrep * 32) anchor_prep_kernel(AnchorPr
 //
 // One CTA takes two 128-query tiles of a head (t = 0, 1) and streams the
 // head's keys and values in 128-token tiles.  Warp 0 issues TMA (q tiles
-// once; k and v through rings of two), warp 1 issues the MMAs, warps 2-5 and
-// 6-9 are the softmax warpgroups of query tiles 0 and 1 (one query row per
-// thread: warp w reads TMEM lane quarter w % 4).
+// once; k through a ring of two slots, v through a ring of three), warp 1
+// issues the MMAs, warps 2-5 and 6-9 are the softmax warpgroups of query
+// tiles 0 and 1 (one query row per thread: warp w reads TMEM lane quarter
+// w % 4).
 //
 // TMEM (512 columns): S_t = q_til_t k_til^T (fp32, 128 columns) at t*128; the
 // softmax weights P_t (bf16 pairs, 64 columns) overwrite the first half of
@@ -118,8 +124,8 @@ __global__ void __launch_bounds__(kAnWarpsPrep * 32) anchor_prep_kernel(AnchorPr
 // Running maximum: a row keeps the maximum it last rescaled to and rescales
 // (O, the row sum) only when a tile's maximum exceeds it by more than 2^8, so
 // that weights stay below 256; the normalisation at the end is the same for
-// any such reference point.  exp2 runs on the MUFU unit for 3 of every 4
-// weight pairs and as a polynomial on the FMA pipes for the 4th.
+// any such reference point.  exp2 runs on the MUFU unit for three of every
+// four weight pairs and as a polynomial on the FMA pipes for the fourth.
 
 constexpr int kAnTile = 128;
 constexpr int kAnQT = 2;                          // query tiles per CTA
@@ -127,16 +133,22 @@ constexpr int kAnSW0 = 2;                         // first softmax warp
 constexpr int kAnThreads = (kAnSW0 + 4 * kAnQT) * 32;
 constexpr uint32_t kAnO = 256;                    // TMEM column of O_0
 constexpr float kAnLazy = 8.f;                    // log2 of the largest weight
+constexpr int kAnVS = 3;                          // v ring slots
+constexpr int kAnPolyPairs = 1;                   // of every 4 weight pairs, by polynomial
+static_assert(kAnQT == 2, "the MMA issue order interleaves exactly two query tiles");
 
 struct AnchorSmem {
   static constexpr uint32_t Q = 0;                        // [2] q_til tiles (fp16)
   static constexpr uint32_t K = Q + kAnQT * kTileBytes;   // [2] k_til tiles (fp16)
-  static constexpr uint32_t V = K + 2 * kTileBytes;       // [2] v tiles (bf16)
-  static constexpr uint32_t BAR = V + 2 * kTileBytes;
-  static constexpr uint32_t NBAR = 1 + 2 * 7 + 1;
+  static constexpr uint32_t V = K + 2 * kTileBytes;       // [3] v tiles (bf16)
+  static constexpr uint32_t BAR = V + kAnVS * kTileBytes;
+  static constexpr uint32_t NBAR = 1 + 2 * 2 + 2 * kAnVS + 3 * kAnQT + 1;
   static constexpr uint32_t MISC = BAR + NBAR * 8;
   static constexpr uint32_t END = MISC + 16;
 };
+// Descriptors are advanced by adding 16-byte units to their 14-bit address
+// field, which therefore must not overflow for any tile.
+static_assert(1024 + 1024 + AnchorSmem::BAR < (1u << 18), "descriptor address field");
 
 struct AnchorParams {
   Geom g;
@@ -163,80 +175,115 @@ __device__ __forceinline__ float an_ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipes: x = i + f with i = floor(x), f in [0, 1);
-// 2^f ~ 1 + f (c1 + f (c2 + f c3)), a degree-3 fit with the constant term
-// fixed at 1, relative error below 8.6e-5 on [0, 1) (the coefficients minimise
-// the largest relative error, by iteratively reweighted least squares); the
-// integer part is added to the exponent field.  x >= -126 (callers clamp).
+// 2^x on the FMA pipes, none of it on the MUFU / conversion unit: x = n + f
+// with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f ~ 1 + f (c1 + f (c2 + f c3)), a degree-3 fit with the
+// constant term fixed at 1, relative error below 1.02e-4 on [-1/2, 1/2] (the
+// coefficients minimise the largest relative error, by iteratively reweighted
+// least squares); n enters the exponent field as (bits of x + 1.5 * 2^23) * 2^23,
+// the magic number's low nine bits being zero.  x >= -125 (callers clamp), x < 2^22.
 __device__ __forceinline__ float an_ex2_poly(float x) {
-  const float xi = floorf(x);
-  const float f = x - xi;
-  const float p = fmaf(fmaf(fmaf(0.07706520f, f, 0.22764701f), f, 0.69511634f), f, 1.f);
-  return __int_as_float(__float_as_int(p) + (int)((uint32_t)(int)xi << 23));
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.05500871f, f, 0.24221054f), f, 0.69328290f), f, 1.f);
+  return __int_as_float(__float_as_int(p) + (int)((uint32_t)__float_as_int(t) << 23));
+}
+
+// Packed fp32 pairs (one f32x2 instruction for both halves).
+__device__ __forceinline__ f2_t an_f2_add(f2_t a, f2_t b) {
+  f2_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// an_ex2_poly on a pair, the additions and the polynomial as f32x2.
+__device__ __forceinline__ void an_ex2_poly2(f2_t x, float& p0, float& p1) {
+  const f2_t magic = f2(12582912.f, 12582912.f), nmagic = f2(-12582912.f, -12582912.f);
+  const f2_t t = an_f2_add(x, magic);
+  const f2_t xr = an_f2_add(t, nmagic);
+  const f2_t f = f2_fma(xr, f2(-1.f, -1.f), x);
+  f2_t p = f2_fma(f2(0.05500871f, 0.05500871f), f, f2(0.24221054f, 0.24221054f));
+  p = f2_fma(p, f, f2(0.69328290f, 0.69328290f));
+  p = f2_fma(p, f, f2(1.f, 1.f));
+  p0 = __int_as_float(__float_as_int(f2_lo(p)) +
+                      (int)((uint32_t)__float_as_int(f2_lo(t)) << 23));
+  p1 = __int_as_float(__float_as_int(f2_hi(p)) +
+                      (int)((uint32_t)__float_as_int(f2_hi(t)) << 23));
 }
 
 __device__ __forceinline__ void tmem_ld32_at(uint32_t taddr, float* r) {
   tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(r));
 }
 
-// Half a tile of one query row (keys 64*kHalf .. 64*kHalf + 63): the weights
-// 2^(s - m) as bf16 pairs into w[32] (as float bit patterns for tcgen05.st),
-// the fp32 sum of the rounded weights returned.  kMask: keys at or past `kcount` get weight 0.
-template <bool kMask, int kHalf>
-__device__ __forceinline__ float an_weights(const float (&s)[128], float m, int kcount,
-                                            float (&w)[32]) {
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+__device__ __forceinline__ float an_max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// a0 += low bf16 half of w, a1 += high half (exact: fp32 sums of the rounded
+// weights, the ones P V multiplies).
+__device__ __forceinline__ void an_add_bf16x2(float& a0, float& a1, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(w));
+}
+
+// One 32-key chunk c of a row's scores: the chunk's maximum into mx, the
+// weights 2^(s - m) as bf16 pairs into w[16c .. 16c + 15] (the last
+// kAnPolyPairs pairs of every four by the polynomial), the rounded weights
+// added to acc.  kMask: keys at or past kcount get weight 0 and no say in the
+// maximum.
+template <bool kMask>
+__device__ __forceinline__ void an_chunk(const float (&s)[32], int c, float m, int kcount,
+                                         float& mx, float (&acc)[4], uint32_t (&w)[64]) {
+  float x[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int k = 64 * kHalf + 2 * i;
-    const float x0 = s[k] - m, x1 = s[k + 1] - m;
+  for (int i = 0; i < 32; ++i)
+    x[i] = (kMask && 32 * c + i >= kcount) ? -INFINITY : s[i];
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) mx = an_max3(mx, x[i], x[i + 1]);
+  const f2_t nm = f2(-m, -m);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const f2_t xm = an_f2_add(f2(x[2 * i], x[2 * i + 1]), nm);
     float p0, p1;
-    if ((i & 3) == 3) {
-      p0 = an_ex2_poly(fmaxf(x0, -126.f));
-      p1 = an_ex2_poly(fmaxf(x1, -126.f));
+    if ((i & 3) >= 4 - kAnPolyPairs) {
+      an_ex2_poly2(f2(fmaxf(f2_lo(xm), -125.f), fmaxf(f2_hi(xm), -125.f)), p0, p1);
+      if (kMask) {
+        if (32 * c + 2 * i >= kcount) p0 = 0.f;
+        if (32 * c + 2 * i + 1 >= kcount) p1 = 0.f;
+      }
     } else {
-      p0 = an_ex2(x0);
-      p1 = an_ex2(x1);
+      p0 = an_ex2(f2_lo(xm));    // 2^-inf = 0 for masked keys
+      p1 = an_ex2(f2_hi(xm));
     }
-    if (kMask) {
-      if (k >= kcount) p0 = 0.f;
-      if (k + 1 >= kcount) p1 = 0.f;
-    }
-    // The row sum adds the rounded weights, the ones P V multiplies: the
-    // normalised output is then a convex combination of v rows whatever the
-    // reference point (a row's largest weight is not exact in bf16 when the
-    // reference point lags the maximum).
     const uint32_t pk = pack_bf16(p0, p1);
-    acc[i & 3] += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xFFFF0000u);
-    w[i] = __uint_as_float(pk);
+    an_add_bf16x2(acc[(i & 1) * 2], acc[(i & 1) * 2 + 1], pk);
+    w[16 * c + i] = pk;
+  }
+}
+
+// A row's weights for one tile against the reference point m: the 128 scores
+// come from TMEM (tS) in four chunks, each load issued before the previous
+// chunk is processed.  Returns the sum of the rounded weights; mx gets the
+// tile's maximum.
+template <bool kMask>
+__device__ __forceinline__ float an_tile(uint32_t tS, float m, int kcount, float& mx,
+                                         uint32_t (&w)[64]) {
+  float sa[32], sb[32];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  mx = -INFINITY;
+  tmem_ld32(tS, sa);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (c < 3) tmem_ld32(tS + 32 * (c + 1), (c & 1) ? sa : sb);
+    an_chunk<kMask>((c & 1) ? sb : sa, c, m, kcount, mx, acc, w);
+    if (c < 3) tmem_wait_ld();
   }
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-
-// Both halves of a row's weights into P (TMEM columns tP .. tP + 63).
-template <bool kMask>
-__device__ __forceinline__ float an_weights_to_tmem(const float (&s)[128], float m, int kcount,
-                                                    uint32_t tP) {
-  float w[32];
-  float l = an_weights<kMask, 0>(s, m, kcount, w);
-  tmem_st32(tP, w);
-  l += an_weights<kMask, 1>(s, m, kcount, w);
-  tmem_st32(tP + 32, w);
-  return l;
-}
-
-template <bool kMask>
-__device__ __forceinline__ float an_rowmax(float (&s)[128], int kcount) {
-  float mx[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < 128; ++i) {
-    if (kMask && i >= kcount) s[i] = -INFINITY;
-    mx[i & 7] = fmaxf(mx[i & 7], s[i]);
-  }
-  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
 }
 
 // 10 warps: three share one SM sub-partition's 16 K registers, so at most
@@ -252,12 +299,12 @@ __global__ void __launch_bounds__(kAnThreads, 1)
   uint64_t* qfull = bars;
   uint64_t* kfull = bars + 1;      // [2]
   uint64_t* kfree = bars + 3;      // [2]
-  uint64_t* vfull = bars + 5;      // [2]
-  uint64_t* vfree = bars + 7;      // [2]
-  uint64_t* sfull = bars + 9;      // [2]: per query tile
-  uint64_t* pready = bars + 11;    // [2]
-  uint64_t* odone = bars + 13;     // [2]
-  uint64_t* drain = bars + 15;
+  uint64_t* vfull = bars + 5;      // [3]
+  uint64_t* vfree = vfull + kAnVS; // [3]
+  uint64_t* sfull = vfree + kAnVS; // [2]: per query tile
+  uint64_t* pready = sfull + kAnQT;
+  uint64_t* odone = pready + kAnQT;
+  uint64_t* drain = odone + kAnQT;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + AnchorSmem::MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + AnchorSmem::MISC + 4);
 
@@ -272,11 +319,15 @@ __global__ void __launch_bounds__(kAnThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&kfull[s], 1);
       mbar_init(&kfree[s], 1);
+    }
+    for (int s = 0; s < kAnVS; ++s) {
       mbar_init(&vfull[s], 1);
       mbar_init(&vfree[s], 1);
-      mbar_init(&sfull[s], 1);
-      mbar_init(&pready[s], 4);
-      mbar_init(&odone[s], 1);
+    }
+    for (int t = 0; t < kAnQT; ++t) {
+      mbar_init(&sfull[t], 1);
+      mbar_init(&pready[t], 4);
+      mbar_init(&odone[t], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -315,11 +366,12 @@ __global__ void __launch_bounds__(kAnThreads, 1)
         tma_load_3d(kt, &tmK, &kfull[s], h * 128, j * kAnTile, b, pol);
         tma_load_3d(kt + kBox, &tmK, &kfull[s], h * 128 + 64, j * kAnTile, b, pol);
         ++nk;
-        if (!mbar_wait(&vfree[s], ph ^ 1u, abort_flag)) break;
-        unsigned char* vt = sm + AnchorSmem::V + s * kTileBytes;
-        mbar_arrive_expect_tx(&vfull[s], kTileBytes);
-        tma_load_3d(vt, &tmV, &vfull[s], h * 128, j * kAnTile, b, pol);
-        tma_load_3d(vt + kBox, &tmV, &vfull[s], h * 128 + 64, j * kAnTile, b, pol);
+        const int sv = j % kAnVS;
+        if (!mbar_wait(&vfree[sv], (uint32_t)((j / kAnVS) & 1) ^ 1u, abort_flag)) break;
+        unsigned char* vt = sm + AnchorSmem::V + sv * kTileBytes;
+        mbar_arrive_expect_tx(&vfull[sv], kTileBytes);
+        tma_load_3d(vt, &tmV, &vfull[sv], h * 128, j * kAnTile, b, pol);
+        tma_load_3d(vt + kBox, &tmV, &vfull[sv], h * 128 + 64, j * kAnTile, b, pol);
         ++nv;
       }
       if (*abort_flag) {
@@ -329,58 +381,77 @@ __global__ void __launch_bounds__(kAnThreads, 1)
         mbar_wait(qfull, 0u, nd);
         for (int i2 = nk - (nk < 2 ? nk : 2); i2 < nk; ++i2)
           mbar_wait(&kfull[i2 & 1], (uint32_t)((i2 >> 1) & 1), nd);
-        for (int i2 = nv - (nv < 2 ? nv : 2); i2 < nv; ++i2)
-          mbar_wait(&vfull[i2 & 1], (uint32_t)((i2 >> 1) & 1), nd);
+        for (int i2 = nv - (nv < kAnVS ? nv : kAnVS); i2 < nv; ++i2)
+          mbar_wait(&vfull[i2 % kAnVS], (uint32_t)((i2 / kAnVS) & 1), nd);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     if (lane == 0) {
+      // The issuing thread shares its scheduler with two softmax warps, so
+      // its loop is kept short: shared-memory descriptors are built once per
+      // slot, and a K step only adds its offset (16-byte units) to them.
       constexpr uint32_t idS = idesc_f16(128, 128, false, false);
       constexpr uint32_t idPV = idesc_bf16(128, 128, false, true);
-      auto scores = [&](int t, int j) {   // S_t = q_til_t k_til_j^T
-        const uint32_t qt = sbase + AnchorSmem::Q + t * kTileBytes;
-        const uint32_t kt = sbase + AnchorSmem::K + (j & 1) * kTileBytes;
+      const uint64_t dQ0 = sdesc_sw128(sbase + AnchorSmem::Q, 16, 1024);
+      const uint64_t dQ1 = dQ0 + (kTileBytes >> 4);
+      const uint64_t dK0 = sdesc_sw128(sbase + AnchorSmem::K, 16, 1024);
+      const uint64_t dK1 = dK0 + (kTileBytes >> 4);
+      const uint64_t dV0 = sdesc_sw128(sbase + AnchorSmem::V, kBox, 1024);
+      auto scores = [&](uint32_t d, uint64_t dq, uint64_t dk) {   // S = q_til k_til^T
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32;
-          umma_f16kind(tmem + t * 128, sdesc_sw128(qt + koff, 16, 1024),
-                       sdesc_sw128(kt + koff, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          const uint32_t koff = (uint32_t)(kk >> 2) * (kBox >> 4) + (uint32_t)(kk & 3) * 2;
+          umma_f16kind(d, dq + koff, dk + koff, idS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&sfull[t]);
       };
-      auto pv = [&](int t, int j) {       // O_t += P_t v_j, P_t from TMEM
-        const uint32_t vt = sbase + AnchorSmem::V + (j & 1) * kTileBytes;
+      auto pv = [&](uint32_t d, uint32_t a, uint64_t dv, uint32_t acc0) {   // O += P v
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_f16kind_ta(tmem + kAnO + t * 128, tmem + t * 128 + kk * 8,
-                          sdesc_sw128(vt + kk * 2048, kBox, 1024), idPV,
-                          (j > 0 || kk > 0) ? 1u : 0u);
+          umma_f16kind_ta(d, a + kk * 8, dv + (uint32_t)kk * (2048 >> 4), idPV,
+                          kk > 0 ? 1u : acc0);
       };
       bool ok = mbar_wait(qfull, 0u, abort_flag) && mbar_wait(&kfull[0], 0u, abort_flag);
       if (ok) {
         tc_fence_after();
-        scores(0, 0);
-        scores(1, 0);
+        scores(tmem, dQ0, dK0);
+        umma_commit(&sfull[0]);
+        scores(tmem + 128, dQ1, dK0);
+        umma_commit(&sfull[1]);
         umma_commit(&kfree[0]);
       }
+      int sv = 0;                 // v slot of tile j
+      uint32_t phv = 0;           // its fill parity
       for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j & 1;
-        if (!(ok = mbar_wait(&vfull[s], (uint32_t)((j >> 1) & 1), abort_flag))) break;
-        for (int t = 0; t < kAnQT; ++t) {
-          if (!(ok = mbar_wait(&pready[t], (uint32_t)(j & 1), abort_flag))) break;
+        if (!(ok = mbar_wait(&vfull[sv], phv, abort_flag))) break;
+        const uint64_t dv = dV0 + (uint32_t)sv * (kTileBytes >> 4);
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
+        const bool more = j + 1 < nkv;
+        const uint64_t dk = ((j + 1) & 1) ? dK1 : dK0;     // k slot of tile j + 1
+        // query tile 0: O_0 += P_0 v_j, then S_0 of tile j + 1
+        if (!(ok = mbar_wait(&pready[0], (uint32_t)(j & 1), abort_flag))) break;
+        tc_fence_after();
+        pv(tmem + kAnO, tmem, dv, acc0);
+        if (more) {
+          if (!(ok = mbar_wait(&kfull[(j + 1) & 1], (uint32_t)(((j + 1) >> 1) & 1), abort_flag)))
+            break;
           tc_fence_after();
-          pv(t, j);
-          if (t == kAnQT - 1) umma_commit(&vfree[s]);
-          if (j + 1 < nkv) {
-            const int s1 = (j + 1) & 1;
-            if (t == 0 && !(ok = mbar_wait(&kfull[s1], (uint32_t)(((j + 1) >> 1) & 1),
-                                           abort_flag)))
-              break;
-            tc_fence_after();
-            scores(t, j + 1);
-            if (t == kAnQT - 1) umma_commit(&kfree[s1]);
-          }
+          scores(tmem, dQ0, dk);
+          umma_commit(&sfull[0]);
+        }
+        // query tile 1
+        if (!(ok = mbar_wait(&pready[1], (uint32_t)(j & 1), abort_flag))) break;
+        tc_fence_after();
+        pv(tmem + kAnO + 128, tmem + 128, dv, acc0);
+        umma_commit(&vfree[sv]);
+        if (more) {
+          scores(tmem + 128, dQ1, dk);
+          umma_commit(&sfull[1]);
+          umma_commit(&kfree[(j + 1) & 1]);
+        }
+        if (++sv == kAnVS) {
+          sv = 0;
+          phv ^= 1u;
         }
       }
       if (ok)
@@ -405,23 +476,30 @@ __global__ void __launch_bounds__(kAnThreads, 1)
         break;
       }
       tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32_at(tS + c * 32, s + c * 32);
-      tmem_wait_ld();
       const int kcount = g.N - j * kAnTile;
-      const float mt = kcount < kAnTile ? an_rowmax<true>(s, kcount) : an_rowmax<false>(s, kcount);
+      const bool last = kcount < kAnTile;
+      // One pass against the current reference point; the tile maximum it
+      // finds decides afterwards whether the point has to move (weights above
+      // 2^8, or the first tile), in which case the tile is redone from TMEM
+      // (P is not written yet) against the new point.
+      uint32_t w[64];
+      float mt;
+      float lt = last ? an_tile<true>(tS, m, kcount, mt, w) : an_tile<false>(tS, m, kcount, mt, w);
       const bool grow = mt > m + kAnLazy;
       float alpha = 1.f;
-      const bool rescale = __any_sync(0xffffffffu, grow) && j > 0;
-      if (grow) {
-        alpha = an_ex2(m - mt);   // 0 on the first tile
-        l *= alpha;
-        m = mt;
+      const bool redo = __any_sync(0xffffffffu, grow);
+      if (redo) {
+        if (grow) {
+          alpha = an_ex2(m - mt);   // 0 on the first tile
+          l *= alpha;
+          m = mt;
+        }
+        lt = last ? an_tile<true>(tS, m, kcount, mt, w) : an_tile<false>(tS, m, kcount, mt, w);
       }
-      l += kcount < kAnTile ? an_weights_to_tmem<true>(s, m, kcount, tS)
-                            : an_weights_to_tmem<false>(s, m, kcount, tS);
-      if (rescale) {
+      l += lt;
+      tmem_st32(tS, *reinterpret_cast<float(*)[32]>(&w[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
+      if (redo && j > 0) {
         // O_t holds the tiles before j at the old reference point; PV_t(j-1)
         // landed before S_t(j) did, and PV_t(j) waits for this warp's arrival.
 #pragma unroll 1
