@@ -128,6 +128,13 @@ _BYTE_UNITS = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1
 _TIME_UNITS = {"ns": 1e-3, "us": 1.0, "usecond": 1.0, "msecond": 1e3, "ms": 1e3, "nsecond": 1e-3}
 
 
+def kernel_base_name(full):
+    """'void gla::tc_apply_kernel<0>(CUtensorMap_st, ...)' -> 'tc_apply_kernel'."""
+    import re
+    head = re.sub(r"<.*>", "", full.split("(")[0])
+    return head.split()[-1].split("::")[-1]
+
+
 def ingest_ncu(csv_path, workload):
     """Per kernel of an ncu raw-page CSV export: the mean over its captured
     launches of dram__bytes_read.sum + dram__bytes_write.sum (bytes per
@@ -145,7 +152,7 @@ def ingest_ncu(csv_path, workload):
     for r in data:
         if len(r) != len(cols):
             continue
-        name = r[ix["Kernel Name"]].split("(")[0].split()[-1].split("<")[0]
+        name = kernel_base_name(r[ix["Kernel Name"]])
         byt = sum(float(r[ix[m]]) * _BYTE_UNITS[units[ix[m]]]
                   for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"))
         dur = float(r[ix["gpu__time_duration.sum"]]) * _TIME_UNITS[units[ix["gpu__time_duration.sum"]]]
