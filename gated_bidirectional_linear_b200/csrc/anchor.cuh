@@ -5,17 +5,15 @@
 // and out.
 //
 //   anchor_prep_kernel  q_til * log2(e) / sqrt(d) and k_til as fp16 in the
-//                       [B][N][Hh][128] layout (one warp per token-head).
-//   anchor_attn_kernel  one CTA per 128 queries of a head: TMA streams the
-//                       head's key / value tiles (128 tokens) through a 2-slot
-//                       ring; one thread issues S = Q K^T (fp16) into one of two
-//                       TMEM score buffers, so the next tile's scores run while
-//                       the softmax warps (one query row per thread) take the
-//                       row maximum, exp2 and the running sum of this one and
-//                       write P (bf16) to shared memory; O += P V (bf16)
-//                       accumulates in TMEM, rescaled by the softmax warps when
-//                       a row maximum grows.  The epilogue divides by the row
-//                       sum, applies the gate and stores bf16 rows.
+//                       [B][N][Hh][128] layout (one warp per token, every head).
+//   anchor_attn_kernel  one CTA per two 128-query tiles of a head: TMA streams
+//                       the head's key / value tiles (128 tokens); one thread
+//                       issues S = Q K^T (fp16) and O += P V (bf16, P read from
+//                       TMEM); two softmax warpgroups (one query row per thread)
+//                       turn each tile's scores into bf16 weights in TMEM while
+//                       the tensor cores work for the other query tile.  The
+//                       epilogue divides by the row sum, applies the gate and
+//                       stores bf16 rows.
 #pragma once
 
 #include "tc.cuh"
@@ -58,7 +56,7 @@ __device__ __forceinline__ uint2 an_prep_row(uint2 r, const float (&c)[2], const
 }
 
 // A grid-stride loop over tokens; one warp per token takes every head of it
-// (the rotation depends on the token only), two heads per step.
+// (the rotation depends on the token only), four heads per step.
 __global__ void __launch_bounds__(kAnWarpsPrep * 32) anchor_prep_kernel(AnchorPrepParams p) {
   pdl_launch_dependents();   // the attention CTAs may set up meanwhile
   const Geom& g = p.g;
@@ -166,6 +164,15 @@ __device__ __forceinline__ void umma_f16kind_ta(uint32_t d_tmem, uint32_t a_tmem
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// One lane of the (fully active) warp gets true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // 2^x on the MUFU unit (ex2.approx: flushes subnormals, 2^-inf = 0).
@@ -387,67 +394,78 @@ __global__ void __launch_bounds__(kAnThreads, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
-      // The issuing thread shares its scheduler with two softmax warps, so
-      // its loop is kept short: shared-memory descriptors are built once per
-      // slot, and a K step only adds its offset (16-byte units) to them.
+    {
+      // The whole warp runs the loop (warp-uniform control and descriptor
+      // arithmetic) and one elected lane issues: the warp shares its
+      // scheduler with two softmax warps, so the issue path is kept short.
+      // Shared-memory descriptors are built once per slot, and a K step only
+      // adds its offset (16-byte units) to them.
       constexpr uint32_t idS = idesc_f16(128, 128, false, false);
       constexpr uint32_t idPV = idesc_bf16(128, 128, false, true);
+      const bool leader = elect_one();
       const uint64_t dQ0 = sdesc_sw128(sbase + AnchorSmem::Q, 16, 1024);
       const uint64_t dQ1 = dQ0 + (kTileBytes >> 4);
       const uint64_t dK0 = sdesc_sw128(sbase + AnchorSmem::K, 16, 1024);
       const uint64_t dK1 = dK0 + (kTileBytes >> 4);
       const uint64_t dV0 = sdesc_sw128(sbase + AnchorSmem::V, kBox, 1024);
-      auto scores = [&](uint32_t d, uint64_t dq, uint64_t dk) {   // S = q_til k_til^T
+      auto scores = [&](uint32_t d, uint64_t dq, uint64_t dk, uint64_t* bar) {   // S = q_til k_til^T
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (uint32_t)(kk >> 2) * (kBox >> 4) + (uint32_t)(kk & 3) * 2;
-          umma_f16kind(d, dq + koff, dk + koff, idS, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (uint32_t)(kk >> 2) * (kBox >> 4) + (uint32_t)(kk & 3) * 2;
+            umma_f16kind(d, dq + koff, dk + koff, idS, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar);
         }
+        __syncwarp();
       };
       auto pv = [&](uint32_t d, uint32_t a, uint64_t dv, uint32_t acc0) {   // O += P v
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_f16kind_ta(d, a + kk * 8, dv + (uint32_t)kk * (2048 >> 4), idPV,
-                          kk > 0 ? 1u : acc0);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16kind_ta(d, a + kk * 8, dv + (uint32_t)kk * (2048 >> 4), idPV,
+                            kk > 0 ? 1u : acc0);
+        }
+        __syncwarp();
       };
-      bool ok = mbar_wait(qfull, 0u, abort_flag) && mbar_wait(&kfull[0], 0u, abort_flag);
+      auto commit = [&](uint64_t* bar) {
+        if (leader) umma_commit(bar);
+        __syncwarp();
+      };
+      bool ok = mbar_wait_warp(qfull, 0u, abort_flag) && mbar_wait_warp(&kfull[0], 0u, abort_flag);
       if (ok) {
         tc_fence_after();
-        scores(tmem, dQ0, dK0);
-        umma_commit(&sfull[0]);
-        scores(tmem + 128, dQ1, dK0);
-        umma_commit(&sfull[1]);
-        umma_commit(&kfree[0]);
+        scores(tmem, dQ0, dK0, &sfull[0]);
+        scores(tmem + 128, dQ1, dK0, &sfull[1]);
+        commit(&kfree[0]);
       }
       int sv = 0;                 // v slot of tile j
       uint32_t phv = 0;           // its fill parity
       for (int j = 0; ok && j < nkv; ++j) {
-        if (!(ok = mbar_wait(&vfull[sv], phv, abort_flag))) break;
+        if (!(ok = mbar_wait_warp(&vfull[sv], phv, abort_flag))) break;
         const uint64_t dv = dV0 + (uint32_t)sv * (kTileBytes >> 4);
         const uint32_t acc0 = j > 0 ? 1u : 0u;
         const bool more = j + 1 < nkv;
         const uint64_t dk = ((j + 1) & 1) ? dK1 : dK0;     // k slot of tile j + 1
         // query tile 0: O_0 += P_0 v_j, then S_0 of tile j + 1
-        if (!(ok = mbar_wait(&pready[0], (uint32_t)(j & 1), abort_flag))) break;
+        if (!(ok = mbar_wait_warp(&pready[0], (uint32_t)(j & 1), abort_flag))) break;
         tc_fence_after();
         pv(tmem + kAnO, tmem, dv, acc0);
         if (more) {
-          if (!(ok = mbar_wait(&kfull[(j + 1) & 1], (uint32_t)(((j + 1) >> 1) & 1), abort_flag)))
+          if (!(ok = mbar_wait_warp(&kfull[(j + 1) & 1], (uint32_t)(((j + 1) >> 1) & 1),
+                                    abort_flag)))
             break;
           tc_fence_after();
-          scores(tmem, dQ0, dk);
-          umma_commit(&sfull[0]);
+          scores(tmem, dQ0, dk, &sfull[0]);
         }
         // query tile 1
-        if (!(ok = mbar_wait(&pready[1], (uint32_t)(j & 1), abort_flag))) break;
+        if (!(ok = mbar_wait_warp(&pready[1], (uint32_t)(j & 1), abort_flag))) break;
         tc_fence_after();
         pv(tmem + kAnO + 128, tmem + 128, dv, acc0);
-        umma_commit(&vfree[sv]);
+        commit(&vfree[sv]);
         if (more) {
-          scores(tmem + 128, dQ1, dk);
-          umma_commit(&sfull[1]);
-          umma_commit(&kfree[(j + 1) & 1]);
+          scores(tmem + 128, dQ1, dk, &sfull[1]);
+          commit(&kfree[(j + 1) & 1]);
         }
         if (++sv == kAnVS) {
           sv = 0;
@@ -455,10 +473,10 @@ __global__ void __launch_bounds__(kAnThreads, 1)
         }
       }
       if (ok)
-        for (int t = 0; t < kAnQT; ++t) umma_commit(&odone[t]);
-      umma_commit(drain);
+        for (int t = 0; t < kAnQT; ++t) commit(&odone[t]);
+      commit(drain);
       int dummy = 0;
-      mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy));
+      mbar_wait_warp(drain, 0, reinterpret_cast<volatile int*>(&dummy));
     }
   } else {
     // --------------------------------------------------------- softmax warps

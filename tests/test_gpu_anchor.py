@@ -4,8 +4,8 @@ attention, sigmoid output gate).
 
 The kernel takes scores on the tensor cores from fp16 q_til / k_til, rounds
 the softmax weights to bf16 for P V and sums those rounded weights in fp32;
-the bar is
-the bf16 one, 2e-2 of the output RMS beyond the output's own bf16 rounding.
+the bar is the bf16 one, 2e-2 of the output RMS beyond the output's own bf16
+rounding.
 Small shapes and 480p are compared on every element; 720p and the 14B-width
 layer on sampled heads and query rows that span the first, a middle and the
 ragged last 128-token tile."""
