@@ -117,20 +117,22 @@ __global__ void __launch_bounds__(kAnWarpsPrep * 32) anchor_prep_kernel(AnchorPr
 // The MMA order S_0(j), S_1(j), PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ... lets
 // one warpgroup's softmax run while the tensor cores work for the other.  A
 // tcgen05.commit tracks every MMA issued before it, so S_t(j) landing also
-// means PV_t(j-1) has: the softmax may then rescale O_t without another wait.
+// means PV_t(j-1) has, and the softmax may overwrite P_t.
 //
-// Running maximum: a row keeps the maximum it last rescaled to and rescales
-// (O, the row sum) only when a tile's maximum exceeds it by more than 2^8, so
-// that weights stay below 256; the normalisation at the end is the same for
-// any such reference point.  exp2 runs on the MUFU unit for three of every
-// four weight pairs and as a polynomial on the FMA pipes for the fourth.
+// No running maximum: q_til and k_til are RMS-normalised and rotated, so
+// |q_til| = |k_til| <= sqrt(d) and every score in base 2,
+// q_til . k_til * log2(e) / sqrt(d), lies within +-sqrt(d) log2(e) = +-16.33
+// (d = 128).  The weights 2^s then lie in [2^-16.4, 2^16.4], normal in bf16 and
+// fp32, and the normalisation O / l at the end is the softmax for any common
+// shift of the scores: no maximum, no rescale of O.  exp2 runs on the MUFU
+// unit for three of every four weight pairs and as a polynomial on the FMA
+// pipes for the fourth.
 
 constexpr int kAnTile = 128;
 constexpr int kAnQT = 2;                          // query tiles per CTA
 constexpr int kAnSW0 = 2;                         // first softmax warp
 constexpr int kAnThreads = (kAnSW0 + 4 * kAnQT) * 32;
 constexpr uint32_t kAnO = 256;                    // TMEM column of O_0
-constexpr float kAnLazy = 8.f;                    // log2 of the largest weight
 constexpr int kAnVS = 3;                          // v ring slots
 constexpr int kAnPolyPairs = 1;                   // of every 4 weight pairs, by polynomial
 static_assert(kAnQT == 2, "the MMA issue order interleaves exactly two query tiles");
@@ -222,12 +224,6 @@ __device__ __forceinline__ void tmem_ld32_at(uint32_t taddr, float* r) {
   tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(r));
 }
 
-__device__ __forceinline__ float an_max3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // a0 += low bf16 half of w, a1 += high half (exact: fp32 sums of the rounded
 // weights, the ones P V multiplies).
 __device__ __forceinline__ void an_add_bf16x2(float& a0, float& a1, uint32_t w) {
@@ -237,57 +233,60 @@ __device__ __forceinline__ void an_add_bf16x2(float& a0, float& a1, uint32_t w) 
       : "r"(w));
 }
 
-// One 32-key chunk c of a row's scores: the chunk's maximum into mx, the
-// weights 2^(s - m) as bf16 pairs into w[16c .. 16c + 15] (the last
-// kAnPolyPairs pairs of every four by the polynomial), the rounded weights
-// added to acc.  kMask: keys at or past kcount get weight 0 and no say in the
-// maximum.
+// 16 consecutive 32-bit TMEM columns of this warp's lane quarter.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&u)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
+      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]),
+      "r"(u[15])
+      : "memory");
+}
+
+// One 32-key chunk c of a row's scores s (base 2, |s| <= 16.33): the weights
+// 2^s as bf16 pairs into w (the last kAnPolyPairs pairs of every four by the
+// polynomial), the rounded weights added to acc.  kMask: keys at or past
+// kcount get weight 0.
 template <bool kMask>
-__device__ __forceinline__ void an_chunk(const float (&s)[32], int c, float m, int kcount,
-                                         float& mx, float (&acc)[4], uint32_t (&w)[64]) {
-  float x[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i)
-    x[i] = (kMask && 32 * c + i >= kcount) ? -INFINITY : s[i];
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) mx = an_max3(mx, x[i], x[i + 1]);
-  const f2_t nm = f2(-m, -m);
+__device__ __forceinline__ void an_chunk(const float (&s)[32], int c, int kcount,
+                                         float (&acc)[4], uint32_t (&w)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const f2_t xm = an_f2_add(f2(x[2 * i], x[2 * i + 1]), nm);
+    const int k0 = 32 * c + 2 * i;
     float p0, p1;
     if ((i & 3) >= 4 - kAnPolyPairs) {
-      an_ex2_poly2(f2(fmaxf(f2_lo(xm), -125.f), fmaxf(f2_hi(xm), -125.f)), p0, p1);
+      an_ex2_poly2(f2(s[2 * i], s[2 * i + 1]), p0, p1);
       if (kMask) {
-        if (32 * c + 2 * i >= kcount) p0 = 0.f;
-        if (32 * c + 2 * i + 1 >= kcount) p1 = 0.f;
+        if (k0 >= kcount) p0 = 0.f;
+        if (k0 + 1 >= kcount) p1 = 0.f;
       }
     } else {
-      p0 = an_ex2(f2_lo(xm));    // 2^-inf = 0 for masked keys
-      p1 = an_ex2(f2_hi(xm));
+      p0 = an_ex2(kMask && k0 >= kcount ? -INFINITY : s[2 * i]);
+      p1 = an_ex2(kMask && k0 + 1 >= kcount ? -INFINITY : s[2 * i + 1]);
     }
     const uint32_t pk = pack_bf16(p0, p1);
     an_add_bf16x2(acc[(i & 1) * 2], acc[(i & 1) * 2 + 1], pk);
-    w[16 * c + i] = pk;
+    w[i] = pk;
   }
 }
 
-// A row's weights for one tile against the reference point m: the 128 scores
-// come from TMEM (tS) in four chunks, each load issued before the previous
-// chunk is processed.  Returns the sum of the rounded weights; mx gets the
-// tile's maximum.
+// A row's weights for one tile: the 128 scores come from TMEM (tS) in four
+// 32-column chunks, each load issued before the previous chunk is processed;
+// chunk c's 16 packed weight columns go to tS + 16c, over score columns that
+// are already in registers.  Returns the sum of the rounded weights.
 template <bool kMask>
-__device__ __forceinline__ float an_tile(uint32_t tS, float m, int kcount, float& mx,
-                                         uint32_t (&w)[64]) {
+__device__ __forceinline__ float an_tile(uint32_t tS, int kcount) {
   float sa[32], sb[32];
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  mx = -INFINITY;
   tmem_ld32(tS, sa);
   tmem_wait_ld();
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     if (c < 3) tmem_ld32(tS + 32 * (c + 1), (c & 1) ? sa : sb);
-    an_chunk<kMask>((c & 1) ? sb : sa, c, m, kcount, mx, acc, w);
+    uint32_t w[16];
+    an_chunk<kMask>((c & 1) ? sb : sa, c, kcount, acc, w);
+    tmem_st16(tS + 16 * c, w);
     if (c < 3) tmem_wait_ld();
   }
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
@@ -486,7 +485,7 @@ __global__ void __launch_bounds__(kAnThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t tS = tmem + t * 128 + lane_off;
     const uint32_t tO = tmem + kAnO + t * 128 + lane_off;
-    float m = -INFINITY, l = 0.f;
+    float l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       if (!mbar_wait_warp(&sfull[t], (uint32_t)(j & 1), abort_flag)) {
@@ -495,41 +494,7 @@ __global__ void __launch_bounds__(kAnThreads, 1)
       }
       tc_fence_after();
       const int kcount = g.N - j * kAnTile;
-      const bool last = kcount < kAnTile;
-      // One pass against the current reference point; the tile maximum it
-      // finds decides afterwards whether the point has to move (weights above
-      // 2^8, or the first tile), in which case the tile is redone from TMEM
-      // (P is not written yet) against the new point.
-      uint32_t w[64];
-      float mt;
-      float lt = last ? an_tile<true>(tS, m, kcount, mt, w) : an_tile<false>(tS, m, kcount, mt, w);
-      const bool grow = mt > m + kAnLazy;
-      float alpha = 1.f;
-      const bool redo = __any_sync(0xffffffffu, grow);
-      if (redo) {
-        if (grow) {
-          alpha = an_ex2(m - mt);   // 0 on the first tile
-          l *= alpha;
-          m = mt;
-        }
-        lt = last ? an_tile<true>(tS, m, kcount, mt, w) : an_tile<false>(tS, m, kcount, mt, w);
-      }
-      l += lt;
-      tmem_st32(tS, *reinterpret_cast<float(*)[32]>(&w[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
-      if (redo && j > 0) {
-        // O_t holds the tiles before j at the old reference point; PV_t(j-1)
-        // landed before S_t(j) did, and PV_t(j) waits for this warp's arrival.
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(tO + c * 32, o);
-        }
-      }
+      l += kcount < kAnTile ? an_tile<true>(tS, kcount) : an_tile<false>(tS, kcount);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
