@@ -56,7 +56,9 @@ __device__ __forceinline__ uint2 an_prep_row(uint2 r, const float (&c)[2], const
 }
 
 // A grid-stride loop over tokens; one warp per token takes every head of it
-// (the rotation depends on the token only), four heads per step.
+// (the rotation depends on the token only), four heads per step.  The loads of
+// the next step (the next four heads, or the first four of the warp's next
+// token) are issued before the current step is processed.
 __global__ void __launch_bounds__(kAnWarpsPrep * 32) anchor_prep_kernel(AnchorPrepParams p) {
   pdl_launch_dependents();   // the attention CTAs may set up meanwhile
   const Geom& g = p.g;
@@ -65,8 +67,20 @@ __global__ void __launch_bounds__(kAnWarpsPrep * 32) anchor_prep_kernel(AnchorPr
   const long long nwarps = (long long)gridDim.x * kAnWarpsPrep;
   const int HW = g.H * g.W;
   constexpr float kQScale = 0.12751743f;   // log2(e) / sqrt(128)
-  for (long long bn = (long long)blockIdx.x * kAnWarpsPrep + (threadIdx.x >> 5); bn < tokens;
-       bn += nwarps) {
+  long long bn = (long long)blockIdx.x * kAnWarpsPrep + (threadIdx.x >> 5);
+  if (bn >= tokens) return;
+  uint2 qn[4], kn[4];     // the next step's rows
+  auto load = [&](long long tok, int h0) {
+    const size_t base = (size_t)tok * g.Hh * 128 + 4 * lane;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const size_t o = base + (size_t)(h0 + u < g.Hh ? h0 + u : h0) * 128;
+      qn[u] = ldg_u2(p.q + o);
+      kn[u] = ldg_u2(p.k + o);
+    }
+  };
+  load(bn, 0);
+  for (; bn < tokens; bn += nwarps) {
     const int n = (int)(bn % g.N);
     const int f = n / HW, hh = (n / g.W) % g.H, ww = n % g.W;
     float c[2] = {1.f, 1.f}, sn[2] = {0.f, 0.f};
@@ -82,14 +96,17 @@ __global__ void __launch_bounds__(kAnWarpsPrep * 32) anchor_prep_kernel(AnchorPr
       }
     }
     const size_t base = (size_t)bn * g.Hh * 128 + 4 * lane;
-    // Four heads per step, all eight loads issued before any use.
     for (int h0 = 0; h0 < g.Hh; h0 += 4) {
       uint2 qr[4], kr[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const size_t o = base + (size_t)(h0 + u < g.Hh ? h0 + u : h0) * 128;
-        qr[u] = ldg_u2(p.q + o);
-        kr[u] = ldg_u2(p.k + o);
+        qr[u] = qn[u];
+        kr[u] = kn[u];
+      }
+      if (h0 + 4 < g.Hh) {
+        load(bn, h0 + 4);
+      } else if (bn + nwarps < tokens) {
+        load(bn + nwarps, 0);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -184,20 +201,6 @@ __device__ __forceinline__ float an_ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipes, none of it on the MUFU / conversion unit: x = n + f
-// with n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa bits) and
-// f in [-1/2, 1/2]; 2^f ~ 1 + f (c1 + f (c2 + f c3)), a degree-3 fit with the
-// constant term fixed at 1, relative error below 1.02e-4 on [-1/2, 1/2] (the
-// coefficients minimise the largest relative error, by iteratively reweighted
-// least squares); n enters the exponent field as (bits of x + 1.5 * 2^23) * 2^23,
-// the magic number's low nine bits being zero.  x >= -125 (callers clamp), x < 2^22.
-__device__ __forceinline__ float an_ex2_poly(float x) {
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.05500871f, f, 0.24221054f), f, 0.69328290f), f, 1.f);
-  return __int_as_float(__float_as_int(p) + (int)((uint32_t)__float_as_int(t) << 23));
-}
-
 // Packed fp32 pairs (one f32x2 instruction for both halves).
 __device__ __forceinline__ f2_t an_f2_add(f2_t a, f2_t b) {
   f2_t d;
@@ -205,14 +208,23 @@ __device__ __forceinline__ f2_t an_f2_add(f2_t a, f2_t b) {
   return d;
 }
 
-// an_ex2_poly on a pair, the additions and the polynomial as f32x2.
+// 2^x for a pair, on the FMA pipes (f32x2), none of it on the MUFU /
+// conversion unit: x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in
+// the low mantissa bits) and f in [-1/2, 1/2]; 2^f ~ 1 + f (c1 + f (c2 + f (c3
+// + f c4))), a degree-4 fit with the constant term fixed at 1, relative error
+// below 2.9e-6 on [-1/2, 1/2] (the coefficients minimise the largest relative
+// error, by iteratively reweighted least squares), so that a weight rounds to
+// the same bf16 as the MUFU's ex2 nearly always; n enters the exponent field
+// as (bits of x + 1.5 * 2^23) * 2^23, the magic number's low nine bits being
+// zero.  |x| < 126.
 __device__ __forceinline__ void an_ex2_poly2(f2_t x, float& p0, float& p1) {
   const f2_t magic = f2(12582912.f, 12582912.f), nmagic = f2(-12582912.f, -12582912.f);
   const f2_t t = an_f2_add(x, magic);
   const f2_t xr = an_f2_add(t, nmagic);
   const f2_t f = f2_fma(xr, f2(-1.f, -1.f), x);
-  f2_t p = f2_fma(f2(0.05500871f, 0.05500871f), f, f2(0.24221054f, 0.24221054f));
-  p = f2_fma(p, f, f2(0.69328290f, 0.69328290f));
+  f2_t p = f2_fma(f2(0.0095828352f, 0.0095828352f), f, f2(0.055906396f, 0.055906396f));
+  p = f2_fma(p, f, f2(0.24024099f, 0.24024099f));
+  p = f2_fma(p, f, f2(0.69312418f, 0.69312418f));
   p = f2_fma(p, f, f2(1.f, 1.f));
   p0 = __int_as_float(__float_as_int(f2_lo(p)) +
                       (int)((uint32_t)__float_as_int(f2_lo(t)) << 23));
@@ -563,7 +575,18 @@ inline gla_status run_anchor(const Geom& g, const void* q, const void* k, const 
   pp.kt = kt;
   const long long tokens = (long long)g.B * g.N;
   const long long blocks = (tokens + kAnWarpsPrep - 1) / kAnWarpsPrep;
-  const int grid = (int)(blocks < 8LL * sms ? blocks : 8LL * sms);
+  // One wave of resident blocks: the grid-stride loop spreads the tokens.
+  static std::atomic<int> resident{0};
+  int per_sm = resident.load(std::memory_order_relaxed);
+  if (per_sm <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, anchor_prep_kernel,
+                                                      kAnWarpsPrep * 32, 0) != cudaSuccess ||
+        per_sm <= 0)
+      return GLA_ERR_CUDA;
+    resident.store(per_sm, std::memory_order_relaxed);
+  }
+  const long long cap = (long long)per_sm * sms;
+  const int grid = (int)(blocks < cap ? blocks : cap);
   anchor_prep_kernel<<<grid, kAnWarpsPrep * 32, 0, stream>>>(pp);
   if (cudaGetLastError() != cudaSuccess || rec(1) != cudaSuccess) return GLA_ERR_CUDA;
 
