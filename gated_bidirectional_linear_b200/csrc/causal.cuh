@@ -646,9 +646,11 @@ __global__ void __launch_bounds__(kCaThreads, 1)
     lane_rope(g, j, smem_u32(tab), lr);
     // The lane's two 16-byte chunks in rows rg and 4 + rg: a row group
     // starting at row R (a multiple of 4) has swizzle phase 4 ((R >> 2) & 1) + rg.
-    uint32_t ch0[2], ch1[2];
-    lane_chunks(0, kCaBox, rg, j, ch0[0], ch1[0]);
-    lane_chunks(0, kCaBox, 4 + rg, j, ch0[1], ch1[1]);
+    // (Four scalars chosen by select, not an array indexed by the phase: that
+    // would live in local memory and be reloaded for every row group.)
+    uint32_t ch0a, ch1a, ch0b, ch1b;
+    lane_chunks(0, kCaBox, rg, j, ch0a, ch1a);
+    lane_chunks(0, kCaBox, 4 + rg, j, ch0b, ch1b);
     // Lanes of the row group above: rg - 1 (rg = lane bit 2 | lane bit 4 << 1),
     // rg - 2, and the group's last row (rg = 3).
     const int src1 = (rg & 1) ? (lane ^ 4) : (lane ^ 20);
@@ -695,7 +697,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         const uint32_t roff = (uint32_t)(R & ~7) * 128u;
         const int ph = (R >> 2) & 1;
         f2_t x[8];
-        unpack8(lds128(kt + ch0[ph] + roff), lds128(kt + ch1[ph] + roff), x);
+        unpack8(lds128(kt + (ph ? ch0b : ch0a) + roff), lds128(kt + (ph ? ch1b : ch1a) + roff), x);
         const float rstd = row_rstd(x);
         const f2_t rstd2 = f2(rstd, rstd);
 #pragma unroll
@@ -757,7 +759,7 @@ __global__ void __launch_bounds__(kCaThreads, 1)
         const int r = R + rg;
         const uint32_t roff = (uint32_t)(R & ~7) * 128u;
         const int ph = (R >> 2) & 1;
-        const uint32_t c0 = ch0[ph] + roff, c1 = ch1[ph] + roff;
+        const uint32_t c0 = (ph ? ch0b : ch0a) + roff, c1 = (ph ? ch1b : ch1a) + roff;
         uint32_t t012 = 0, t345 = 0, t67 = 0;
         if (g.rope_on) lane_rope_row(lr, rec_s + r * kRecBytes, t012, t345, t67);
         const uint4 k0 = lds128(kt + c0), k1 = lds128(kt + c1);
