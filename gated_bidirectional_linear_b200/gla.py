@@ -520,9 +520,11 @@ def gla_softmax_anchor(q, k, v, g, T, H, W, rope_theta=10000.0, out=None, worksp
     shape = tuple(q.shape)
     for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("out", out)):
         if tuple(t.shape) != shape or t.dtype != torch.bfloat16 or t.device != q.device \
-                or t.device.type != "cuda" or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous bf16 GPU tensor of shape {shape} "
+                or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor of shape {shape} "
                              f"on {q.device}")
+    if q.device.type != "cuda":
+        raise ValueError(f"q is on {q.device}; gla_softmax_anchor takes GPU tensors")
     if workspace is None:
         workspace = alloc_workspace(gla_softmax_anchor_workspace_size(B, Hh, d, T, H, W),
                                     q.device)

@@ -80,3 +80,29 @@ def test_stream_of_another_device_is_refused():
     with pytest.raises(ValueError, match="stream"):
         gla._stream(_FakeStream("cuda:1"), torch.device("cuda", 0))
     assert gla._stream(_FakeStream("cuda:0"), torch.device("cuda", 0)).value in (None, 0)
+
+
+def test_other_entries_reject_host_tensors():
+    x = host_inputs()
+    S = torch.zeros(B, HEADS, D, D)
+    z = torch.zeros(B, HEADS, D)
+    with pytest.raises(ValueError, match="GPU"):
+        gla.gla_causal_step(S, z, x["q"], x["k"], x["v"], x["beta"], x["g"], T, H, W)
+    with pytest.raises(ValueError, match="GPU"):
+        gla.gla_softmax_anchor(x["q"], x["k"], x["v"], x["g"], T, H, W)
+    a = torch.zeros(16, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="GPU"):
+        gla.gla_gemm_bf16(a, a)
+    mx = {n: torch.zeros(B, T * H * W, HEADS, D, dtype=torch.uint8) for n in "qkvg"}
+    mx.update({n + "_scale": torch.zeros(B, T * H * W, HEADS, 4, dtype=torch.uint8) for n in "qkvg"})
+    mx["beta"] = x["beta"]
+    with pytest.raises(ValueError):
+        gla.gla_forward_mx(mx, T, H, W)
+
+
+def test_anchor_checks_dtype_and_shape():
+    x = host_inputs()
+    with pytest.raises(ValueError, match="v"):
+        gla.gla_softmax_anchor(x["q"], x["k"], x["v"].float(), x["g"], T, H, W)
+    with pytest.raises(ValueError, match="tokens"):
+        gla.gla_softmax_anchor(x["q"], x["k"], x["v"], x["g"], T + 1, H, W)
