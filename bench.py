@@ -827,11 +827,11 @@ def run_layer(args, wl, gla, dev, dist, world, rank, local):
     if gla.gla_get_device_status(stream) != gla.GLA_OK:
         raise RuntimeError("device status after the timed region")
 
-    # Per stage, events around the three calls (the stages then do not overlap).
-    p = {}
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    t_in, t_op, t_out = [], [], []
-    for _ in range(steps):
+    # Per stage, events around the three calls (the stages then do not
+    # overlap), one set per step, the steps back to back with one
+    # synchronisation at the end.
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for ev in evs:
         ev[0].record(stream)
         p = gla.gla_project_in(x, W_in, wl.batch, wl.tokens, Hh, d, stream=stream)
         ev[1].record(stream)
@@ -840,10 +840,10 @@ def run_layer(args, wl, gla, dev, dist, world, rank, local):
         ev[2].record(stream)
         gla.gla_gemm_bf16(o.view(tokens, C), W_o, out=y, stream=stream)
         ev[3].record(stream)
-        torch.cuda.synchronize(dev)
-        t_in.append(ev[0].elapsed_time(ev[1]))
-        t_op.append(ev[1].elapsed_time(ev[2]))
-        t_out.append(ev[2].elapsed_time(ev[3]))
+    torch.cuda.synchronize(dev)
+    t_in = [ev[0].elapsed_time(ev[1]) for ev in evs]
+    t_op = [ev[1].elapsed_time(ev[2]) for ev in evs]
+    t_out = [ev[2].elapsed_time(ev[3]) for ev in evs]
     k_in, k_op, k_out = (float(np.median(t)) for t in (t_in, t_op, t_out))
 
     ms_per_step = elapsed_ms / steps
@@ -868,7 +868,8 @@ def run_layer(args, wl, gla, dev, dist, world, rank, local):
                          "peak_kind": peak_kind + " sustained bf16",
                          "traffic": None, "alg_flops_per_launch": flops_in, "ms_per_launch": k_in},
             "stages_ms": {"project_in": k_in, "gla_forward": k_op, "project_out": k_out,
-                          "how": "events around each of the three calls, per step, median"},
+                          "how": "events around each of the three calls, steps back to back, "
+                                 "median"},
             "stages_tflops": {"project_in": in_tf,
                               "project_out": flops_out / (k_out * 1e-3) / 1e12},
             "e2e": None,
