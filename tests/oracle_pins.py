@@ -440,6 +440,21 @@ def check_anchor_matches_library_sdpa():
     _close(r["attn"], lib.numpy().transpose(0, 2, 1, 3), 1e-12, "anchor vs torch SDPA")
 
 
+def check_anchor_time_shift_invariance():
+    """RoPE makes q_til . k_til depend on position differences only, so a
+    global time offset t0 leaves the anchor's output unchanged (both q and k
+    rotated the same way, by the same positions)."""
+    rng = np.random.default_rng(12)
+    T, H, W, d, Hh = 3, 2, 2, 16, 2
+    N = T * H * W
+    q, k, v, g = (rng.standard_normal((1, N, Hh, d)) for _ in range(4))
+    a = O.softmax_anchor(q, k, v, g, T, H, W, 1e4, t0=0)["out"]
+    b = O.softmax_anchor(q, k, v, g, T, H, W, 1e4, t0=7)["out"]
+    _close(b, a, 1e-11, "anchor under a time shift")
+    c = O.softmax_anchor(q, k, v, g, T, H, W, 0.0, t0=0)["out"]
+    assert np.max(np.abs(c - a)) > 1e-3, "RoPE must change the anchor's output"
+
+
 def check_anchor_uniform_scores():
     """q = 0 gives q_hat = 0 and all scores 0: every token reads the mean of v."""
     rng = np.random.default_rng(10)

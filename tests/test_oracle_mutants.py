@@ -154,6 +154,15 @@ def _anchor_gate_inside(q, k, v, g, T, H, W, rope_theta, t0=0, queries=None):
     return r
 
 
+def _anchor_k_rotated_backwards(q, k, v, g, T, H, W, rope_theta, t0=0, queries=None):
+    ang = O.rope_angles(q.shape[-1], T, H, W, rope_theta, t0) if rope_theta > 0 else None
+    if ang is None:
+        return _orig["softmax_anchor"](q, k, v, g, T, H, W, rope_theta, t0, queries)
+    qt = O.rope_rotate(O.rms_normalize(q), ang)
+    kt = O.rope_rotate(O.rms_normalize(k), -ang)
+    return _orig["softmax_anchor"](qt, kt, v, g, T, H, W, 0.0, t0, queries)
+
+
 def _anchor_softmax_over_queries(q, k, v, g, T, H, W, rope_theta, t0=0, queries=None):
     return _orig["softmax_anchor"](k, q, v, g, T, H, W, rope_theta, t0, queries)
 
@@ -206,6 +215,7 @@ MUTANTS = {
     "project_out_channel_major": ("project_out", _project_out_transposed),
     "anchor_gate_on_values": ("softmax_anchor", _anchor_gate_inside),
     "anchor_q_k_swapped": ("softmax_anchor", _anchor_softmax_over_queries),
+    "anchor_k_rotated_backwards": ("softmax_anchor", _anchor_k_rotated_backwards),
     "e4m3_bias8": ("e4m3_decode", _e4m3_bias8),
     "e4m3_no_subnormals": ("e4m3_decode", _e4m3_no_subnormals),
     "e8m0_bias128": ("e8m0_decode", _e8m0_bias128),
