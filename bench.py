@@ -15,6 +15,13 @@ extra flush is done.
 
 --impl reference times the fp64 CPU oracle (oracle/gla_oracle.py) as it
 stands, on the host cores, on a bounded sample of the same workload per step.
+
+--variant causal | mx | layer | anchor times the other entry points on the
+workload's shape (token-level causal read-out from a zero state, FP8 inputs,
+projection + operator + W_o, the gated softmax anchor), each with its own
+metric and roofline kernel; --workload blk runs the block-causal sequence.
+--profile runs warm-up + steps only (for ncu); --ingest-ncu turns an ncu raw
+export into profiles/traffic.json entries.
 """
 import argparse
 import hashlib
