@@ -324,9 +324,13 @@ GLA_API gla_status gla_layer_forward(const void* x, const void* W_in, const void
  * device buffers (16-byte aligned), N = T*H*W in raster order; head_dim 128
  * (GLA_ERR_UNSUPPORTED otherwise); rope_theta <= 0 turns the rotation off.
  * Scores are taken on the tensor cores from fp16 q_til, k_til (fp32
- * accumulate), the softmax weights are rounded to bf16 for P*V, and the
- * row sums add those rounded weights in fp32.  Errors: GLA_ERR_INVALID_ARG for bad sizes or
- * pointers, GLA_ERR_WORKSPACE for a short or misaligned workspace (256-byte
+ * accumulate); the exponentials need no shift by the row maximum, because
+ * the normalisation bounds every score by sqrt(head_dim); the softmax
+ * weights are rounded to bf16 for P*V and the row sums add those rounded
+ * weights in fp32.  batch * heads <= 65535.  The caller owns every buffer;
+ * the call is asynchronous on `stream`.  Errors: GLA_ERR_INVALID_ARG for bad
+ * sizes or pointers, GLA_ERR_UNSUPPORTED for head_dim != 128 or too many
+ * heads, GLA_ERR_WORKSPACE for a short or misaligned workspace (256-byte
  * aligned), GLA_ERR_CUDA for a failed launch. */
 
 /* Workspace bytes of gla_softmax_anchor (fp16 q_til and k_til), 0 for
