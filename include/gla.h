@@ -282,7 +282,12 @@ GLA_API gla_status gla_forward_mx_ex(const void* q, const void* q_scale, const v
  * heads*head_dim), times W_o.  The pages print no input projection; here q, k,
  * v, g and the beta logits are one linear map of the layer input x, and beta is
  * the sigmoid of its logits.  All matrices are bf16, row-major, device memory,
- * 16-byte aligned; products accumulate in fp32 on the tensor cores (tcgen05). */
+ * 16-byte aligned, owned by the caller; products accumulate in fp32 on the
+ * tensor cores (tcgen05).  Every call is asynchronous on `stream` and checks
+ * its arguments before any launch: GLA_ERR_INVALID_ARG for non-positive or
+ * unaligned sizes and null or misaligned pointers, GLA_ERR_UNSUPPORTED for
+ * widths the kernels do not take (stated per call), GLA_ERR_WORKSPACE for a
+ * short or misaligned workspace, GLA_ERR_CUDA for a failed launch. */
 
 /* C [M][N] = A [M][K] B[N][K]^T, bf16 out (rounded to nearest even).  K and N
  * multiples of 8 (16-byte rows). */
