@@ -311,7 +311,9 @@ GLA_API size_t gla_layer_workspace_size(int batch, int heads, int head_dim, int 
 /* y [batch*N][C_out] = W_o applied to gla_forward of the projections of x
  * [batch*N][C]: gla_project_in, gla_forward, gla_gemm_bf16, each kernel a
  * programmatic dependent of the one before.  W_in [4*heads*head_dim +
- * heads][C], W_o [C_out][heads*head_dim]. */
+ * heads][C], W_o [C_out][heads*head_dim]; C and C_out multiples of 8 and
+ * heads*head_dim of 32 (GLA_ERR_UNSUPPORTED otherwise); rope_theta and eps as
+ * for gla_forward. */
 GLA_API gla_status gla_layer_forward(const void* x, const void* W_in, const void* W_o, int batch,
                                      int C, int C_out, int heads, int head_dim, int T, int H,
                                      int W, float rope_theta, float eps, void* y,
